@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark of the ARCHead packed LM-head forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2|3|4|5] [--T T] [--impl ours|reference]
+
+One step = one forward call of the packed head over one batch of seeded
+synthetic hidden states (the whole hot path: low-rank prologue, the
+vocabulary pass with its fused epilogue).  The default workload is the
+Qwen3-8B-shaped head (V=151,936, d=4,096, core rank 512, INT4 group 128,
+correction rank 64) decoding one token, with fp32 logits and argmax out.
+The packed head (382 MB) is larger than L2 (126 MB), so every step streams
+it from HBM; no L2 flush is needed between steps.
+
+Multi-GPU: one process per GPU under torchrun; each rank serves its own batch
+with its own copy of the head (replicas, no collective on the data path).
+Timing is on the device with CUDA events, max over ranks.
+
+--impl reference times the CPU oracle (float64 numpy) on the host cores, on a
+bounded sample of vocabulary rows, scaled to the full head.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import archead_inputs as gen  # noqa: E402
+
+METRIC = "packed LM-head tokens/s & µs/call at V=151936,d=4096; % HBM or MMA roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+OPS = {  # config -> what one call produces
+    2: dict(logits=True, argmax=True, lse=False, ce=False),
+    3: dict(logits=False, argmax=True, lse=True, ce=False),
+    4: dict(logits=False, argmax=True, lse=True, ce=True),
+    5: dict(logits=False, argmax=True, lse=True, ce=True),
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(OPS))
+    ap.add_argument("--T", type=int, default=None, help="override the token count of the config")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def workload(cfg, T):
+    wl = gen.WORKLOADS[cfg]
+    T = wl.T if T is None else T
+    return wl, T
+
+
+def row_bytes(shape):
+    V, d, r_c, r_r, g, g_B = shape
+    return 5 * r_c / 8 + 2 + d / 2 + 2 * d / g + r_r + 2
+
+
+def algorithmic(shape, T, op):
+    """Bytes and flops of one forward call (the method's own work, no dense head)."""
+    V, d, r_c, r_r, g, g_B = shape
+    head = V * row_bytes(shape) + r_c * (d + 2) + r_r * (d + 2 * d / g_B)
+    io = 2 * T * d + (4 * T * V if op["logits"] else 0) + 4 * T * (op["argmax"] + op["lse"] + op["ce"])
+    flops = 2 * T * V * (d + r_c + r_r) + 2 * T * d * (r_c + r_r)
+    return head + io, flops
+
+
+def vocab_pass_bytes_per_launch(shape, nt, op, Kz):
+    """Algorithmic bytes of one vocabulary-pass launch covering nt tokens: the
+    per-row packed payload (V x row_bytes) + h and z of those tokens + outputs."""
+    V, d = shape[0], shape[1]
+    return (V * row_bytes(shape) + 2 * nt * d + 4 * nt * Kz + (4 * nt * V if op["logits"] else 0)
+            + 4 * nt * (op["argmax"] + op["lse"] + op["ce"]))
+
+
+def source_hash():
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "quantized_output_head_b200", "csrc")
+    for f in sorted(os.listdir(cs)):
+        h.update(open(os.path.join(cs, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(cfg, T):
+    """dram bytes per vocabulary-pass launch from the committed ncu summary, if
+    it was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"decode_kernel_cfg{cfg}_T{T}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*(\d+)", txt)
+    s = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
+    if not m or not s or s.group(1) != source_hash():
+        return None
+    return int(m.group(1))
+
+
+class ClockSampler:
+    """SM clock and throttle reasons from NVML, sampled in a thread."""
+
+    def __init__(self, index, period=0.005):
+        self.samples, self.max_mhz, self.err = [], None, None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report no clocks
+            self._nv, self.err = None, repr(e)
+        self._period = period
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((mhz, rs))
+            except Exception as e:
+                self.err = repr(e)
+                return
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "note": self.err}
+        nv = self._nv
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        seen = sorted({n for _, rs in self.samples for n, bit in names.items() if rs & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": seen, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- reference
+def run_reference(args, cfg, wl, T):
+    """The CPU oracle as it stands, timed on a bounded sample of vocabulary rows."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    shape = wl.shape
+    sh = (shape.V, shape.d, shape.r_c, shape.r_r, shape.g, shape.g_B)
+    comps = gen.draw_components(shape, wl.head_seed_cfg)
+    h_bits, targets = gen.draw_activations(shape.d, T, shape.V, cfg)
+    rows = np.arange(min(shape.V, 8192))
+    for _ in range(args.warmup):
+        oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
+    dt = (time.perf_counter() - t0) / args.steps
+    per_call = dt * shape.V / rows.size
+    value = T / per_call
+    sample = f"{rows.size} of {shape.V} vocabulary rows x {T} tokens per step, scaled to the full head"
+    return dict(impl="reference", metric=METRIC, value=value, unit="tokens/s", n_gpus=args.gpus,
+                steps=args.steps, warmup=args.warmup, ms_per_step=per_call * 1e3, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(workload=wl.name, V=shape.V, d=shape.d, r_c=shape.r_c, r_r=shape.r_r, g=shape.g,
+                            g_B=shape.g_B, T=T),
+                cpu_baseline=dict(kind="oracle", value=value, unit="tokens/s", cores=cores, sample=sample),
+                e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0),
+                algorithmic=dict(zip(("bytes", "flops"), algorithmic(sh, T, OPS[cfg]))))
+
+
+def cpu_baseline(cfg, wl, T, comps, h_bits):
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    shape = wl.shape
+    n_rows = min(shape.V, 32768)
+    rows = np.arange(n_rows)
+    t0 = time.perf_counter()
+    oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
+    dt = time.perf_counter() - t0
+    per_call = dt * shape.V / n_rows
+    return dict(value=T / per_call, unit="tokens/s", cores=cores, kind="oracle",
+                sample=f"oracle on {n_rows} of {shape.V} vocabulary rows for {T} token(s), "
+                       f"{dt:.1f} s, scaled to the full head")
+
+
+# -------------------------------------------------------------------- ours
+def main():
+    args = parse_args()
+    cfg = args.config
+    wl, T = workload(cfg, args.T)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg, wl, T)))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    import datetime
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    import quantized_output_head_b200 as qoh
+
+    shape = wl.shape
+    sh = (shape.V, shape.d, shape.r_c, shape.r_r, shape.g, shape.g_B)
+    op = OPS[cfg]
+    comps = gen.draw_components(shape, wl.head_seed_cfg)
+    h_bits, targets = gen.draw_activations(shape.d, T, shape.V, cfg)
+    head = qoh.PackedHead(*sh, comps)
+    dev = head.device
+    hd = torch.from_numpy(h_bits.view(np.int16)).to(dev)
+    td = torch.from_numpy(targets).to(dev)
+    logits = torch.empty((T, shape.V), dtype=torch.float32, device=dev) if op["logits"] else None
+    am = torch.empty(T, dtype=torch.int32, device=dev)
+    lse = torch.empty(T, dtype=torch.float32, device=dev)
+    ce = torch.empty(T, dtype=torch.float32, device=dev) if op["ce"] else None
+    ws = head.workspace(T)
+
+    def step():
+        if op["logits"]:
+            head.logits_into(hd, logits, am, ws)
+        else:
+            head.lse_argmax_into(hd, td if op["ce"] else None, lse, am, ce, ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    # Timed region: K steps on the device, bracketed by barrier + synchronize.
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record()
+        for _ in range(args.steps):
+            step()
+        ev1.record()
+        torch.cuda.synchronize()
+        barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * T * args.steps / (ms / 1e3)
+
+    # Dominant kernel (the vocabulary pass): CUDA events around it, recorded on
+    # the call's stream by the library, over a second timed loop.
+    n_launch = math.ceil(T / 8)
+    kb, ka = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    head.set_profile_events(kb, ka)
+    k_steps = max(10, min(args.steps, 2000))
+    tot = 0.0
+    for _ in range(k_steps):
+        step()
+        ka.synchronize()
+        tot += kb.elapsed_time(ka)
+    head.set_profile_events(None, None)
+    kernel_ms = tot / k_steps / n_launch
+    hbm, bf16, peak_src = peaks()
+    Kz = -(-shape.r_c // 64) * 64 + -(-shape.r_r // 32) * 32
+    nt = min(T, 8)
+    kbytes = vocab_pass_bytes_per_launch(sh, nt, op, Kz)
+    achieved = kbytes / (kernel_ms / 1e3) / 1e9
+    traffic = recorded_traffic(cfg, T)
+    status = head.status(ws)
+
+    out = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(cfg, wl, T, comps, h_bits)
+        e2e = None
+        if not args.no_e2e:
+            hh = torch.from_numpy(h_bits.view(np.int16)).pin_memory().numpy().view(np.uint16)
+            th = torch.from_numpy(targets).pin_memory().numpy()
+            outs = (torch.empty(T, dtype=torch.float32).pin_memory().numpy(),
+                    torch.empty(T, dtype=torch.int32).pin_memory().numpy(),
+                    torch.empty(T, dtype=torch.float32).pin_memory().numpy())
+            for _ in range(3):
+                head.lse_argmax_host(hh, th, outs)
+            e_steps = max(10, min(args.steps, 2000))
+            t0 = time.perf_counter()
+            for _ in range(e_steps):
+                head.lse_argmax_host(hh, th, outs)
+            e_dt = (time.perf_counter() - t0) / e_steps
+            e2e = dict(value=T / e_dt, unit="tokens/s", h2d_bytes_per_step=T * shape.d * 2 + 4 * T,
+                       d2h_bytes_per_step=12 * T, us_per_call=e_dt * 1e6,
+                       call="archead_lse_argmax_host (host buffers, lse+argmax+ce)")
+        ab, af = algorithmic(sh, T, op)
+        out = dict(
+            metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+            ms_per_step=ms_per_step, us_per_call=ms_per_step * 1e3, higher_is_better=True, scaling="weak",
+            vs_baseline=None, dtype="bf16 MMA on exact int4/int5/int8 codes, fp32 accumulate",
+            data="synthetic (seeded, shapes of the pages' heads)",
+            config=dict(workload=wl.name, V=shape.V, d=shape.d, r_c=shape.r_c, r_r=shape.r_r, g=shape.g,
+                        g_B=shape.g_B, T=T, outputs=[k for k, v in op.items() if v],
+                        parallelism=f"replicas x{world}", l2="inputs larger than L2 (packed head 382 MB)"),
+            roofline=dict(bound="hbm", achieved=achieved, peak=hbm, unit="GB/s", frac=achieved / hbm,
+                          traffic=traffic, kernel="archead::decode_kernel", kernel_us=kernel_ms * 1e3,
+                          algorithmic_bytes_per_launch=kbytes, peak_source=peak_src),
+            call=dict(algorithmic_bytes=ab, algorithmic_flops=af, gbs=ab / (ms_per_step / 1e3) / 1e9,
+                      hbm_frac=ab / (ms_per_step / 1e3) / 1e9 / hbm),
+            cpu_baseline=cpu, e2e=e2e, clocks=clk.summary(),
+            gpu_launches=args.steps * (1 + n_launch), device_status=status,
+        )
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,188 @@
+/*
+ * archead.h -- C ABI of the B200 (sm_100a) library for the forward pass of an
+ * ARCHead packed LM-head.
+ *
+ * Source: "ARCHead: Activation-Metric Residual Correction for Large Language
+ * Model Output Heads" (arXiv 2608.02703).
+ *   §3.2 Eq. 3   W_d   = Q5(A_c) Q8(B_c) + Q_SC4(W - A_c B_c)   quantised core
+ *   §3.2 Eq. 6   W_hat = W_d + A_w B_w                           with INT8 A_w, B_w
+ *   §3.2 Eq. 7   Y_hat = H W_d^T + (H B_w^T) A_w^T               factored forward
+ *   §3.3         the module registers only the packed tensors and shape metadata;
+ *                the dense head is discarded after conversion.
+ *
+ * In this library's names:
+ *   L  [V, r_c]  INT5 codes of Q5(A_c), one fp16 scale per row     s_L [V]
+ *   R  [r_c, d]  INT8 codes of Q8(B_c), one fp16 scale per row     s_R [r_c]
+ *   q  [V, d]    signed INT4 residual codes (SC4)                  s_res [V, d/g]
+ *   A  [V, r_r]  INT8 codes of A_w, one fp16 scale per row         s_A [V]
+ *   B  [r_r, d]  INT8 codes of B_w, one fp16 scale per d-group     s_B [r_r, d/g_B]
+ * and for hidden states h [T, d] (bf16) the logits are
+ *   y[t,v] = s_L[v] sum_k L[v,k] z_c[t,k] + sum_j s_res[v,j/g] q[v,j] h[t,j]
+ *          + s_A[v] sum_k A[v,k] z_r[t,k],
+ *   z_c[t,k] = s_R[k] sum_j R[k,j] h[t,j],  z_r[t,k] = sum_j s_B[k,j/g_B] B[k,j] h[t,j].
+ * The dense V x d head is never formed on the device.
+ *
+ * Conventions for every call
+ *   - Return value: ARCHEAD_OK (0) or a negative ARCHEAD_E* code.  No C++
+ *     exception crosses this boundary.
+ *   - Device pointers are plain CUDA device addresses owned by the caller; the
+ *     library allocates no device memory.  Host pointers are only read during
+ *     the call (or, for the *_host entry point, until it returns).
+ *   - Forward calls are asynchronous on the given stream and never synchronise
+ *     the host (except archead_lse_argmax_host, which is the host-buffer form).
+ *     A fault inside a kernel surfaces at the caller's next synchronisation.
+ *   - Alignment: arena and workspace 256 bytes, hidden 16 bytes, every other
+ *     device buffer 4 bytes; otherwise ARCHEAD_EALIGN.
+ *   - The kernels are built for sm_100a only; pack_load returns ARCHEAD_EUNSUP
+ *     on any other device.
+ */
+#ifndef ARCHEAD_H
+#define ARCHEAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ARCHEAD_API __attribute__((visibility("default")))
+
+typedef struct CUstream_st* archead_stream_t; /* == cudaStream_t; NULL = legacy default stream */
+
+enum {
+  ARCHEAD_OK = 0,
+  ARCHEAD_EINVAL = -1,   /* null pointer, bad shape, T <= 0, code out of range, bad scale */
+  ARCHEAD_EALIGN = -2,   /* a pointer is not aligned as required */
+  ARCHEAD_EUNSUP = -3,   /* shape or device the compiled kernels do not support */
+  ARCHEAD_ECUDA = -4,    /* a CUDA runtime call failed: see archead_last_cuda_error() */
+  ARCHEAD_ENOMEM = -5,   /* a host allocation failed, or a caller buffer is too small */
+  ARCHEAD_ETIMEOUT = -6  /* a bounded device-side wait expired (read back by archead_workspace_status) */
+};
+
+/* Device-side status bits written into the workspace by the kernels. */
+enum {
+  ARCHEAD_STATUS_WAIT_TIMEOUT = 1, /* a pipeline wait gave up; that call's outputs are invalid */
+  ARCHEAD_STATUS_BAD_TARGET = 2    /* a target id was outside [0, V); its CE is NaN */
+};
+
+/* Shape metadata of one packed head (§3.3: "group size and shape metadata").
+ * Supported: V >= 1; d a positive multiple of 64; g a power of two >= 16
+ * dividing d; g_B >= 1 dividing d; r_c >= 0; r_r >= 0. */
+typedef struct archead_desc {
+  int32_t V, d, r_c, r_r, g, g_B;
+} archead_desc;
+
+/* Canonical packed components in host memory, row-major, one code per int8
+ * element holding the two's-complement value; scales are IEEE fp16 bit
+ * patterns.  Ranges: L in [-16,15], q in [-8,7], R / A / B in [-128,127].
+ * The list is the state-dict component list of §3.3. */
+typedef struct archead_host_components {
+  const int8_t* L;   const uint16_t* s_L;    /* [V, r_c],  [V]          */
+  const int8_t* R;   const uint16_t* s_R;    /* [r_c, d],  [r_c]        */
+  const int8_t* q;   const uint16_t* s_res;  /* [V, d],    [V, d/g]     */
+  const int8_t* A;   const uint16_t* s_A;    /* [V, r_r],  [V]          */
+  const int8_t* B;   const uint16_t* s_B;    /* [r_r, d],  [r_r, d/g_B] */
+} archead_host_components;
+
+typedef struct archead_handle archead_handle;
+
+/* §3.3 Eq. 10: bytes(ARCHead) = sum_i numel(theta_i) * element_size(theta_i)
+ * over the registered components, with INT5 and INT4 codes at 5 and 4 bits:
+ *   V(5 r_c/8 + 2 + d/2 + 2d/g + r_r + 2) + r_c(d + 2) + r_r(d + 2d/g_B).
+ * Returns 0 for an unsupported or null desc. */
+ARCHEAD_API size_t archead_packed_bytes(const archead_desc* desc);
+
+/* Device bytes the packed arena needs: the Eq. 10 payload in the kernels'
+ * tile layout plus padding (vocabulary rounded up to 16 rows, r_c to 64,
+ * r_r to 32, segments to 16 and regions to 256 bytes).  0 if unsupported. */
+ARCHEAD_API size_t archead_arena_bytes(const archead_desc* desc);
+
+/* Validate the components, re-lay them out for the kernels and copy them into
+ * the caller-owned device arena (>= archead_arena_bytes, 256-byte aligned, on
+ * the current device).  This is the conversion step of §3.3: afterwards the
+ * arena is immutable and the host arrays may be freed.  Synchronises `stream`
+ * before returning (the host staging buffer is released).  On success *out is
+ * a new host-side handle that points into the arena without owning it; free it
+ * with archead_free.  Codes out of range, or inf / NaN scales: ARCHEAD_EINVAL. */
+ARCHEAD_API int archead_pack_load(const archead_desc* desc, const archead_host_components* comps,
+                                  void* dev_arena, size_t arena_bytes, archead_stream_t stream,
+                                  archead_handle** out);
+
+/* Host-side form of the conversion: validate the components and write the
+ * arena image (the exact bytes archead_pack_load copies to the device) into
+ * host memory of >= archead_arena_bytes bytes.  The image can be stored and
+ * later copied into an arena as is; it is position independent.  Same error
+ * codes as archead_pack_load; no CUDA call is made. */
+ARCHEAD_API int archead_pack_image(const archead_desc* desc, const archead_host_components* comps,
+                                   void* host_image, size_t image_bytes);
+
+/* Workspace bytes one forward call with T tokens needs (256-byte aligned
+ * scratch, caller-owned; reused across calls on one stream).  Holds the
+ * low-rank prologue output z, per-block log-sum-exp partials, a completion
+ * counter and the status word.  Zero-fill a workspace once before its first
+ * use (the status word is sticky); afterwards the calls keep it consistent.
+ * Calls that share a workspace must be ordered (same stream).  0 if handle is
+ * null or T <= 0. */
+ARCHEAD_API size_t archead_workspace_bytes(const archead_handle* handle, int32_t T);
+
+/* Logits of Eq. 7 for T tokens.
+ *   hidden   [T, d] bf16 bit patterns, row-major, device.
+ *   logits   [T, V] fp32, row-major, device; may be NULL.
+ *   argmax   [T] int32, device, lowest index of the row maximum; may be NULL.
+ * At least one of logits / argmax must be non-NULL. */
+ARCHEAD_API int archead_logits(const archead_handle* handle, const uint16_t* hidden, int32_t T,
+                               float* logits, int32_t* argmax,
+                               void* workspace, size_t workspace_bytes, archead_stream_t stream);
+
+/* Fused vocabulary-wide epilogue (the head feeds softmax directly, §1): per
+ * token, without writing the [T, V] logits,
+ *   lse[t]    = log sum_v exp(y[t,v])                    fp32, device, required
+ *   argmax[t] = lowest v attaining max_v y[t,v]          int32, device, required
+ *   ce[t]     = lse[t] - y[t, targets[t]]                fp32, device; NULL to skip
+ * targets [T] int32 in [0, V), device; required when ce is non-NULL.  A
+ * target outside [0, V) gives ce = NaN and sets ARCHEAD_STATUS_BAD_TARGET.
+ * log_softmax(y)[t,v] = y[t,v] - lse[t]. */
+ARCHEAD_API int archead_logits_lse_argmax(const archead_handle* handle, const uint16_t* hidden,
+                                          int32_t T, const int32_t* targets, float* lse,
+                                          int32_t* argmax, float* ce, void* workspace,
+                                          size_t workspace_bytes, archead_stream_t stream);
+
+/* Host-buffer form of archead_logits_lse_argmax: hidden [T, d] and targets [T]
+ * are HOST pointers (pinned memory recommended), copied to the device inside
+ * the workspace; lse / argmax / ce are HOST pointers filled before return.
+ * workspace must be >= archead_host_workspace_bytes(handle, T).  Synchronises
+ * the stream. */
+ARCHEAD_API size_t archead_host_workspace_bytes(const archead_handle* handle, int32_t T);
+ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint16_t* hidden_host,
+                                        int32_t T, const int32_t* targets_host, float* lse_host,
+                                        int32_t* argmax_host, float* ce_host, void* workspace,
+                                        size_t workspace_bytes, archead_stream_t stream);
+
+/* Read (and with clear != 0, reset) the device status word of a workspace:
+ * a bitwise OR of ARCHEAD_STATUS_* since the last clear.  Synchronises the
+ * stream.  Returns ARCHEAD_ETIMEOUT if ARCHEAD_STATUS_WAIT_TIMEOUT is set. */
+ARCHEAD_API int archead_workspace_status(void* workspace, int clear, archead_stream_t stream,
+                                         uint32_t* status_out);
+
+/* Optional profiling hook: when both are non-NULL (cudaEvent_t handles), every
+ * later forward call on this handle records `before` on its stream just before
+ * the first vocabulary-pass launch and `after` just after the last one, so
+ * cudaEventElapsedTime(before, after) is the device time of the vocabulary
+ * pass alone (the low-rank prologue excluded).  NULL, NULL switches it off. */
+ARCHEAD_API int archead_set_profile_events(archead_handle* handle, void* before, void* after);
+
+/* Free a handle (host memory only; the arena stays with the caller). */
+ARCHEAD_API void archead_free(archead_handle* handle);
+
+/* The last cudaError_t seen by a call that returned ARCHEAD_ECUDA (thread-local). */
+ARCHEAD_API int archead_last_cuda_error(void);
+
+/* Static text for a status code. */
+ARCHEAD_API const char* archead_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARCHEAD_H */

@@ -1,0 +1,233 @@
+// Forward entry points of the C ABI (include/archead.h): argument checks,
+// workspace carving, and the launch sequence
+//   prologue (z_c, z_r)  ->  decode launches of <= 8 tokens each
+// on the caller's stream, with no host synchronisation.
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "handle.h"
+
+namespace archead {
+
+namespace {
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxTokens = 1 << 20;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_device(const archead_handle* h) {
+  int dev = -1;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  return dev == h->device ? ARCHEAD_OK : ARCHEAD_EINVAL;
+}
+
+int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const int32_t* targets, float* logits,
+            int32_t* argmax, float* lse, float* ce, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (h == nullptr || hidden == nullptr || ws == nullptr) return ARCHEAD_EINVAL;
+  if (T <= 0 || T > kMaxTokens) return ARCHEAD_EINVAL;
+  if (logits == nullptr && argmax == nullptr && lse == nullptr) return ARCHEAD_EINVAL;
+  if (ce != nullptr && targets == nullptr) return ARCHEAD_EINVAL;
+  if (!aligned(hidden, 16) || !aligned(ws, 256)) return ARCHEAD_EALIGN;
+  if (!aligned(logits, 4) || !aligned(argmax, 4) || !aligned(lse, 4) || !aligned(ce, 4) || !aligned(targets, 4))
+    return ARCHEAD_EALIGN;
+  const WsLayout w = ws_layout(*h, T);
+  if (ws_bytes < w.total) return ARCHEAD_ENOMEM;
+  const int dc = check_device(h);
+  if (dc != ARCHEAD_OK) return dc;
+
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  const Layout& L = h->L;
+  uint32_t* counter = reinterpret_cast<uint32_t*>(wb + w.counter);
+  uint32_t* status = reinterpret_cast<uint32_t*>(wb + w.status);
+  uint16_t* zhi = reinterpret_cast<uint16_t*>(wb + w.zhi);
+  uint16_t* zlo = reinterpret_cast<uint16_t*>(wb + w.zlo);
+
+  PrologueParams pp{};
+  pp.hidden = hidden;
+  pp.R = reinterpret_cast<const int8_t*>(h->arena + L.off_R);
+  pp.s_R = reinterpret_cast<const uint16_t*>(h->arena + L.off_sR);
+  pp.B = reinterpret_cast<const int8_t*>(h->arena + L.off_B);
+  pp.s_B = reinterpret_cast<const uint16_t*>(h->arena + L.off_sB);
+  pp.targets = targets;
+  pp.zhi = zhi;
+  pp.zlo = zlo;
+  pp.counter = counter;
+  pp.status = status;
+  pp.T = T;
+  pp.d = L.d;
+  pp.rcp = L.rcp;
+  pp.rrp = L.rrp;
+  pp.Kz = L.Kz;
+  pp.g_B = L.g_B;
+  pp.V = L.V;
+  cudaError_t e = launch_prologue(pp, stream);
+  if (e != cudaSuccess) return set_cuda_error(e);
+
+  DecodeParams dp{};
+  dp.mtiles = h->arena;
+  dp.hidden = hidden;
+  dp.zhi = zhi;
+  dp.zlo = zlo;
+  dp.targets = targets;
+  dp.logits = logits;
+  dp.argmax = argmax;
+  dp.lse = lse;
+  dp.ce = ce;
+  dp.partials = reinterpret_cast<float4*>(wb + w.partials);
+  dp.tgt = reinterpret_cast<float*>(wb + w.tgt);
+  dp.counter = counter;
+  dp.status = status;
+  dp.T = T;
+  dp.V = L.V;
+  dp.d = L.d;
+  dp.Kz = L.Kz;
+  dp.rcp = L.rcp;
+  dp.n_res = L.n_res;
+  dp.n_L = L.n_L;
+  dp.n_A = L.n_A;
+  dp.n_mtiles = L.n_mtiles;
+  int lg = 0;
+  while ((1 << lg) < L.g_steps) ++lg;
+  dp.g_steps_log2 = lg;
+  dp.off_res = L.off_res;
+  dp.off_Lnib = L.off_Lnib;
+  dp.off_Lhi = L.off_Lhi;
+  dp.off_A = L.off_A;
+  dp.off_sres = L.off_sres;
+  dp.off_sL = L.off_sL;
+  dp.off_sA = L.off_sA;
+  dp.mblk_bytes = L.mblk_bytes;
+  dp.nw_res = h->nw_res;
+  dp.nw_L = h->nw_L;
+  dp.nw_A = h->nw_A;
+  dp.nw_work = h->nw_work;
+  dp.nw_cons = h->nw_cons;
+  dp.stages = h->stages;
+  if (h->ev_before != nullptr) {
+    e = cudaEventRecord(h->ev_before, stream);
+    if (e != cudaSuccess) return set_cuda_error(e);
+  }
+  for (int t0 = 0; t0 < T; t0 += kDecodeTokens) {
+    dp.t0 = t0;
+    dp.nt = (T - t0 < kDecodeTokens) ? (T - t0) : kDecodeTokens;
+    e = launch_decode(h->cres, dp, h->grid, h->smem, stream);
+    if (e != cudaSuccess) return set_cuda_error(e);
+  }
+  if (h->ev_after != nullptr) {
+    e = cudaEventRecord(h->ev_after, stream);
+    if (e != cudaSuccess) return set_cuda_error(e);
+  }
+  return ARCHEAD_OK;
+}
+
+}  // namespace
+
+int set_cuda_error(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return ARCHEAD_ECUDA;
+}
+
+}  // namespace archead
+
+using namespace archead;
+
+extern "C" ARCHEAD_API size_t archead_workspace_bytes(const archead_handle* handle, int32_t T) {
+  if (handle == nullptr || T <= 0 || T > kMaxTokens) return 0;
+  return ws_layout(*handle, T).total;
+}
+
+extern "C" ARCHEAD_API size_t archead_host_workspace_bytes(const archead_handle* handle, int32_t T) {
+  if (handle == nullptr || T <= 0 || T > kMaxTokens) return 0;
+  return ws_layout(*handle, T).host_total;
+}
+
+extern "C" ARCHEAD_API int archead_logits(const archead_handle* handle, const uint16_t* hidden, int32_t T,
+                                          float* logits, int32_t* argmax, void* workspace, size_t workspace_bytes,
+                                          archead_stream_t stream) {
+  if (logits == nullptr && argmax == nullptr) return ARCHEAD_EINVAL;
+  return forward(handle, hidden, T, nullptr, logits, argmax, nullptr, nullptr, workspace, workspace_bytes,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" ARCHEAD_API int archead_logits_lse_argmax(const archead_handle* handle, const uint16_t* hidden,
+                                                     int32_t T, const int32_t* targets, float* lse,
+                                                     int32_t* argmax, float* ce, void* workspace,
+                                                     size_t workspace_bytes, archead_stream_t stream) {
+  if (lse == nullptr || argmax == nullptr) return ARCHEAD_EINVAL;
+  return forward(handle, hidden, T, targets, nullptr, argmax, lse, ce, workspace, workspace_bytes,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint16_t* hidden_host,
+                                                   int32_t T, const int32_t* targets_host, float* lse_host,
+                                                   int32_t* argmax_host, float* ce_host, void* workspace,
+                                                   size_t workspace_bytes, archead_stream_t stream) {
+  if (handle == nullptr || hidden_host == nullptr || lse_host == nullptr || argmax_host == nullptr ||
+      workspace == nullptr)
+    return ARCHEAD_EINVAL;
+  if (T <= 0 || T > kMaxTokens) return ARCHEAD_EINVAL;
+  if (ce_host != nullptr && targets_host == nullptr) return ARCHEAD_EINVAL;
+  if (!aligned(workspace, 256)) return ARCHEAD_EALIGN;
+  const WsLayout w = ws_layout(*handle, T);
+  if (workspace_bytes < w.host_total) return ARCHEAD_ENOMEM;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(workspace);
+  uint16_t* d_hidden = reinterpret_cast<uint16_t*>(wb + w.h_hidden);
+  int32_t* d_targets = targets_host ? reinterpret_cast<int32_t*>(wb + w.h_targets) : nullptr;
+  float* d_lse = reinterpret_cast<float*>(wb + w.h_lse);
+  int32_t* d_argmax = reinterpret_cast<int32_t*>(wb + w.h_argmax);
+  float* d_ce = ce_host ? reinterpret_cast<float*>(wb + w.h_ce) : nullptr;
+  const size_t t = static_cast<size_t>(T);
+  cudaError_t e = cudaMemcpyAsync(d_hidden, hidden_host, t * handle->L.d * 2, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && d_targets)
+    e = cudaMemcpyAsync(d_targets, targets_host, t * 4, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  const int rc = forward(handle, d_hidden, T, d_targets, nullptr, d_argmax, d_lse, d_ce, workspace, w.total, s);
+  if (rc != ARCHEAD_OK) return rc;
+  e = cudaMemcpyAsync(lse_host, d_lse, t * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(argmax_host, d_argmax, t * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && ce_host) e = cudaMemcpyAsync(ce_host, d_ce, t * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  return ARCHEAD_OK;
+}
+
+extern "C" ARCHEAD_API int archead_workspace_status(void* workspace, int clear, archead_stream_t stream,
+                                                    uint32_t* status_out) {
+  if (workspace == nullptr || status_out == nullptr) return ARCHEAD_EINVAL;
+  if (!aligned(workspace, 256)) return ARCHEAD_EALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* st = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + 4);
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, st, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(st, 0, 4, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  *status_out = v;
+  return (v & ARCHEAD_STATUS_WAIT_TIMEOUT) ? ARCHEAD_ETIMEOUT : ARCHEAD_OK;
+}
+
+extern "C" ARCHEAD_API int archead_set_profile_events(archead_handle* handle, void* before, void* after) {
+  if (handle == nullptr || ((before == nullptr) != (after == nullptr))) return ARCHEAD_EINVAL;
+  handle->ev_before = static_cast<cudaEvent_t>(before);
+  handle->ev_after = static_cast<cudaEvent_t>(after);
+  return ARCHEAD_OK;
+}
+
+extern "C" ARCHEAD_API int archead_last_cuda_error(void) { return g_last_cuda_error; }
+
+extern "C" ARCHEAD_API const char* archead_status_string(int status) {
+  switch (status) {
+    case ARCHEAD_OK: return "ok";
+    case ARCHEAD_EINVAL: return "invalid argument";
+    case ARCHEAD_EALIGN: return "misaligned pointer";
+    case ARCHEAD_EUNSUP: return "unsupported shape or device";
+    case ARCHEAD_ECUDA: return "CUDA runtime error";
+    case ARCHEAD_ENOMEM: return "out of memory or buffer too small";
+    case ARCHEAD_ETIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}

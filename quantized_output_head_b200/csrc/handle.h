@@ -1,0 +1,61 @@
+// Host-side handle of a packed head loaded into a caller-owned device arena.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "layout.h"
+#include "params.h"
+
+struct archead_handle {
+  archead::Layout L;
+  const uint8_t* arena;     // device, not owned
+  int device;
+  int num_sms;
+  int grid;                 // decode blocks (one per SM, at most one per m-tile)
+  int cres;                 // residual chunks per residual warp (kernel instance)
+  int nw_res, nw_L, nw_A, nw_work, nw_cons, stages;
+  size_t smem;              // dynamic shared memory of the decode kernel
+  cudaEvent_t ev_before;    // optional profiling events (not owned)
+  cudaEvent_t ev_after;
+};
+
+namespace archead {
+
+// Workspace regions of one forward call with T tokens.
+struct WsLayout {
+  size_t counter, status, zhi, zlo, partials, tgt, total;
+  // host-buffer form only
+  size_t h_hidden, h_targets, h_lse, h_argmax, h_ce, host_total;
+};
+
+inline WsLayout ws_layout(const archead_handle& h, int T) {
+  WsLayout w{};
+  const size_t t = static_cast<size_t>(T);
+  size_t o = 0;
+  w.counter = 0;
+  w.status = 4;
+  o = 256;
+  w.zhi = o;      o += round_up(t * h.L.Kz * 2, 256);
+  w.zlo = o;      o += round_up(t * h.L.Kz * 2, 256);
+  w.partials = o; o += round_up(t * h.grid * 16, 256);
+  w.tgt = o;      o += round_up(t * 4, 256);
+  w.total = o;
+  w.h_hidden = o;  o += round_up(t * h.L.d * 2, 256);
+  w.h_targets = o; o += round_up(t * 4, 256);
+  w.h_lse = o;     o += round_up(t * 4, 256);
+  w.h_argmax = o;  o += round_up(t * 4, 256);
+  w.h_ce = o;      o += round_up(t * 4, 256);
+  w.host_total = o;
+  return w;
+}
+
+// Kernel launchers and attributes (decode.cu, prologue.cu).
+size_t decode_smem_bytes(int stages, uint32_t mblk_bytes, int nw_work);
+cudaError_t decode_set_attributes(int cres, size_t smem);
+cudaError_t launch_decode(int cres, const DecodeParams& p, int grid, size_t smem, cudaStream_t stream);
+cudaError_t launch_prologue(const PrologueParams& p, cudaStream_t stream);
+
+// Thread-local record of the last CUDA error (api.cu).
+int set_cuda_error(cudaError_t e);
+
+}  // namespace archead

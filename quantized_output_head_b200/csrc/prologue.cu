@@ -1,0 +1,81 @@
+// Low-rank prologue of the factored forward (ARCHead paper, §3.2 Eq. 7 and
+// the same factoring of the core of Eq. 3):
+//   z_c[t,k] = s_R[k] sum_j R[k,j] h[t,j]                k < r_c
+//   z_r[t,k] = sum_j s_B[k, j/g_B] B[k,j] h[t,j]         k < r_r
+// accumulated in fp32 and stored as a bf16 pair (high part, remainder) so the
+// tensor-core pass can consume z at ~16 significant bits.  One warp per output
+// row k (R and B rows are read once per token from L1/L2).  The kernel also
+// resets the decode kernel's completion ticket and checks the target ids.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "device.cuh"
+#include "params.h"
+
+namespace archead {
+
+__global__ void __launch_bounds__(256) prologue_kernel(const PrologueParams p) {
+  // Let the dependent decode grid start streaming the packed head right away;
+  // it waits (griddepcontrol.wait) before it reads anything written here.
+  grid_launch_dependents();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.counter = 0u;
+  if (p.targets != nullptr) {
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < p.T; t += gridDim.x * blockDim.x) {
+      const int v = p.targets[t];
+      if (v < 0 || v >= p.V) atomicOr(p.status, static_cast<uint32_t>(ARCHEAD_STATUS_BAD_TARGET));
+    }
+  }
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p.Kz) return;
+  const bool core = row < p.rcp;
+  const int k = core ? row : row - p.rcp;
+  const int8_t* codes = (core ? p.R : p.B) + static_cast<size_t>(k) * p.d;
+  const int ngB = p.d / p.g_B;
+  const float s_row = core ? __half2float(__ushort_as_half(p.s_R[k])) : 1.f;
+  for (int t = 0; t < p.T; ++t) {
+    const uint16_t* h = p.hidden + static_cast<size_t>(t) * p.d;
+    float acc = 0.f;
+    for (int j = lane * 16; j < p.d; j += 32 * 16) {
+      const int4 cv = *reinterpret_cast<const int4*>(codes + j);
+      const uint4 hv0 = *reinterpret_cast<const uint4*>(h + j);
+      const uint4 hv1 = *reinterpret_cast<const uint4*>(h + j + 8);
+      const int8_t* c8 = reinterpret_cast<const int8_t*>(&cv);
+      const __nv_bfloat16* hb0 = reinterpret_cast<const __nv_bfloat16*>(&hv0);
+      const __nv_bfloat16* hb1 = reinterpret_cast<const __nv_bfloat16*>(&hv1);
+      if (core) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc = fmaf(static_cast<float>(c8[e]), __bfloat162float(hb0[e]), acc);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc = fmaf(static_cast<float>(c8[8 + e]), __bfloat162float(hb1[e]), acc);
+      } else {
+        const uint16_t* sb = p.s_B + static_cast<size_t>(k) * ngB;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float sc = __half2float(__ushort_as_half(sb[(j + e) / p.g_B]));
+          const float hv = e < 8 ? __bfloat162float(hb0[e]) : __bfloat162float(hb1[e - 8]);
+          acc = fmaf(sc * static_cast<float>(c8[e]), hv, acc);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (lane == 0) {
+      const float z = acc * s_row;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(z);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(z - __bfloat162float(hi));
+      p.zhi[static_cast<size_t>(t) * p.Kz + row] = __bfloat16_as_ushort(hi);
+      p.zlo[static_cast<size_t>(t) * p.Kz + row] = __bfloat16_as_ushort(lo);
+    }
+  }
+}
+
+cudaError_t launch_prologue(const PrologueParams& p, cudaStream_t stream) {
+  const int rows_per_block = 8;
+  const int grid = p.Kz > 0 ? (p.Kz + rows_per_block - 1) / rows_per_block : 1;
+  prologue_kernel<<<grid, 32 * rows_per_block, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace archead

@@ -1,0 +1,143 @@
+"""The C-ABI library loads, exports every symbol include/archead.h declares,
+and its host-only logic (byte counts, argument checks) behaves.  No GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "archead.h")
+
+
+def _load_build_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_archead_build", os.path.join(ROOT, "quantized_output_head_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.fixture(scope="module")
+def qoh():
+    _load_build_module().build()
+    import quantized_output_head_b200 as m
+    return m
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ARCHEAD_API\s+[\w\s\*]*?\b(archead_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for must in ("archead_pack_load", "archead_logits", "archead_logits_lse_argmax"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(qoh):
+    names = declared_symbols()
+    lib = ctypes.CDLL(qoh.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", qoh.LIB_PATH], capture_output=True, text=True).stdout
+    exported = sorted(set(re.findall(r"\bT (archead_\w+)", out)))
+    assert exported == names
+    assert sorted(qoh.EXPORTED) == names
+
+
+SHAPES = [
+    (1024, 256, 32, 8, 64, 64),
+    (151936, 4096, 512, 64, 128, 128),
+    (262144, 2560, 384, 64, 128, 128),
+    (1000, 320, 0, 0, 16, 1),
+    (17, 320, 100, 3, 64, 10),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_packed_bytes_matches_oracle(qoh, shape):
+    assert qoh.archead_packed_bytes(*shape) == oracle.packed_bytes(*shape)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_arena_holds_payload(qoh, shape):
+    arena = qoh.archead_arena_bytes(*shape)
+    assert arena >= qoh.archead_packed_bytes(*shape)
+    assert arena % 256 == 0
+
+
+def test_arena_padding_small_at_qwen_shape(qoh):
+    shape = (151936, 4096, 512, 64, 128, 128)
+    assert qoh.archead_arena_bytes(*shape) - qoh.archead_packed_bytes(*shape) < 4096
+
+
+@pytest.mark.parametrize("shape", [
+    (0, 256, 32, 8, 64, 64),      # V < 1
+    (16, 100, 8, 8, 4, 4),        # d not a multiple of 64
+    (16, 256, 8, 8, 48, 64),      # g not a power of two
+    (16, 256, 8, 8, 8, 64),       # g < 16
+    (16, 256, 8, 8, 64, 7),       # g_B does not divide d
+    (16, 256, -1, 8, 64, 64),     # negative rank
+])
+def test_unsupported_shapes_report_zero(qoh, shape):
+    assert qoh.archead_packed_bytes(*shape) == 0
+    assert qoh.archead_arena_bytes(*shape) == 0
+
+
+def _host_components(V, d, r_c, r_r, g, g_B):
+    import archead_inputs as gen
+    return gen.random_components(gen.HeadShape(V, d, r_c, r_r, g, g_B), 5)
+
+
+def _pack_load_raw(qoh, shape, comps, arena_ptr=4096, arena_bytes=1 << 30):
+    desc = qoh.ArcheadDesc(*shape)
+    keep = {k: np.ascontiguousarray(v) for k, v in comps.items()}
+    hc = qoh.ArcheadHostComponents(**{k: v.ctypes.data for k, v in keep.items()})
+    h = ctypes.c_void_p()
+    return qoh._lib.archead_pack_load(ctypes.byref(desc), ctypes.byref(hc), arena_ptr, arena_bytes, None,
+                                      ctypes.byref(h))
+
+
+def test_pack_load_rejects_out_of_range_codes(qoh):
+    shape = (32, 64, 8, 4, 16, 16)
+    c = _host_components(*shape)
+    c["q"][3, 5] = 8                       # INT4 residual range is [-8, 7]
+    assert _pack_load_raw(qoh, shape, c) == qoh.ARCHEAD_EINVAL
+    c = _host_components(*shape)
+    c["L"][0, 0] = -17                     # INT5 core range is [-16, 15]
+    assert _pack_load_raw(qoh, shape, c) == qoh.ARCHEAD_EINVAL
+
+
+def test_pack_load_rejects_non_finite_scales(qoh):
+    shape = (32, 64, 8, 4, 16, 16)
+    c = _host_components(*shape)
+    c["s_res"][1, 1] = 0x7C00              # +inf in fp16
+    assert _pack_load_raw(qoh, shape, c) == qoh.ARCHEAD_EINVAL
+    c = _host_components(*shape)
+    c["s_B"][0, 0] = 0x7E00                # NaN
+    assert _pack_load_raw(qoh, shape, c) == qoh.ARCHEAD_EINVAL
+
+
+def test_pack_load_argument_checks(qoh):
+    shape = (32, 64, 8, 4, 16, 16)
+    c = _host_components(*shape)
+    assert _pack_load_raw(qoh, shape, c, arena_ptr=4096 + 16) == qoh.ARCHEAD_EALIGN
+    assert _pack_load_raw(qoh, shape, c, arena_bytes=16) == qoh.ARCHEAD_ENOMEM
+    assert _pack_load_raw(qoh, (32, 60, 8, 4, 16, 16), c) == qoh.ARCHEAD_EUNSUP
+    assert qoh._lib.archead_pack_load(None, None, None, 0, None, None) == qoh.ARCHEAD_EINVAL
+
+
+def test_forward_rejects_null_handle(qoh):
+    L = qoh._lib
+    assert L.archead_logits(None, 4096, 1, 4096, None, 4096, 1 << 20, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_logits_lse_argmax(None, 4096, 1, None, 4096, 4096, None, 4096, 1 << 20, None) == \
+        qoh.ARCHEAD_EINVAL
+    assert L.archead_workspace_bytes(None, 4) == 0
+    assert L.archead_status_string(qoh.ARCHEAD_EUNSUP) == b"unsupported shape or device"

@@ -1,0 +1,238 @@
+"""GPU parity: the CUDA path against the float64 CPU oracle, element by element.
+
+Every call goes through the C ABI of libarchead.so (via the ctypes binding).
+Inputs are the seeded synthetic workloads of archead_inputs; expected values
+come only from oracle/.  Rules (tests/parity.py): per-logit tolerance
+2e-3 * ||h_t|| * max_j |W_hat[v, j]|, LSE within the row's largest tolerance,
+CE within twice that, argmax exact unless the oracle's gap is within tolerance.
+"""
+import numpy as np
+import pytest
+import torch
+
+import archead_inputs as gen
+import oracle
+from parity import check_argmax, check_lse_ce, check_logits
+
+pytestmark = pytest.mark.gpu
+
+QWEN = (151936, 4096, 512, 64, 128, 128)
+GEMMA = (262144, 2560, 384, 64, 128, 128)
+
+
+@pytest.fixture(scope="module")
+def qoh():
+    import quantized_output_head_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
+def _dev_hidden(h_bits):
+    return torch.from_numpy(h_bits.view(np.int16)).cuda()
+
+
+def _oracle(comps, shape, h_bits):
+    y, rowmax = oracle.logits(comps, shape[4], shape[5], h_bits)
+    return y, oracle.tolerance(h_bits, rowmax)
+
+
+# ------------------------------------------------------------- config 1
+@pytest.fixture(scope="module")
+def cfg1(qoh):
+    W, H, h_bits, targets = gen.dense_head_inputs()
+    built = oracle.build_packed_head(W, H, r_c=32, r_r=8, g=64, g_B=64, p=0.75, lam=1e-2)
+    comps = {k: v for k, v in built.items() if not k.startswith("_")}
+    shape = (1024, 256, 32, 8, 64, 64)
+    head = qoh.PackedHead(*shape, comps)
+    y, tol = _oracle(comps, shape, h_bits)
+    return head, h_bits, targets, y, tol
+
+
+def test_cfg1_logits_and_argmax(cfg1):
+    head, h_bits, _, y, tol = cfg1
+    lg, am = head.logits(_dev_hidden(h_bits))
+    check_logits(lg.cpu().numpy(), y, tol)
+    check_argmax(am.cpu().numpy(), y, tol)
+
+
+def test_cfg1_fused_epilogue(cfg1):
+    head, h_bits, targets, y, tol = cfg1
+    lse, am, ce = head.lse_argmax(_dev_hidden(h_bits), torch.from_numpy(targets))
+    check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, targets)
+    check_argmax(am.cpu().numpy(), y, tol)
+
+
+def test_cfg1_host_buffer_entry_matches_device_entry(cfg1):
+    head, h_bits, targets, y, tol = cfg1
+    lse_d, am_d, ce_d = head.lse_argmax(_dev_hidden(h_bits), torch.from_numpy(targets))
+    lse_h, am_h, ce_h = head.lse_argmax_host(h_bits, targets)
+    assert np.array_equal(lse_h, lse_d.cpu().numpy())
+    assert np.array_equal(am_h, am_d.cpu().numpy())
+    assert np.array_equal(ce_h, ce_d.cpu().numpy())
+
+
+# ------------------------------------------------ Qwen-shaped head (2, 3, 5)
+@pytest.fixture(scope="module")
+def qwen(qoh):
+    shape, _, _, comps = gen.make_workload(2)
+    head = qoh.PackedHead(*shape, comps)
+    h1, t1 = gen.draw_activations(4096, 1, shape[0], 2)
+    h64, t64 = gen.draw_activations(4096, 64, shape[0], 3)
+    h5, t5 = gen.draw_activations(4096, 4096, shape[0], 5)
+    sample5 = np.linspace(0, 4095, 12).astype(int)
+    stacked = np.concatenate([h1, h64, h5[sample5]], axis=0)
+    y, tol = _oracle(comps, QWEN, stacked)
+    return dict(head=head, h1=h1, t1=t1, h64=h64, t64=t64, h5=h5, t5=t5, sample5=sample5,
+                y1=y[:1], tol1=tol[:1], y64=y[1:65], tol64=tol[1:65], y5=y[65:], tol5=tol[65:])
+
+
+def test_qwen_decode_T1_logits_argmax(qwen):
+    head = qwen["head"]
+    lg, am = head.logits(_dev_hidden(qwen["h1"]))
+    check_logits(lg.cpu().numpy(), qwen["y1"], qwen["tol1"])
+    check_argmax(am.cpu().numpy(), qwen["y1"], qwen["tol1"])
+
+
+def test_qwen_decode_T1_fused(qwen):
+    head = qwen["head"]
+    lse, am, ce = head.lse_argmax(_dev_hidden(qwen["h1"]), torch.from_numpy(qwen["t1"]))
+    check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), qwen["y1"], qwen["tol1"], qwen["t1"])
+    check_argmax(am.cpu().numpy(), qwen["y1"], qwen["tol1"])
+
+
+@pytest.mark.parametrize("T", gen.SWEEP_T)
+def test_qwen_decode_sweep_fused(qwen, T):
+    head = qwen["head"]
+    h, tg = qwen["h64"][:T], qwen["t64"][:T]
+    lse, am, ce = head.lse_argmax(_dev_hidden(h), torch.from_numpy(tg))
+    y, tol = qwen["y64"][:T], qwen["tol64"][:T]
+    check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, tg)
+    check_argmax(am.cpu().numpy(), y, tol)
+
+
+def test_qwen_decode_T64_logits(qwen):
+    head = qwen["head"]
+    lg, am = head.logits(_dev_hidden(qwen["h64"]))
+    check_logits(lg.cpu().numpy(), qwen["y64"], qwen["tol64"])
+    check_argmax(am.cpu().numpy(), qwen["y64"], qwen["tol64"])
+
+
+def test_qwen_prefill_T4096_sampled(qwen):
+    """Full 4096-token call; the oracle checks 12 evenly spaced tokens over all V."""
+    head = qwen["head"]
+    lse, am, ce = head.lse_argmax(_dev_hidden(qwen["h5"]), torch.from_numpy(qwen["t5"]))
+    s = qwen["sample5"]
+    lse, am, ce = lse.cpu().numpy()[s], am.cpu().numpy()[s], ce.cpu().numpy()[s]
+    check_lse_ce(lse, ce, qwen["y5"], qwen["tol5"], qwen["t5"][s])
+    check_argmax(am, qwen["y5"], qwen["tol5"])
+
+
+def test_qwen_calls_are_deterministic(qwen):
+    head = qwen["head"]
+    hd = _dev_hidden(qwen["h64"][:8])
+    a = head.lse_argmax(hd)
+    b = head.lse_argmax(hd)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_qwen_status_clean(qwen):
+    head = qwen["head"]
+    head.lse_argmax(_dev_hidden(qwen["h1"]), torch.from_numpy(qwen["t1"]))
+    assert head.status(head.workspace(1)) == 0
+
+
+# ------------------------------------------------------------- config 4
+@pytest.fixture(scope="module")
+def gemma(qoh):
+    shape, h, tg, comps = gen.make_workload(4)
+    head = qoh.PackedHead(*shape, comps)
+    y, tol = _oracle(comps, GEMMA, h)
+    return head, h, tg, y, tol
+
+
+def test_gemma_decode_T16_fused_ce(gemma):
+    head, h, tg, y, tol = gemma
+    lse, am, ce = head.lse_argmax(_dev_hidden(h), torch.from_numpy(tg))
+    check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, tg)
+    check_argmax(am.cpu().numpy(), y, tol)
+
+
+def test_gemma_decode_T16_logits(gemma):
+    head, h, tg, y, tol = gemma
+    lg, am = head.logits(_dev_hidden(h))
+    check_logits(lg.cpu().numpy(), y, tol)
+
+
+# ------------------------------------------------ ragged and edge shapes
+SMALL = [
+    # V,    d,   r_c, r_r, g,   g_B, T
+    (1000, 320, 32, 8, 64, 64, 3),       # ragged vocabulary tail (not a multiple of 16)
+    (1003, 256, 100, 40, 16, 10, 9),     # ragged ranks, g = 16, g_B not a power of two, two launches
+    (16, 64, 0, 0, 64, 1, 1),            # residual only, one m-tile
+    (47, 128, 64, 32, 128, 128, 17),     # three launches of <= 8 tokens
+    (4099, 512, 64, 64, 256, 32, 8),     # group of 256 spans a whole residual warp
+    (2048, 1024, 512, 64, 512, 128, 5),  # group larger than a warp's columns
+]
+
+
+@pytest.mark.parametrize("V,d,r_c,r_r,g,g_B,T", SMALL)
+def test_small_shapes(qoh, V, d, r_c, r_r, g, g_B, T):
+    shape = (V, d, r_c, r_r, g, g_B)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=V + d + T)
+    h_bits, tg = gen.random_hidden(d, T, seed=T + 7, V=V)
+    head = qoh.PackedHead(*shape, comps)
+    y, tol = _oracle(comps, shape, h_bits)
+    lg, am = head.logits(_dev_hidden(h_bits))
+    check_logits(lg.cpu().numpy(), y, tol)
+    check_argmax(am.cpu().numpy(), y, tol)
+    lse, am2, ce = head.lse_argmax(_dev_hidden(h_bits), torch.from_numpy(tg))
+    check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, tg)
+    assert np.array_equal(am.cpu().numpy(), am2.cpu().numpy())
+
+
+def test_zero_residual_and_correction_is_core_product(qoh):
+    shape = (512, 256, 64, 32, 64, 64)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=99)
+    comps["q"][:] = 0
+    comps["A"][:] = 0
+    h_bits, _ = gen.random_hidden(256, 4, seed=98)
+    head = qoh.PackedHead(*shape, comps)
+    lg, _ = head.logits(_dev_hidden(h_bits))
+    h = oracle.bf16_decode(h_bits)
+    Rh = oracle.dequantize(comps["R"], comps["s_R"], None)
+    Lh = oracle.dequantize(comps["L"], comps["s_L"], None)
+    ref = (h @ Rh.T) @ Lh.T
+    _, rowmax = oracle.logits(comps, 64, 64, h_bits)
+    check_logits(lg.cpu().numpy(), ref, oracle.tolerance(h_bits, rowmax))
+
+
+def test_bad_target_gives_nan_and_status(qoh):
+    shape = (64, 64, 16, 8, 16, 16)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=3)
+    head = qoh.PackedHead(*shape, comps)
+    h_bits, _ = gen.random_hidden(64, 2, seed=4)
+    ws = head.workspace(2)
+    head.status(ws, clear=True)
+    lse, am, ce = head.lse_argmax(_dev_hidden(h_bits), torch.tensor([5, 64], dtype=torch.int32))
+    ce = ce.cpu().numpy()
+    assert np.isfinite(ce[0]) and np.isnan(ce[1])
+    assert head.status(ws, clear=True) == qoh.STATUS_BAD_TARGET
+    assert head.status(ws) == 0
+
+
+def test_forward_argument_errors(qoh):
+    shape = (64, 64, 16, 8, 16, 16)
+    head = qoh.PackedHead(*shape, gen.random_components(gen.HeadShape(*shape), seed=5))
+    h = torch.zeros((2, 64), dtype=torch.bfloat16, device="cuda")
+    ws = head.workspace(2)
+    lse = torch.empty(2, device="cuda")
+    am = torch.empty(2, dtype=torch.int32, device="cuda")
+    with pytest.raises(qoh.ArcheadError) as e:
+        head.lse_argmax_into(h[:0], None, lse, am, None, ws)
+    assert e.value.status == qoh.ARCHEAD_EINVAL
+    with pytest.raises(qoh.ArcheadError) as e:
+        head.lse_argmax_into(h, None, lse, am, None, ws[:64])
+    assert e.value.status == qoh.ARCHEAD_ENOMEM
+    with pytest.raises(qoh.ArcheadError) as e:
+        head.lse_argmax_into(h.view(-1)[1:129].view(2, 64), None, lse, am, None, ws)
+    assert e.value.status == qoh.ARCHEAD_EALIGN
