@@ -43,6 +43,9 @@ class HeadShape:
     g: int      # group size of the signed-INT4 residual scales along d
     g_B: int    # group size of the INT8 correction factor B_w along d
 
+    def as_tuple(self):
+        return (self.V, self.d, self.r_c, self.r_r, self.g, self.g_B)
+
 
 @dataclasses.dataclass(frozen=True)
 class Workload:

@@ -304,15 +304,20 @@ def main():
     # Dominant kernel (the vocabulary pass): CUDA events around it, recorded on
     # the call's stream by the library, over a second timed loop.
     n_launch = math.ceil(T / 8)
-    kb, ka = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    head.set_profile_events(kb, ka)
+    from cuda.bindings import runtime as cudart
+    _, kb = cudart.cudaEventCreate()
+    _, ka = cudart.cudaEventCreate()
+    head.set_profile_events(int(kb), int(ka))
     k_steps = max(10, min(args.steps, 2000))
     tot = 0.0
     for _ in range(k_steps):
         step()
-        ka.synchronize()
-        tot += kb.elapsed_time(ka)
+        cudart.cudaEventSynchronize(ka)
+        err, dt = cudart.cudaEventElapsedTime(kb, ka)
+        tot += dt
     head.set_profile_events(None, None)
+    cudart.cudaEventDestroy(kb)
+    cudart.cudaEventDestroy(ka)
     kernel_ms = tot / k_steps / n_launch
     hbm, bf16, peak_src = peaks()
     Kz = -(-shape.r_c // 64) * 64 + -(-shape.r_r // 32) * 32

@@ -229,10 +229,13 @@ class PackedHead:
                "archead_lse_argmax_host")
         return lse, am, ce
 
-    def set_profile_events(self, before: Optional[torch.cuda.Event], after: Optional[torch.cuda.Event]) -> None:
-        """Record `before` / `after` around the vocabulary pass of every later call (None, None: off)."""
-        b = None if before is None else int(before.cuda_event)
-        a = None if after is None else int(after.cuda_event)
+    def set_profile_events(self, before, after) -> None:
+        """Record `before` / `after` (cudaEvent_t handles as ints, or objects with a
+        ``cuda_event`` attribute) around the vocabulary pass of every later call.
+        None, None switches it off."""
+        def raw(e):
+            return None if e is None else int(getattr(e, "cuda_event", e))
+        b, a = raw(before), raw(after)
         _check(_lib.archead_set_profile_events(self.handle, b, a), "archead_set_profile_events")
 
     def status(self, workspace: torch.Tensor, clear: bool = True) -> int:

@@ -75,10 +75,10 @@ def test_cfg1_host_buffer_entry_matches_device_entry(cfg1):
 @pytest.fixture(scope="module")
 def qwen(qoh):
     shape, _, _, comps = gen.make_workload(2)
-    head = qoh.PackedHead(*shape, comps)
-    h1, t1 = gen.draw_activations(4096, 1, shape[0], 2)
-    h64, t64 = gen.draw_activations(4096, 64, shape[0], 3)
-    h5, t5 = gen.draw_activations(4096, 4096, shape[0], 5)
+    head = qoh.PackedHead(*shape.as_tuple(), comps)
+    h1, t1 = gen.draw_activations(4096, 1, shape.V, 2)
+    h64, t64 = gen.draw_activations(4096, 64, shape.V, 3)
+    h5, t5 = gen.draw_activations(4096, 4096, shape.V, 5)
     sample5 = np.linspace(0, 4095, 12).astype(int)
     stacked = np.concatenate([h1, h64, h5[sample5]], axis=0)
     y, tol = _oracle(comps, QWEN, stacked)
@@ -145,7 +145,7 @@ def test_qwen_status_clean(qwen):
 @pytest.fixture(scope="module")
 def gemma(qoh):
     shape, h, tg, comps = gen.make_workload(4)
-    head = qoh.PackedHead(*shape, comps)
+    head = qoh.PackedHead(*shape.as_tuple(), comps)
     y, tol = _oracle(comps, GEMMA, h)
     return head, h, tg, y, tol
 
@@ -167,7 +167,7 @@ def test_gemma_decode_T16_logits(gemma):
 SMALL = [
     # V,    d,   r_c, r_r, g,   g_B, T
     (1000, 320, 32, 8, 64, 64, 3),       # ragged vocabulary tail (not a multiple of 16)
-    (1003, 256, 100, 40, 16, 10, 9),     # ragged ranks, g = 16, g_B not a power of two, two launches
+    (1003, 320, 100, 40, 16, 10, 9),     # ragged ranks, g = 16, g_B not a power of two, two launches
     (16, 64, 0, 0, 64, 1, 1),            # residual only, one m-tile
     (47, 128, 64, 32, 128, 128, 17),     # three launches of <= 8 tokens
     (4099, 512, 64, 64, 256, 32, 8),     # group of 256 spans a whole residual warp
