@@ -94,6 +94,8 @@ def dequantize(codes: np.ndarray, s_bits: np.ndarray, group: Optional[int]) -> n
     """codes [rows, cols] x per-group fp16 scales -> float64 (exact)."""
     codes = np.asarray(codes)
     rows, cols = codes.shape
+    if codes.size == 0:          # a rank-0 factor: the branch is an empty sum
+        return np.zeros((rows, cols))
     s = fp16_decode(s_bits).reshape(rows, -1)
     G = cols if group is None else group
     return codes.astype(np.float64) * np.repeat(s, G, axis=1)

@@ -219,6 +219,18 @@ def test_zero_residual_and_correction_is_core_product():
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-15)
 
 
+def test_rank_zero_branches_are_empty_sums():
+    """r_c = r_r = 0: only the SC4 residual remains (Eq. 3 and Eq. 6 with empty factors)."""
+    comp = gen.random_components(gen.HeadShape(16, 64, 0, 0, 16, 1), 2)
+    h_bits, _ = gen.random_hidden(64, 2, seed=3)
+    y, _ = oracle.logits(comp, 16, 1, h_bits)
+    exact = _exact_logits(comp, h_bits, 16, 1, ("res",))
+    for t in range(2):
+        for v in range(16):
+            e = float(exact[t][v])
+            assert abs(y[t, v] - e) <= 1e-12 * abs(e) + 1e-18
+
+
 def test_factored_equals_dense():
     """Eq. 6 (dense W_hat) and Eq. 7 (factored) give the same logits."""
     comp = gen.random_components(gen.HeadShape(300, 256, 32, 8, 64, 64), 21)
