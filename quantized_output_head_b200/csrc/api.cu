@@ -42,6 +42,7 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   const Layout& L = h->L;
   uint32_t* counter = reinterpret_cast<uint32_t*>(wb + w.counter);
   uint32_t* status = reinterpret_cast<uint32_t*>(wb + w.status);
+  int32_t* escale = reinterpret_cast<int32_t*>(wb + w.escale);
   uint16_t* zhi = reinterpret_cast<uint16_t*>(wb + w.zhi);
   uint16_t* zlo = reinterpret_cast<uint16_t*>(wb + w.zlo);
 
@@ -54,8 +55,10 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   pp.targets = targets;
   pp.zhi = zhi;
   pp.zlo = zlo;
+  pp.escale = escale;
   pp.counter = counter;
   pp.status = status;
+  pp.e_B = h->e_B;
   pp.T = T;
   pp.d = L.d;
   pp.rcp = L.rcp;
@@ -71,6 +74,7 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   dp.hidden = hidden;
   dp.zhi = zhi;
   dp.zlo = zlo;
+  dp.escale = escale;
   dp.targets = targets;
   dp.logits = logits;
   dp.argmax = argmax;
@@ -85,6 +89,7 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   dp.d = L.d;
   dp.Kz = L.Kz;
   dp.rcp = L.rcp;
+  dp.e_B = h->e_B;
   dp.n_res = L.n_res;
   dp.n_L = L.n_L;
   dp.n_A = L.n_A;
@@ -104,8 +109,6 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   dp.nw_L = h->nw_L;
   dp.nw_A = h->nw_A;
   dp.nw_work = h->nw_work;
-  dp.nw_cons = h->nw_cons;
-  dp.stages = h->stages;
   if (h->ev_before != nullptr) {
     e = cudaEventRecord(h->ev_before, stream);
     if (e != cudaSuccess) return set_cuda_error(e);
@@ -113,7 +116,12 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   for (int t0 = 0; t0 < T; t0 += kDecodeTokens) {
     dp.t0 = t0;
     dp.nt = (T - t0 < kDecodeTokens) ? (T - t0) : kDecodeTokens;
-    e = launch_decode(h->cres, dp, h->grid, h->smem, stream);
+    const size_t fixed = decode_smem_bytes(0, L.mblk_bytes, h->nw_work, dp.nt);
+    const size_t per_stage = decode_smem_bytes(1, L.mblk_bytes, h->nw_work, dp.nt) - fixed;
+    int stages = static_cast<int>((static_cast<size_t>(h->smem_optin) - fixed) / per_stage);
+    stages = stages < kMaxStages ? stages : kMaxStages;
+    dp.stages = stages;
+    e = launch_decode(L.g_steps, dp, h->grid, decode_smem_bytes(stages, L.mblk_bytes, h->nw_work, dp.nt), stream);
     if (e != cudaSuccess) return set_cuda_error(e);
   }
   if (h->ev_after != nullptr) {

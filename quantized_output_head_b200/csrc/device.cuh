@@ -1,7 +1,8 @@
 // sm_100a device helpers: mbarriers, bulk copies, dependent-launch control,
-// the m16n8k16 bf16 tensor-core fragment op, and exact code -> bf16 unpacking.
+// the m16n8k16 fp16 tensor-core fragment op, and exact code -> fp16 unpacking.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "layout.h"
@@ -77,10 +78,10 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 }
 
 // ------------------------------------------------------------- tensor core
-// D += A(16x16, row) * B(16x8, col), bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+// D += A(16x16, row) * B(16x8, col), fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -99,58 +100,58 @@ __device__ __forceinline__ uint32_t and_or_r(uint32_t x, uint32_t mask, uint32_t
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(mask), "r"(bits));
   return r;
 }
-// a * 1 + c on bf16 pairs (exact here: the operands are small integers).
-__device__ __forceinline__ uint32_t bf16x2_add_const(uint32_t a, uint32_t c) {
-  uint32_t r;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(0x3F803F80u), "r"(c));
-  return r;
-}
-
-// bf16 bit patterns used below: 0x4300 = 128.0, 0xC308 = -136.0, 0xC310 = -144.0.
-// A nibble u placed under the exponent of 128 gives 128 + u exactly.
-
-// Offset-binary INT4 word (8 codes) -> the four A-fragment registers.
-__device__ __forceinline__ void unpack_int4(uint32_t w, uint32_t (&a)[4]) {
-  a[0] = bf16x2_add_const(and_or<0x000F000Fu, 0x43004300u>(w), 0xC308C308u);
-  a[1] = bf16x2_add_const(and_or<0x000F000Fu, 0x43004300u>(w >> 4), 0xC308C308u);
-  a[2] = bf16x2_add_const(and_or<0x000F000Fu, 0x43004300u>(w >> 8), 0xC308C308u);
-  a[3] = bf16x2_add_const(and_or<0x000F000Fu, 0x43004300u>(w >> 12), 0xC308C308u);
-}
-
 template <int kShift>
 __device__ __forceinline__ uint32_t shift_to(uint32_t x) {
   if constexpr (kShift >= 0) return x >> kShift;
   else return x << (-kShift);
 }
 
-// Offset-binary INT5 codes of k16 step S: low nibbles in w, fifth bits in hb.
-template <int S>
-__device__ __forceinline__ void unpack_int5(uint32_t w, uint32_t hb, uint32_t (&a)[4]) {
-  const uint32_t t0 = and_or<0x000F000Fu, 0x43004300u>(w);
-  const uint32_t t1 = and_or<0x000F000Fu, 0x43004300u>(w >> 4);
-  const uint32_t t2 = and_or<0x000F000Fu, 0x43004300u>(w >> 8);
-  const uint32_t t3 = and_or<0x000F000Fu, 0x43004300u>(w >> 12);
-  a[0] = bf16x2_add_const(and_or_r(shift_to<4 * S + 0 - 4>(hb), 0x00100010u, t0), 0xC310C310u);
-  a[1] = bf16x2_add_const(and_or_r(shift_to<4 * S + 1 - 4>(hb), 0x00100010u, t1), 0xC310C310u);
-  a[2] = bf16x2_add_const(and_or_r(shift_to<4 * S + 2 - 4>(hb), 0x00100010u, t2), 0xC310C310u);
-  a[3] = bf16x2_add_const(and_or_r(shift_to<4 * S + 3 - 4>(hb), 0x00100010u, t3), 0xC310C310u);
+// fp16 fragment unpacking with a bias.  A 4-bit field placed under the fp16
+// exponent of 1024 (0x6400, mantissa step 1 at bit 0) reads as 1024 + u; the
+// same field at bits 4-7 under the exponent of 64 (0x5400, mantissa step 1 at
+// bit 4) reads as 64 + u.  Both are exact, so the tensor core sees
+// (bias + code + offset) and the bias is removed once per scale group in fp32.
+// Per k16 step the A columns 2cc, 2cc+1 (registers a0, a1) carry the 1024 bias
+// and the columns 2cc+8, 2cc+9 (a2, a3) the 64 bias.
+constexpr float kBiasLo = 1024.f;
+constexpr float kBiasHi = 64.f;
+
+// Offset-binary INT4 word: nibbles of (a0, a2, a1, a3) at bits 0, 4, 8, 12 (low
+// columns) and 16, 20, 24, 28 (high columns).
+__device__ __forceinline__ void unpack_int4_biased(uint32_t w, uint32_t (&a)[4]) {
+  const uint32_t w8 = w >> 8;
+  a[0] = and_or<0x000F000Fu, 0x64006400u>(w);
+  a[2] = and_or<0x00F000F0u, 0x54005400u>(w);
+  a[1] = and_or<0x000F000Fu, 0x64006400u>(w8);
+  a[3] = and_or<0x00F000F0u, 0x54005400u>(w8);
 }
 
-// Two offset-binary INT8 codes (bytes b, b+1 of w) -> one bf16 pair, exact:
-// 0x4B0000uu is the float 2^23 + u, and 2^23 + 128 is subtracted.
-template <int kByte>
-__device__ __forceinline__ float int8_offset_to_float(uint32_t w) {
-  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7650u | kByte)) - 8388736.0f;
+// Offset-binary INT5 codes of k16 step S: low nibbles as for INT4 in w, the
+// fifth bit of the low / high column of position q (q = 0..3 for a0, a2, a1,
+// a3) at bits 4S+q / 4S+q+16 of hb.  The fifth bit goes to bit 4 (1024 bias)
+// or bit 8 (64 bias, whose mantissa step is at bit 4).
+template <int S>
+__device__ __forceinline__ void unpack_int5_biased(uint32_t w, uint32_t hb, uint32_t (&a)[4]) {
+  const uint32_t w8 = w >> 8;
+  a[0] = and_or_r(shift_to<4 * S + 0 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w));
+  a[2] = and_or_r(shift_to<4 * S + 1 - 8>(hb), 0x01000100u, and_or<0x00F000F0u, 0x54005400u>(w));
+  a[1] = and_or_r(shift_to<4 * S + 2 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w8));
+  a[3] = and_or_r(shift_to<4 * S + 3 - 8>(hb), 0x01000100u, and_or<0x00F000F0u, 0x54005400u>(w8));
 }
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+
+// Offset-binary INT8 bytes (row gr col c, row gr col c+1, row gr+8 col c,
+// row gr+8 col c+1) of w0 (columns c) and w1 (columns c+8): one byte permute
+// per pair puts each byte under the exponent of 1024.
+__device__ __forceinline__ void unpack_int8_biased(uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
+  a[0] = __byte_perm(w0, 0x64646464u, 0x4140u);
+  a[1] = __byte_perm(w0, 0x64646464u, 0x4342u);
+  a[2] = __byte_perm(w1, 0x64646464u, 0x4140u);
+  a[3] = __byte_perm(w1, 0x64646464u, 0x4342u);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ void unpack_int8_pair_words(uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
-  a[0] = pack_bf16x2(int8_offset_to_float<0>(w0), int8_offset_to_float<1>(w0));
-  a[1] = pack_bf16x2(int8_offset_to_float<2>(w0), int8_offset_to_float<3>(w0));
-  a[2] = pack_bf16x2(int8_offset_to_float<0>(w1), int8_offset_to_float<1>(w1));
-  a[3] = pack_bf16x2(int8_offset_to_float<2>(w1), int8_offset_to_float<3>(w1));
 }
 
 __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t bits) {

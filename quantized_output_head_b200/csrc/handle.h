@@ -12,9 +12,9 @@ struct archead_handle {
   int device;
   int num_sms;
   int grid;                 // decode blocks (one per SM, at most one per m-tile)
-  int cres;                 // residual chunks per residual warp (kernel instance)
-  int nw_res, nw_L, nw_A, nw_work, nw_cons, stages;
-  size_t smem;              // dynamic shared memory of the decode kernel
+  int nw_res, nw_L, nw_A, nw_work;   // decode compute warps by role
+  int smem_optin;           // shared memory a block may use on this device
+  int e_B;                  // 2^e_B bounds the L1 norm of every dequantised R / B row
   cudaEvent_t ev_before;    // optional profiling events (not owned)
   cudaEvent_t ev_after;
 };
@@ -23,7 +23,7 @@ namespace archead {
 
 // Workspace regions of one forward call with T tokens.
 struct WsLayout {
-  size_t counter, status, zhi, zlo, partials, tgt, total;
+  size_t counter, status, escale, zhi, zlo, partials, tgt, total;
   // host-buffer form only
   size_t h_hidden, h_targets, h_lse, h_argmax, h_ce, host_total;
 };
@@ -35,6 +35,7 @@ inline WsLayout ws_layout(const archead_handle& h, int T) {
   w.counter = 0;
   w.status = 4;
   o = 256;
+  w.escale = o;   o += round_up(t * 4, 256);
   w.zhi = o;      o += round_up(t * h.L.Kz * 2, 256);
   w.zlo = o;      o += round_up(t * h.L.Kz * 2, 256);
   w.partials = o; o += round_up(t * h.grid * 16, 256);
@@ -50,9 +51,9 @@ inline WsLayout ws_layout(const archead_handle& h, int T) {
 }
 
 // Kernel launchers and attributes (decode.cu, prologue.cu).
-size_t decode_smem_bytes(int stages, uint32_t mblk_bytes, int nw_work);
-cudaError_t decode_set_attributes(int cres, size_t smem);
-cudaError_t launch_decode(int cres, const DecodeParams& p, int grid, size_t smem, cudaStream_t stream);
+size_t decode_smem_bytes(int stages, uint32_t mblk_bytes, int nw_work, int nt);
+cudaError_t decode_set_attributes(int g_steps, size_t smem);
+cudaError_t launch_decode(int g_steps, const DecodeParams& p, int grid, size_t smem, cudaStream_t stream);
 cudaError_t launch_prologue(const PrologueParams& p, cudaStream_t stream);
 
 // Thread-local record of the last CUDA error (api.cu).

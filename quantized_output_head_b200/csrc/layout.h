@@ -16,16 +16,17 @@
 //   lane l = 4*gr + cc;  fragment register p (p = 0..3) holds the pair
 //   (row gr + 8*(p&1), col k0 + 2*cc + 8*(p>>1)) and the column after it.
 // Codes are stored in offset binary (code + 8 for INT4, code + 16 for INT5,
-// code + 128 for INT8) so that unpacking is a mask, an OR with the exponent of
-// 128.0 and one subtraction, all exact in bf16.
+// code + 128 for INT8), so one mask-and-OR under an fp16 exponent turns a field
+// into an exact fp16 number (bias + offset code).
 //
 // m-tile block (all offsets multiples of 16 bytes):
-//   res   [d/64 chunks][32 lanes][4 words]   word s = k16 step s of the chunk:
-//          nibble p at bits 4p..4p+3 = low column of pair p, at bits
-//          4p+16..4p+19 = high column of pair p                (512 B / chunk)
+//   res   [d/64 chunks][32 lanes][4 words]   word s = k16 step s of the chunk;
+//          register p sits at nibble position q = (0, 2, 1, 3)[p]: bits
+//          4q..4q+3 hold the low column, bits 4q+16..4q+19 the high column
+//                                                               (512 B / chunk)
 //   Lnib  [r_c'/64 chunks][32][4 words]      same, low 4 bits of (code + 16)
-//   Lhi   [r_c'/64 chunks][32 lanes] u32     bit 4s+p / 4s+p+16 = bit 4 of the
-//          low / high column of pair p at step s                (128 B / chunk)
+//   Lhi   [r_c'/64 chunks][32 lanes] u32     bit 4s+q / 4s+q+16 = bit 4 of the
+//          low / high column of position q at step s            (128 B / chunk)
 //   A     [r_r'/32 chunks][32][2 steps][2 words]  word 2s+h: bytes
 //          (row gr col c, row gr col c+1, row gr+8 col c, row gr+8 col c+1),
 //          c = k0 + 2cc + 8h                                   (512 B / chunk)

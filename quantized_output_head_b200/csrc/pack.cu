@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <new>
@@ -18,6 +19,12 @@ namespace archead {
 namespace {
 
 bool fp16_finite(uint16_t b) { return (b & 0x7C00u) != 0x7C00u; }
+
+double half_to_double(uint16_t b) {
+  const int e = (b >> 10) & 0x1F, m = b & 0x3FF;
+  const double v = (e == 0) ? std::ldexp(static_cast<double>(m), -24) : std::ldexp(1024.0 + m, e - 25);
+  return (b & 0x8000u) ? -v : v;
+}
 
 bool codes_in_range(const int8_t* p, size_t n, int lo, int hi) {
   for (size_t i = 0; i < n; ++i)
@@ -46,9 +53,12 @@ struct Src {
   uint16_t s_A(int r) const { return (r < L.V && L.r_r > 0) ? C.s_A[r] : 0; }
 };
 
-// Row and column of fragment pair p (low column) for lane (gr, cc) at k16 step base k0.
+// Row and column of fragment register p (p = 0..3: a0..a3; low column of the
+// pair) for lane (gr, cc) at k16 step base k0, and the nibble position q of
+// that register in a packed word (a0, a2, a1, a3 at q = 0, 1, 2, 3).
 inline int frag_row(int v0, int gr, int p) { return v0 + gr + 8 * (p & 1); }
 inline int frag_col(int k0, int cc, int p) { return k0 + 2 * cc + 8 * (p >> 1); }
+inline int nib_pos(int p) { return (p == 1) ? 2 : (p == 2) ? 1 : p; }
 
 void pack_mtile(const Src& S, int mt, uint8_t* blk) {
   const Layout& L = S.L;
@@ -65,7 +75,8 @@ void pack_mtile(const Src& S, int mt, uint8_t* blk) {
           const int r = frag_row(v0, gr, p), c = frag_col(k0, cc, p);
           const uint32_t lo = static_cast<uint32_t>(S.code_q(r, c) + 8);
           const uint32_t hi = static_cast<uint32_t>(S.code_q(r, c + 1) + 8);
-          w |= (lo << (4 * p)) | (hi << (4 * p + 16));
+          const int q = nib_pos(p);
+          w |= (lo << (4 * q)) | (hi << (4 * q + 16));
         }
         dst[s] = w;
       }
@@ -81,8 +92,9 @@ void pack_mtile(const Src& S, int mt, uint8_t* blk) {
           const int r = frag_row(v0, gr, p), c = frag_col(k0, cc, p);
           const uint32_t lo = static_cast<uint32_t>(S.code_L(r, c) + 16);
           const uint32_t hi = static_cast<uint32_t>(S.code_L(r, c + 1) + 16);
-          w |= ((lo & 15u) << (4 * p)) | ((hi & 15u) << (4 * p + 16));
-          hb |= ((lo >> 4) << (4 * s + p)) | ((hi >> 4) << (4 * s + p + 16));
+          const int q = nib_pos(p);
+          w |= ((lo & 15u) << (4 * q)) | ((hi & 15u) << (4 * q + 16));
+          hb |= ((lo >> 4) << (4 * s + q)) | ((hi >> 4) << (4 * s + q + 16));
         }
         dst[s] = w;
       }
@@ -122,28 +134,41 @@ void pack_mtile(const Src& S, int mt, uint8_t* blk) {
 
 bool plan_decode(archead_handle* h, int smem_optin) {
   const Layout& L = h->L;
-  for (int cres : {kCRes, 2 * kCRes}) {
-    const int nw_res = (L.n_res + cres - 1) / cres;
-    const int nw_L = (L.n_L + kCL - 1) / kCL;
-    const int nw_A = (L.n_A + kCA - 1) / kCA;
-    const int nw_work = nw_res + nw_L + nw_A;
-    const int nw_cons = std::max(nw_work, 4);
-    if (1 + nw_cons > kMaxDecodeWarps) continue;
-    const size_t fixed = decode_smem_bytes(0, L.mblk_bytes, nw_work) + 16 * kMaxStages;
-    if (fixed >= static_cast<size_t>(smem_optin)) return false;
-    const int stages = static_cast<int>(std::min<size_t>(kMaxStages, (smem_optin - fixed) / L.mblk_bytes));
-    if (stages < 2) return false;
-    h->cres = cres;
-    h->nw_res = nw_res;
-    h->nw_L = nw_L;
-    h->nw_A = nw_A;
-    h->nw_work = nw_work;
-    h->nw_cons = nw_cons;
-    h->stages = stages;
-    h->smem = decode_smem_bytes(stages, L.mblk_bytes, nw_work);
-    return true;
+  const int nw_res = (L.n_res + kCRes - 1) / kCRes;
+  const int nw_L = (L.n_L + kCL - 1) / kCL;
+  const int nw_A = (L.n_A + kCA - 1) / kCA;
+  const int nw_work = nw_res + nw_L + nw_A;
+  if (2 + nw_work > kMaxDecodeWarps) return false;
+  // Two stages at the widest launch (8 tokens) must fit.
+  if (decode_smem_bytes(2, L.mblk_bytes, nw_work, kDecodeTokens) > static_cast<size_t>(smem_optin)) return false;
+  h->nw_res = nw_res;
+  h->nw_L = nw_L;
+  h->nw_A = nw_A;
+  h->nw_work = nw_work;
+  h->smem_optin = smem_optin;
+  return true;
+}
+
+// Smallest e with 2^e >= the largest L1 norm of a dequantised R or B row.
+int row_norm_exponent(const Layout& L, const archead_host_components& C) {
+  double bmax = 0.0;
+  const size_t d = L.d;
+  for (int k = 0; k < L.r_c; ++k) {
+    double a = 0.0;
+    for (size_t j = 0; j < d; ++j) a += std::abs(static_cast<double>(C.R[k * d + j]));
+    bmax = std::max(bmax, a * half_to_double(C.s_R[k]));
   }
-  return false;
+  const size_t ngB = d / L.g_B;
+  for (int k = 0; k < L.r_r; ++k) {
+    double a = 0.0;
+    for (size_t j = 0; j < d; ++j)
+      a += std::abs(static_cast<double>(C.B[k * d + j])) * half_to_double(C.s_B[k * ngB + j / L.g_B]);
+    bmax = std::max(bmax, a);
+  }
+  if (bmax <= 0.0) return 0;
+  int e = 0;
+  std::frexp(bmax, &e);   // bmax < 2^e
+  return e;
 }
 
 }  // namespace
@@ -251,7 +276,8 @@ extern "C" ARCHEAD_API int archead_pack_load(const archead_desc* desc, const arc
     delete h;
     return ARCHEAD_EUNSUP;
   }
-  e = decode_set_attributes(h->cres, h->smem);
+  h->e_B = row_norm_exponent(L, *comps);
+  e = decode_set_attributes(L.g_steps, static_cast<size_t>(optin));
   if (e != cudaSuccess) {
     delete h;
     return set_cuda_error(e);

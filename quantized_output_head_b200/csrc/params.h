@@ -4,21 +4,25 @@
 
 namespace archead {
 
-// Warps per role in the decode kernel: each residual warp owns kCRes 64-column
-// chunks of d, each core warp kCL 64-column chunks of r_c', each correction
-// warp kCA 32-column chunks of r_r'.
+// Work split of the decode kernel: each residual warp owns kCRes 64-column
+// chunks of d (16 k16 steps), each core warp kCL 64-column chunks of r_c',
+// each correction warp kCA 32-column chunks of r_r'.
 constexpr int kCRes = 4;
 constexpr int kCL = 2;
 constexpr int kCA = 2;
 constexpr int kMaxDecodeWarps = 24;      // launch bound of the decode kernel
 constexpr int kDecodeTokens = 8;         // N of one m16n8k16 fragment
 constexpr int kMaxStages = 6;
+// h is scaled per token by 2^(kScaleExp - E_t), E_t the binary exponent of
+// max|h_t| (max|h_t| < 2^E_t), so the fp16 copy is below 2^kScaleExp.
+constexpr int kScaleExp = 14;
 
 struct DecodeParams {
   const uint8_t* mtiles;       // arena: m-tile blocks
   const uint16_t* hidden;      // [T, d] bf16
-  const uint16_t* zhi;         // [T, Kz] bf16: high part of (z_c | z_r)
-  const uint16_t* zlo;         // [T, Kz] bf16: z - high part
+  const uint16_t* zhi;         // [T, Kz] fp16: high part of (z_c | z_r) * 2^(kScaleExp - E_t - e_B)
+  const uint16_t* zlo;         // [T, Kz] fp16: remainder
+  const int32_t* escale;       // [T] E_t
   const int32_t* targets;      // [T] or null
   float* logits;               // [T, V] or null
   int32_t* argmax;             // [T] or null
@@ -29,10 +33,10 @@ struct DecodeParams {
   uint32_t* counter;           // completion ticket
   uint32_t* status;            // ARCHEAD_STATUS_* bits
   int32_t T, t0, nt;           // this launch covers tokens [t0, t0 + nt), nt <= 8
-  int32_t V, d, Kz, rcp;
+  int32_t V, d, Kz, rcp, e_B;
   int32_t n_res, n_L, n_A, n_mtiles, g_steps_log2;
   uint32_t off_res, off_Lnib, off_Lhi, off_A, off_sres, off_sL, off_sA, mblk_bytes;
-  int32_t nw_res, nw_L, nw_A, nw_work, nw_cons;   // consumer warps (nw_cons >= 4)
+  int32_t nw_res, nw_L, nw_A, nw_work;   // compute warps by role
   int32_t stages;
 };
 
@@ -43,11 +47,12 @@ struct PrologueParams {
   const int8_t* B;             // [rrp, d]
   const uint16_t* s_B;         // [rrp, d / g_B]
   const int32_t* targets;      // [T] or null
-  uint16_t* zhi;               // [T, Kz]
-  uint16_t* zlo;               // [T, Kz]
+  uint16_t* zhi;               // [T, Kz] fp16
+  uint16_t* zlo;               // [T, Kz] fp16
+  int32_t* escale;             // [T]
   uint32_t* counter;
   uint32_t* status;
-  int32_t T, d, rcp, rrp, Kz, g_B, V;
+  int32_t T, d, rcp, rrp, Kz, g_B, V, e_B;
 };
 
 }  // namespace archead

@@ -2,10 +2,14 @@
 // the same factoring of the core of Eq. 3):
 //   z_c[t,k] = s_R[k] sum_j R[k,j] h[t,j]                k < r_c
 //   z_r[t,k] = sum_j s_B[k, j/g_B] B[k,j] h[t,j]         k < r_r
-// accumulated in fp32 and stored as a bf16 pair (high part, remainder) so the
-// tensor-core pass can consume z at ~16 significant bits.  One warp per output
-// row k (R and B rows are read once per token from L1/L2).  The kernel also
-// resets the decode kernel's completion ticket and checks the target ids.
+// accumulated in fp32.  For the fp16 tensor-core pass each token gets a power
+// of two: E_t with max_j |h[t,j]| < 2^E_t.  z is stored scaled by
+// 2^(kScaleExp - E_t - e_B), where 2^e_B bounds the L1 norm of every
+// dequantised R / B row (so |scaled z| < 2^kScaleExp), as an fp16 pair: the
+// rounded value and the rounded remainder.  One warp per output row k; every
+// warp finds max|h_t| itself from the row it reads, and warp 0 of block 0
+// publishes E_t.  The kernel also resets the decode kernel's completion ticket
+// and checks the target ids.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -28,45 +32,62 @@ __global__ void __launch_bounds__(256) prologue_kernel(const PrologueParams p) {
   }
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= p.Kz) return;
+  const bool publisher = row == 0;
+  const bool has_row = row < p.Kz;
+  if (!has_row && !publisher) return;
   const bool core = row < p.rcp;
   const int k = core ? row : row - p.rcp;
-  const int8_t* codes = (core ? p.R : p.B) + static_cast<size_t>(k) * p.d;
+  const int8_t* codes = has_row ? (core ? p.R : p.B) + static_cast<size_t>(k) * p.d : nullptr;
   const int ngB = p.d / p.g_B;
-  const float s_row = core ? __half2float(__ushort_as_half(p.s_R[k])) : 1.f;
+  const float s_row = (has_row && core) ? __half2float(__ushort_as_half(p.s_R[k])) : 1.f;
   for (int t = 0; t < p.T; ++t) {
     const uint16_t* h = p.hidden + static_cast<size_t>(t) * p.d;
     float acc = 0.f;
+    float hmax = 0.f;
     for (int j = lane * 16; j < p.d; j += 32 * 16) {
-      const int4 cv = *reinterpret_cast<const int4*>(codes + j);
       const uint4 hv0 = *reinterpret_cast<const uint4*>(h + j);
       const uint4 hv1 = *reinterpret_cast<const uint4*>(h + j + 8);
-      const int8_t* c8 = reinterpret_cast<const int8_t*>(&cv);
+      float hf[16];
       const __nv_bfloat16* hb0 = reinterpret_cast<const __nv_bfloat16*>(&hv0);
       const __nv_bfloat16* hb1 = reinterpret_cast<const __nv_bfloat16*>(&hv1);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        hf[e] = __bfloat162float(hb0[e]);
+        hf[8 + e] = __bfloat162float(hb1[e]);
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) hmax = fmaxf(hmax, fabsf(hf[e]));
+      if (!has_row) continue;
+      const int4 cv = *reinterpret_cast<const int4*>(codes + j);
+      const int8_t* c8 = reinterpret_cast<const int8_t*>(&cv);
       if (core) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc = fmaf(static_cast<float>(c8[e]), __bfloat162float(hb0[e]), acc);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc = fmaf(static_cast<float>(c8[8 + e]), __bfloat162float(hb1[e]), acc);
+        for (int e = 0; e < 16; ++e) acc = fmaf(static_cast<float>(c8[e]), hf[e], acc);
       } else {
         const uint16_t* sb = p.s_B + static_cast<size_t>(k) * ngB;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float sc = __half2float(__ushort_as_half(sb[(j + e) / p.g_B]));
-          const float hv = e < 8 ? __bfloat162float(hb0[e]) : __bfloat162float(hb1[e - 8]);
-          acc = fmaf(sc * static_cast<float>(c8[e]), hv, acc);
+          acc = fmaf(sc * static_cast<float>(c8[e]), hf[e], acc);
         }
       }
     }
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    for (int m = 16; m >= 1; m >>= 1) {
+      acc += __shfl_xor_sync(0xffffffffu, acc, m);
+      hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, m));
+    }
+    int E = 0;
+    frexpf(hmax, &E);   // hmax < 2^E (E = 0 when hmax = 0)
     if (lane == 0) {
-      const float z = acc * s_row;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(z);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(z - __bfloat162float(hi));
-      p.zhi[static_cast<size_t>(t) * p.Kz + row] = __bfloat16_as_ushort(hi);
-      p.zlo[static_cast<size_t>(t) * p.Kz + row] = __bfloat16_as_ushort(lo);
+      if (publisher) p.escale[t] = E;
+      if (has_row) {
+        const float z = ldexpf(acc * s_row, kScaleExp - E - p.e_B);
+        const __half hi = __float2half_rn(z);
+        const __half lo = __float2half_rn(z - __half2float(hi));
+        p.zhi[static_cast<size_t>(t) * p.Kz + row] = __half_as_ushort(hi);
+        p.zlo[static_cast<size_t>(t) * p.Kz + row] = __half_as_ushort(lo);
+      }
     }
   }
 }

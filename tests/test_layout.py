@@ -25,6 +25,10 @@ def qoh():
     return m
 
 
+# nibble position of fragment register a0..a3 inside a packed word
+NIB_POS = (0, 2, 1, 3)
+
+
 def _ru(x, m):
     return (x + m - 1) // m * m
 
@@ -61,8 +65,9 @@ def decode_image(img, V, d, r_c, r_r, g, g_B):
     rows = frag_rows()[:, None, :, None, :]                         # [mt, 1, lane, 1, p]
     cols = frag_cols(n_res, 64, 4)[None]                           # [1, ch, lane, s, p]
     for p in range(4):
-        lo = (w >> (4 * p)) & 15
-        hi = (w >> (4 * p + 16)) & 15
+        q_ = NIB_POS[p]
+        lo = (w >> (4 * q_)) & 15
+        hi = (w >> (4 * q_ + 16)) & 15
         r = np.broadcast_to(rows[..., p], lo.shape)
         c = np.broadcast_to(cols[..., p], lo.shape)
         q[r, c] = lo.astype(np.int64) - 8
@@ -76,8 +81,9 @@ def decode_image(img, V, d, r_c, r_r, g, g_B):
         cols = frag_cols(n_L, 64, 4)[None]
         s_idx = np.arange(4)[None, None, None, :]
         for p in range(4):
-            lo = ((w >> (4 * p)) & 15) | (((hb[..., None] >> (4 * s_idx + p)) & 1) << 4)
-            hi = ((w >> (4 * p + 16)) & 15) | (((hb[..., None] >> (4 * s_idx + p + 16)) & 1) << 4)
+            q_ = NIB_POS[p]
+            lo = ((w >> (4 * q_)) & 15) | (((hb[..., None] >> (4 * s_idx + q_)) & 1) << 4)
+            hi = ((w >> (4 * q_ + 16)) & 15) | (((hb[..., None] >> (4 * s_idx + q_ + 16)) & 1) << 4)
             r = np.broadcast_to(rows[..., p], lo.shape)
             c = np.broadcast_to(cols[..., p], lo.shape)
             Lc[r, c] = lo.astype(np.int64) - 16
