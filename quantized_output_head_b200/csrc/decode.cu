@@ -401,8 +401,17 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     for (int k = 0; k < kEpiSlots; ++k) {
       const int e = lane + 32 * k;
       if (ok && e < nel) {
-        float y = 0.f;
-        for (int w = 0; w < p.nw_work; ++w) y += red[w * nel + e];
+        // four independent partial sums so the shared-memory loads overlap
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        int w = 0;
+        for (; w + 4 <= p.nw_work; w += 4) {
+          y0 += red[(w + 0) * nel + e];
+          y1 += red[(w + 1) * nel + e];
+          y2 += red[(w + 2) * nel + e];
+          y3 += red[(w + 3) * nel + e];
+        }
+        for (; w < p.nw_work; ++w) y0 += red[w * nel + e];
+        const float y = (y0 + y1) + (y2 + y3);
         const int row = e & 15, t = e >> 4;
         const int v = vbase + row;
         if (v < p.V) {

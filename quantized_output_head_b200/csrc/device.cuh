@@ -169,13 +169,15 @@ struct LseState {
 __device__ __forceinline__ LseState lse_init() { return LseState{-INFINITY, 0.f, 0x7fffffff}; }
 // Elements arrive in increasing index order per thread, so a strict > keeps
 // the lowest index among equal maxima.
+// The fast exponential is enough here: each term carries a relative error of a
+// few ulp, far inside the LSE tolerance, and the maximum itself is exact.
 __device__ __forceinline__ void lse_push(LseState& st, float y, int v) {
   if (y > st.m) {
-    st.s = st.s * expf(st.m - y) + 1.f;
+    st.s = st.s * __expf(st.m - y) + 1.f;
     st.m = y;
     st.idx = v;
   } else {
-    st.s += expf(y - st.m);
+    st.s += __expf(y - st.m);
   }
 }
 __device__ __forceinline__ LseState lse_merge(const LseState& a, const LseState& b) {

@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(256) prologue_kernel(const PrologueParams p) {
     const uint16_t* h = p.hidden + static_cast<size_t>(t) * p.d;
     float acc = 0.f;
     float hmax = 0.f;
+#pragma unroll 4
     for (int j = lane * 16; j < p.d; j += 32 * 16) {
       const uint4 hv0 = *reinterpret_cast<const uint4*>(h + j);
       const uint4 hv1 = *reinterpret_cast<const uint4*>(h + j + 8);
