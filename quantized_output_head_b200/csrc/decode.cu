@@ -18,7 +18,7 @@
 // barrier after setup):
 //   warp 0            producer: bulk-copies whole m-tile blocks HBM -> SMEM
 //                     into a ring of `stages` slots                 (full[s])
-//   warp 1            epilogue: sums the compute warps' 16 x nt partial tiles
+//   warp 1            epilogue: takes the summed 16 x nt logit tile of a stage
 //                     (reduced[s]), pushes each logit into a running
 //                     log-sum-exp / argmax state, writes logits when asked,
 //                     then frees the slot                          (empty[s])
@@ -26,7 +26,9 @@
 //                     h fragments of its columns stay in registers
 //   core warps        each owns kCL 64-column chunks of r_c'
 //   correction warps  each owns kCA 32-column chunks of r_r'
-// At the end every block writes one partial per token; the last block to
+// Each compute warp stores its 16 x nt partial tile and bumps a per-stage
+// counter; the last one sums the tiles in warp order (deterministic) and
+// signals the epilogue warp.  At the end every block writes one partial per token; the last block to
 // finish (atomic ticket, no spinning) merges them into LSE, argmax and CE.
 // Every wait on an mbarrier is bounded (kWaitLimitNs); on expiry the block
 // raises ARCHEAD_STATUS_WAIT_TIMEOUT, skips the remaining work and drains its
@@ -44,21 +46,26 @@ constexpr int kEpiSlots = 4;     // 16 rows x 8 tokens / 32 lanes
 
 struct SmemView {
   uint8_t* stages;
-  float* red;          // [stages][nw_work][nt][16]
+  float* red;          // [stages][nw_work][16 rows][nt]   per-warp partial tiles
+  float* tsum;         // [stages][nt][16 rows]            summed tile
   uint64_t* full;      // [stages] producer -> compute warps
-  uint64_t* reduced;   // [stages] compute warps -> epilogue warp
+  uint64_t* reduced;   // [stages] last compute warp -> epilogue warp
   uint64_t* empty;     // [stages] epilogue warp -> producer
+  int* arrivals;       // [stages] compute warps done with the stage
   int* flags;          // [0] abort
 };
 
 __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams& p) {
   SmemView v;
+  const size_t tile = static_cast<size_t>(p.nt) * 16;
   v.stages = smem;
   v.red = reinterpret_cast<float*>(smem + static_cast<size_t>(p.stages) * p.mblk_bytes);
-  v.full = reinterpret_cast<uint64_t*>(v.red + static_cast<size_t>(p.stages) * p.nw_work * p.nt * 16);
+  v.tsum = v.red + static_cast<size_t>(p.stages) * p.nw_work * tile;
+  v.full = reinterpret_cast<uint64_t*>(v.tsum + static_cast<size_t>(p.stages) * tile);
   v.reduced = v.full + p.stages;
   v.empty = v.reduced + p.stages;
-  v.flags = reinterpret_cast<int*>(v.empty + p.stages);
+  v.arrivals = reinterpret_cast<int*>(v.empty + p.stages);
+  v.flags = v.arrivals + p.stages;
   return v;
 }
 
@@ -145,19 +152,65 @@ __device__ __forceinline__ float quad_sum(float v) {
   return v;
 }
 
+// Partial tile of one warp for one stage, [16 rows][nt] (row-major, so a
+// lane's two token columns are one 8-byte store and a warp's stores hit
+// distinct banks).
 __device__ __forceinline__ void store_partial(const SmemView& sv, const DecodeParams& p, int s, int cw, int lane,
                                               const float (&acc)[4]) {
   const int gr = lane >> 2, cc = lane & 3;
-  float* r = sv.red + (static_cast<size_t>(s) * p.nw_work + cw) * p.nt * 16;
-  const int t0 = 2 * cc, t1 = 2 * cc + 1;
-  if (t0 < p.nt) {
-    r[t0 * 16 + gr] = acc[0];
-    r[t0 * 16 + gr + 8] = acc[2];
+  const int nt = p.nt;
+  float* r = sv.red + (static_cast<size_t>(s) * p.nw_work + cw) * nt * 16;
+  const int t0 = 2 * cc;
+  if ((nt & 1) == 0 && t0 < nt) {
+    // nt even: gr * nt + t0 is even, so the 8-byte stores are aligned
+    *reinterpret_cast<float2*>(r + gr * nt + t0) = make_float2(acc[0], acc[1]);
+    *reinterpret_cast<float2*>(r + (gr + 8) * nt + t0) = make_float2(acc[2], acc[3]);
+  } else {
+    if (t0 < nt) {
+      r[gr * nt + t0] = acc[0];
+      r[(gr + 8) * nt + t0] = acc[2];
+    }
+    if (t0 + 1 < nt) {
+      r[gr * nt + t0 + 1] = acc[1];
+      r[(gr + 8) * nt + t0 + 1] = acc[3];
+    }
   }
-  if (t1 < p.nt) {
-    r[t1 * 16 + gr] = acc[1];
-    r[t1 * 16 + gr + 8] = acc[3];
+}
+
+// After a compute warp has stored its partial tile of stage s: count it, and
+// if it is the last of the nw_work warps, sum the tiles in warp order (fixed,
+// so results are deterministic) into tsum[s] and hand the stage to the
+// epilogue warp.  No warp ever waits here.
+__device__ __forceinline__ void finish_stage(const SmemView& sv, const DecodeParams& p, int s, int lane) {
+  __syncwarp();
+  int prev = 0;
+  if (lane == 0) {
+    __threadfence_block();
+    prev = atomicAdd(&sv.arrivals[s], 1);
   }
+  prev = __shfl_sync(0xffffffffu, prev, 0);
+  if (prev != p.nw_work - 1) return;
+  if (lane == 0) sv.arrivals[s] = 0;
+  __syncwarp();
+  __threadfence_block();
+  const int nt = p.nt, nel = 16 * nt;
+  const float* red = sv.red + static_cast<size_t>(s) * p.nw_work * nel;
+  float* out = sv.tsum + static_cast<size_t>(s) * nel;
+  for (int e = lane; e < nel; e += 32) {          // e = t * 16 + row
+    const int src = (e & 15) * nt + (e >> 4);
+    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+    int w = 0;
+    for (; w + 4 <= p.nw_work; w += 4) {
+      y0 += red[(w + 0) * nel + src];
+      y1 += red[(w + 1) * nel + src];
+      y2 += red[(w + 2) * nel + src];
+      y3 += red[(w + 3) * nel + src];
+    }
+    for (; w < p.nw_work; ++w) y0 += red[w * nel + src];
+    out[e] = (y0 + y1) + (y2 + y3);
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[s]));
 }
 
 // ------------------------------------------------------------ residual warps
@@ -246,8 +299,7 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
       acc[3] *= unscale.y;
     }
     store_partial(sv, p, s, cw, lane, acc);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[s]));
+    finish_stage(sv, p, s, lane);
   }
 }
 
@@ -314,8 +366,7 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
       }
     }
     store_partial(sv, p, s, cw, lane, acc);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[s]));
+    finish_stage(sv, p, s, lane);
   }
 }
 
@@ -375,8 +426,7 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
       }
     }
     store_partial(sv, p, s, cw, lane, acc);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[s]));
+    finish_stage(sv, p, s, lane);
   }
 }
 
@@ -395,23 +445,13 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
   for (int i = 0; i < n_my; ++i) {
     const int s = i % S;
     const bool ok = warp_wait(sv, &sv.reduced[s], (i / S) & 1, p.status, lane);
-    const float* red = sv.red + static_cast<size_t>(s) * p.nw_work * nel;
+    const float* tsum = sv.tsum + static_cast<size_t>(s) * nel;
     const int vbase = mtile_of(i) * kMT;
 #pragma unroll
     for (int k = 0; k < kEpiSlots; ++k) {
       const int e = lane + 32 * k;
       if (ok && e < nel) {
-        // four independent partial sums so the shared-memory loads overlap
-        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-        int w = 0;
-        for (; w + 4 <= p.nw_work; w += 4) {
-          y0 += red[(w + 0) * nel + e];
-          y1 += red[(w + 1) * nel + e];
-          y2 += red[(w + 2) * nel + e];
-          y3 += red[(w + 3) * nel + e];
-        }
-        for (; w < p.nw_work; ++w) y0 += red[w * nel + e];
-        const float y = (y0 + y1) + (y2 + y3);
+        const float y = tsum[e];
         const int row = e & 15, t = e >> 4;
         const int v = vbase + row;
         if (v < p.V) {
@@ -478,8 +518,9 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_addr(&sv.full[s]), 1);
-      mbar_init(smem_addr(&sv.reduced[s]), p.nw_work);
+      mbar_init(smem_addr(&sv.reduced[s]), 1);
       mbar_init(smem_addr(&sv.empty[s]), 1);
+      sv.arrivals[s] = 0;
     }
     sv.flags[0] = 0;
     mbar_fence_init();
@@ -507,8 +548,8 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
 }
 
 size_t decode_smem_bytes(int stages, uint32_t mblk_bytes, int nw_work, int nt) {
-  return static_cast<size_t>(stages) * mblk_bytes + static_cast<size_t>(stages) * nw_work * nt * 16 * 4 +
-         static_cast<size_t>(3) * stages * 8 + 16;
+  return static_cast<size_t>(stages) * mblk_bytes + static_cast<size_t>(stages) * (nw_work + 1) * nt * 16 * 4 +
+         static_cast<size_t>(3) * stages * 8 + static_cast<size_t>(stages) * 4 + 16;
 }
 
 namespace {
