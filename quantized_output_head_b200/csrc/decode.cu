@@ -17,11 +17,13 @@
 // Block organisation (one block per SM, persistent over m-tiles; no block-wide
 // barrier after setup):
 //   warp 0            producer: bulk-copies whole m-tile blocks HBM -> SMEM
-//                     into a ring of `stages` slots                 (full[s])
-//   warp 1            epilogue: takes the summed 16 x nt logit tile of a stage
-//                     (reduced[s]), pushes each logit into a running
-//                     log-sum-exp / argmax state, writes logits when asked,
-//                     then frees the slot                          (empty[s])
+//                     into a ring of `stages` buffers (full[s]); a buffer is
+//                     refilled as soon as every compute warp has read it
+//                     (empty[s]), independent of the epilogue
+//   warp 1            epilogue: takes the summed 16 x nt logit tile of a
+//                     partial-tile slot (reduced[r]), pushes each logit into a
+//                     running log-sum-exp / argmax state, writes logits when
+//                     asked, then frees the slot                  (redfree[r])
 //   residual warps    each owns 16 k16 steps of d for every m-tile; the fp16
 //                     h fragments of its columns stay in registers
 //   core warps        each owns kCL 64-column chunks of r_c'
@@ -46,12 +48,13 @@ constexpr int kEpiSlots = 4;     // 16 rows x 8 tokens / 32 lanes
 
 struct SmemView {
   uint8_t* stages;
-  float* red;          // [stages][nw_work][16 rows][nt]   per-warp partial tiles
-  float* tsum;         // [stages][nt][16 rows]            summed tile
-  uint64_t* full;      // [stages] producer -> compute warps
-  uint64_t* reduced;   // [stages] last compute warp -> epilogue warp
-  uint64_t* empty;     // [stages] epilogue warp -> producer
-  int* arrivals;       // [stages] compute warps done with the stage
+  float* red;          // [slots][nw_work][16 rows][nt]   per-warp partial tiles
+  float* tsum;         // [slots][nt][16 rows]            summed tile
+  uint64_t* full;      // [stages] producer -> compute warps (bytes landed)
+  uint64_t* empty;     // [stages] compute warps -> producer (stage read)
+  uint64_t* reduced;   // [slots]  last compute warp -> epilogue warp
+  uint64_t* redfree;   // [slots]  epilogue warp -> compute warps
+  int* arrivals;       // [slots]  compute warps done with the slot
   int* flags;          // [0] abort
 };
 
@@ -60,12 +63,13 @@ __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams&
   const size_t tile = static_cast<size_t>(p.nt) * 16;
   v.stages = smem;
   v.red = reinterpret_cast<float*>(smem + static_cast<size_t>(p.stages) * p.mblk_bytes);
-  v.tsum = v.red + static_cast<size_t>(p.stages) * p.nw_work * tile;
-  v.full = reinterpret_cast<uint64_t*>(v.tsum + static_cast<size_t>(p.stages) * tile);
-  v.reduced = v.full + p.stages;
-  v.empty = v.reduced + p.stages;
-  v.arrivals = reinterpret_cast<int*>(v.empty + p.stages);
-  v.flags = v.arrivals + p.stages;
+  v.tsum = v.red + static_cast<size_t>(p.slots) * p.nw_work * tile;
+  v.full = reinterpret_cast<uint64_t*>(v.tsum + static_cast<size_t>(p.slots) * tile);
+  v.empty = v.full + p.stages;
+  v.reduced = v.empty + p.stages;
+  v.redfree = v.reduced + p.slots;
+  v.arrivals = reinterpret_cast<int*>(v.redfree + p.slots);
+  v.flags = v.arrivals + p.slots;
   return v;
 }
 
@@ -177,11 +181,11 @@ __device__ __forceinline__ void store_partial(const SmemView& sv, const DecodePa
   }
 }
 
-// After a compute warp has stored its partial tile of stage s: count it, and
+// After a compute warp has stored its partial tile in slot s: count it, and
 // if it is the last of the nw_work warps, sum the tiles in warp order (fixed,
-// so results are deterministic) into tsum[s] and hand the stage to the
+// so results are deterministic) into tsum[s] and hand the slot to the
 // epilogue warp.  No warp ever waits here.
-__device__ __forceinline__ void finish_stage(const SmemView& sv, const DecodeParams& p, int s, int lane) {
+__device__ __forceinline__ void finish_slot(const SmemView& sv, const DecodeParams& p, int s, int lane) {
   __syncwarp();
   int prev = 0;
   if (lane == 0) {
@@ -298,8 +302,13 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
       acc[2] *= unscale.x;
       acc[3] *= unscale.y;
     }
-    store_partial(sv, p, s, cw, lane, acc);
-    finish_stage(sv, p, s, lane);
+    // The stage's bytes are consumed: give it back to the producer now.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
+    const int r = i % p.slots;
+    if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
+    store_partial(sv, p, r, cw, lane, acc);
+    finish_slot(sv, p, r, lane);
   }
 }
 
@@ -365,8 +374,13 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
         acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
       }
     }
-    store_partial(sv, p, s, cw, lane, acc);
-    finish_stage(sv, p, s, lane);
+    // The stage's bytes are consumed: give it back to the producer now.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
+    const int r = i % p.slots;
+    if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
+    store_partial(sv, p, r, cw, lane, acc);
+    finish_slot(sv, p, r, lane);
   }
 }
 
@@ -425,14 +439,18 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
         acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
       }
     }
-    store_partial(sv, p, s, cw, lane, acc);
-    finish_stage(sv, p, s, lane);
+    // The stage's bytes are consumed: give it back to the producer now.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
+    const int r = i % p.slots;
+    if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
+    store_partial(sv, p, r, cw, lane, acc);
+    finish_slot(sv, p, r, lane);
   }
 }
 
 // ------------------------------------------------------------ epilogue warp
 __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int lane) {
-  const int S = p.stages;
   const int nel = 16 * p.nt;
   LseState st[kEpiSlots];
   int target[kEpiSlots];
@@ -443,9 +461,9 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     target[k] = (e < nel && p.targets != nullptr) ? p.targets[p.t0 + (e >> 4)] : -1;
   }
   for (int i = 0; i < n_my; ++i) {
-    const int s = i % S;
-    const bool ok = warp_wait(sv, &sv.reduced[s], (i / S) & 1, p.status, lane);
-    const float* tsum = sv.tsum + static_cast<size_t>(s) * nel;
+    const int r = i % p.slots;
+    const bool ok = warp_wait(sv, &sv.reduced[r], (i / p.slots) & 1, p.status, lane);
+    const float* tsum = sv.tsum + static_cast<size_t>(r) * nel;
     const int vbase = mtile_of(i) * kMT;
 #pragma unroll
     for (int k = 0; k < kEpiSlots; ++k) {
@@ -462,7 +480,7 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
+    if (lane == 0) mbar_arrive(smem_addr(&sv.redfree[r]));
   }
   // Block partial per token: slot k of lanes 16h..16h+15 holds token 2k + h.
 #pragma unroll
@@ -518,9 +536,12 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_addr(&sv.full[s]), 1);
-      mbar_init(smem_addr(&sv.reduced[s]), 1);
-      mbar_init(smem_addr(&sv.empty[s]), 1);
-      sv.arrivals[s] = 0;
+      mbar_init(smem_addr(&sv.empty[s]), p.nw_work);
+    }
+    for (int r = 0; r < p.slots; ++r) {
+      mbar_init(smem_addr(&sv.reduced[r]), 1);
+      mbar_init(smem_addr(&sv.redfree[r]), 1);
+      sv.arrivals[r] = 0;
     }
     sv.flags[0] = 0;
     mbar_fence_init();
@@ -547,9 +568,10 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
   }
 }
 
-size_t decode_smem_bytes(int stages, uint32_t mblk_bytes, int nw_work, int nt) {
-  return static_cast<size_t>(stages) * mblk_bytes + static_cast<size_t>(stages) * (nw_work + 1) * nt * 16 * 4 +
-         static_cast<size_t>(3) * stages * 8 + static_cast<size_t>(stages) * 4 + 16;
+size_t decode_smem_bytes(int stages, int slots, uint32_t mblk_bytes, int nw_work, int nt) {
+  return static_cast<size_t>(stages) * mblk_bytes + static_cast<size_t>(slots) * (nw_work + 1) * nt * 16 * 4 +
+         static_cast<size_t>(2) * stages * 8 + static_cast<size_t>(2) * slots * 8 + static_cast<size_t>(slots) * 4 +
+         16;
 }
 
 namespace {

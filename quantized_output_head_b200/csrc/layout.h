@@ -41,7 +41,7 @@
 #pragma once
 #include <stdint.h>
 
-#include "../../include/archead.h"
+#include "archead.h"
 
 namespace archead {
 

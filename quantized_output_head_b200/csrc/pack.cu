@@ -140,7 +140,7 @@ bool plan_decode(archead_handle* h, int smem_optin) {
   const int nw_work = nw_res + nw_L + nw_A;
   if (2 + nw_work > kMaxDecodeWarps) return false;
   // Two stages at the widest launch (8 tokens) must fit.
-  if (decode_smem_bytes(2, L.mblk_bytes, nw_work, kDecodeTokens) > static_cast<size_t>(smem_optin)) return false;
+  if (decode_smem_bytes(2, 2, L.mblk_bytes, nw_work, kDecodeTokens) > static_cast<size_t>(smem_optin)) return false;
   h->nw_res = nw_res;
   h->nw_L = nw_L;
   h->nw_A = nw_A;

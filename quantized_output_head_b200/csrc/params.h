@@ -37,7 +37,8 @@ struct DecodeParams {
   int32_t n_res, n_L, n_A, n_mtiles, g_steps_log2;
   uint32_t off_res, off_Lnib, off_Lhi, off_A, off_sres, off_sL, off_sA, mblk_bytes;
   int32_t nw_res, nw_L, nw_A, nw_work;   // compute warps by role
-  int32_t stages;
+  int32_t stages;              // m-tile buffers in shared memory
+  int32_t slots;               // partial-tile slots between compute and epilogue warps
 };
 
 struct PrologueParams {
