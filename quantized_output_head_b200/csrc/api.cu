@@ -116,9 +116,9 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   for (int t0 = 0; t0 < T; t0 += kDecodeTokens) {
     dp.t0 = t0;
     dp.nt = (T - t0 < kDecodeTokens) ? (T - t0) : kDecodeTokens;
-    // Partial-tile slots: 4 while they are small, 2 at the widest launch;
-    // the rest of shared memory holds m-tile buffers (at most kMaxStages).
-    const int slots = dp.nt <= 4 ? 4 : 2;
+    // Eight fixed-point logit slots (at most 8 KB); the rest of shared memory
+    // holds m-tile buffers (at most kMaxStages).
+    const int slots = 8;
     const size_t fixed = decode_smem_bytes(0, slots, L.mblk_bytes, h->nw_work, dp.nt);
     const size_t per_stage = decode_smem_bytes(1, slots, L.mblk_bytes, h->nw_work, dp.nt) - fixed;
     int stages = static_cast<int>((static_cast<size_t>(h->smem_optin) - fixed) / per_stage);

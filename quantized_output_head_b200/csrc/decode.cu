@@ -20,17 +20,17 @@
 //                     into a ring of `stages` buffers (full[s]); a buffer is
 //                     refilled as soon as every compute warp has read it
 //                     (empty[s]), independent of the epilogue
-//   warp 1            epilogue: takes the summed 16 x nt logit tile of a
-//                     partial-tile slot (reduced[r]), pushes each logit into a
-//                     running log-sum-exp / argmax state, writes logits when
-//                     asked, then frees the slot                  (redfree[r])
+//   warp 1            epilogue: takes the summed 16 x nt logit tile of a slot
+//                     (reduced[r]), pushes each logit into a running
+//                     log-sum-exp / argmax state, writes logits when asked,
+//                     clears the slot and frees it                (redfree[r])
 //   residual warps    each owns 16 k16 steps of d for every m-tile; the fp16
 //                     h fragments of its columns stay in registers
 //   core warps        each owns kCL 64-column chunks of r_c'
 //   correction warps  each owns kCA 32-column chunks of r_r'
-// Each compute warp stores its 16 x nt partial tile and bumps a per-stage
-// counter; the last one sums the tiles in warp order (deterministic) and
-// signals the epilogue warp.  At the end every block writes one partial per token; the last block to
+// Each compute warp adds its 16 x nt partial logits into a fixed-point slot
+// tile (integer adds: same bits in any order) and signals the epilogue warp;
+// no warp ever waits for another to finish an m-tile.  At the end every block writes one partial per token; the last block to
 // finish (atomic ticket, no spinning) merges them into LSE, argmax and CE.
 // Every wait on an mbarrier is bounded (kWaitLimitNs); on expiry the block
 // raises ARCHEAD_STATUS_WAIT_TIMEOUT, skips the remaining work and drains its
@@ -48,13 +48,11 @@ constexpr int kEpiSlots = 4;     // 16 rows x 8 tokens / 32 lanes
 
 struct SmemView {
   uint8_t* stages;
-  float* red;          // [slots][nw_work][16 rows][nt]   per-warp partial tiles
-  float* tsum;         // [slots][nt][16 rows]            summed tile
+  unsigned long long* tsum;  // [slots][nt][16 rows] fixed-point logit sums
   uint64_t* full;      // [stages] producer -> compute warps (bytes landed)
   uint64_t* empty;     // [stages] compute warps -> producer (stage read)
-  uint64_t* reduced;   // [slots]  last compute warp -> epilogue warp
+  uint64_t* reduced;   // [slots]  compute warps -> epilogue warp
   uint64_t* redfree;   // [slots]  epilogue warp -> compute warps
-  int* arrivals;       // [slots]  compute warps done with the slot
   int* flags;          // [0] abort
 };
 
@@ -62,14 +60,12 @@ __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams&
   SmemView v;
   const size_t tile = static_cast<size_t>(p.nt) * 16;
   v.stages = smem;
-  v.red = reinterpret_cast<float*>(smem + static_cast<size_t>(p.stages) * p.mblk_bytes);
-  v.tsum = v.red + static_cast<size_t>(p.slots) * p.nw_work * tile;
+  v.tsum = reinterpret_cast<unsigned long long*>(smem + static_cast<size_t>(p.stages) * p.mblk_bytes);
   v.full = reinterpret_cast<uint64_t*>(v.tsum + static_cast<size_t>(p.slots) * tile);
   v.empty = v.full + p.stages;
   v.reduced = v.empty + p.stages;
   v.redfree = v.reduced + p.slots;
-  v.arrivals = reinterpret_cast<int*>(v.redfree + p.slots);
-  v.flags = v.arrivals + p.slots;
+  v.flags = reinterpret_cast<int*>(v.redfree + p.slots);
   return v;
 }
 
@@ -156,65 +152,42 @@ __device__ __forceinline__ float quad_sum(float v) {
   return v;
 }
 
-// Partial tile of one warp for one stage, [16 rows][nt] (row-major, so a
-// lane's two token columns are one 8-byte store and a warp's stores hit
-// distinct banks).
-__device__ __forceinline__ void store_partial(const SmemView& sv, const DecodeParams& p, int s, int cw, int lane,
-                                              const float (&acc)[4]) {
+// Logit partial sums of the compute warps meet in a fixed-point tile: each
+// value is rounded to a multiple of 2^-32 (error <= 2^-33, far below the
+// logit tolerance) and added as a 64-bit integer.  Integer addition is
+// associative, so the tile holds the same bits whatever the order in which the
+// warps arrive.  |partial| < 2^31 is assumed (the conversion saturates).
+constexpr float kFixScale = 4294967296.0f;   // 2^32
+
+__device__ __forceinline__ void add_partial(const SmemView& sv, const DecodeParams& p, int r, int lane,
+                                            const float (&acc)[4]) {
   const int gr = lane >> 2, cc = lane & 3;
-  const int nt = p.nt;
-  float* r = sv.red + (static_cast<size_t>(s) * p.nw_work + cw) * nt * 16;
+  unsigned long long* tile = sv.tsum + static_cast<size_t>(r) * p.nt * 16;
   const int t0 = 2 * cc;
-  if ((nt & 1) == 0 && t0 < nt) {
-    // nt even: gr * nt + t0 is even, so the 8-byte stores are aligned
-    *reinterpret_cast<float2*>(r + gr * nt + t0) = make_float2(acc[0], acc[1]);
-    *reinterpret_cast<float2*>(r + (gr + 8) * nt + t0) = make_float2(acc[2], acc[3]);
-  } else {
-    if (t0 < nt) {
-      r[gr * nt + t0] = acc[0];
-      r[(gr + 8) * nt + t0] = acc[2];
-    }
-    if (t0 + 1 < nt) {
-      r[gr * nt + t0 + 1] = acc[1];
-      r[(gr + 8) * nt + t0 + 1] = acc[3];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int t = t0 + j;
+    if (t < p.nt) {
+      const long long lo = __float2ll_rn(acc[j] * kFixScale);
+      const long long hi = __float2ll_rn(acc[2 + j] * kFixScale);
+      atomicAdd(tile + t * 16 + gr, static_cast<unsigned long long>(lo));
+      atomicAdd(tile + t * 16 + gr + 8, static_cast<unsigned long long>(hi));
     }
   }
 }
 
-// After a compute warp has stored its partial tile in slot s: count it, and
-// if it is the last of the nw_work warps, sum the tiles in warp order (fixed,
-// so results are deterministic) into tsum[s] and hand the slot to the
-// epilogue warp.  No warp ever waits here.
-__device__ __forceinline__ void finish_slot(const SmemView& sv, const DecodeParams& p, int s, int lane) {
+// End of one m-tile for a compute warp: release the stage buffer, add the
+// partial logits into slot r (after the epilogue has drained the slot's
+// previous use) and report to the epilogue warp.
+__device__ __forceinline__ void finish_mtile(const SmemView& sv, const DecodeParams& p, int i, int s, int lane,
+                                             const float (&acc)[4]) {
   __syncwarp();
-  int prev = 0;
-  if (lane == 0) {
-    __threadfence_block();
-    prev = atomicAdd(&sv.arrivals[s], 1);
-  }
-  prev = __shfl_sync(0xffffffffu, prev, 0);
-  if (prev != p.nw_work - 1) return;
-  if (lane == 0) sv.arrivals[s] = 0;
+  if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
+  const int r = i % p.slots;
+  if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
+  add_partial(sv, p, r, lane, acc);
   __syncwarp();
-  __threadfence_block();
-  const int nt = p.nt, nel = 16 * nt;
-  const float* red = sv.red + static_cast<size_t>(s) * p.nw_work * nel;
-  float* out = sv.tsum + static_cast<size_t>(s) * nel;
-  for (int e = lane; e < nel; e += 32) {          // e = t * 16 + row
-    const int src = (e & 15) * nt + (e >> 4);
-    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-    int w = 0;
-    for (; w + 4 <= p.nw_work; w += 4) {
-      y0 += red[(w + 0) * nel + src];
-      y1 += red[(w + 1) * nel + src];
-      y2 += red[(w + 2) * nel + src];
-      y3 += red[(w + 3) * nel + src];
-    }
-    for (; w < p.nw_work; ++w) y0 += red[w * nel + src];
-    out[e] = (y0 + y1) + (y2 + y3);
-  }
-  __syncwarp();
-  if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[s]));
+  if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[r]));
 }
 
 // ------------------------------------------------------------ residual warps
@@ -302,13 +275,7 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
       acc[2] *= unscale.x;
       acc[3] *= unscale.y;
     }
-    // The stage's bytes are consumed: give it back to the producer now.
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
-    const int r = i % p.slots;
-    if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
-    store_partial(sv, p, r, cw, lane, acc);
-    finish_slot(sv, p, r, lane);
+    finish_mtile(sv, p, i, s, lane, acc);
   }
 }
 
@@ -374,13 +341,7 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
         acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
       }
     }
-    // The stage's bytes are consumed: give it back to the producer now.
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
-    const int r = i % p.slots;
-    if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
-    store_partial(sv, p, r, cw, lane, acc);
-    finish_slot(sv, p, r, lane);
+    finish_mtile(sv, p, i, s, lane, acc);
   }
 }
 
@@ -439,13 +400,7 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
         acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
       }
     }
-    // The stage's bytes are consumed: give it back to the producer now.
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
-    const int r = i % p.slots;
-    if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
-    store_partial(sv, p, r, cw, lane, acc);
-    finish_slot(sv, p, r, lane);
+    finish_mtile(sv, p, i, s, lane, acc);
   }
 }
 
@@ -463,13 +418,16 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
   for (int i = 0; i < n_my; ++i) {
     const int r = i % p.slots;
     const bool ok = warp_wait(sv, &sv.reduced[r], (i / p.slots) & 1, p.status, lane);
-    const float* tsum = sv.tsum + static_cast<size_t>(r) * nel;
+    unsigned long long* tsum = sv.tsum + static_cast<size_t>(r) * nel;
     const int vbase = mtile_of(i) * kMT;
 #pragma unroll
     for (int k = 0; k < kEpiSlots; ++k) {
       const int e = lane + 32 * k;
-      if (ok && e < nel) {
-        const float y = tsum[e];
+      if (e < nel) {
+        const long long fx = static_cast<long long>(tsum[e]);
+        tsum[e] = 0ull;   // ready for the slot's next use
+        if (!ok) continue;
+        const float y = __ll2float_rn(fx) * (1.0f / kFixScale);
         const int row = e & 15, t = e >> 4;
         const int v = vbase + row;
         if (v < p.V) {
@@ -539,10 +497,10 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
       mbar_init(smem_addr(&sv.empty[s]), p.nw_work);
     }
     for (int r = 0; r < p.slots; ++r) {
-      mbar_init(smem_addr(&sv.reduced[r]), 1);
+      mbar_init(smem_addr(&sv.reduced[r]), p.nw_work);
       mbar_init(smem_addr(&sv.redfree[r]), 1);
-      sv.arrivals[r] = 0;
     }
+    for (int e = 0; e < p.slots * p.nt * 16; ++e) sv.tsum[e] = 0ull;
     sv.flags[0] = 0;
     mbar_fence_init();
   }
@@ -569,9 +527,9 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
 }
 
 size_t decode_smem_bytes(int stages, int slots, uint32_t mblk_bytes, int nw_work, int nt) {
-  return static_cast<size_t>(stages) * mblk_bytes + static_cast<size_t>(slots) * (nw_work + 1) * nt * 16 * 4 +
-         static_cast<size_t>(2) * stages * 8 + static_cast<size_t>(2) * slots * 8 + static_cast<size_t>(slots) * 4 +
-         16;
+  (void)nw_work;
+  return static_cast<size_t>(stages) * mblk_bytes + static_cast<size_t>(slots) * nt * 16 * 8 +
+         static_cast<size_t>(2) * stages * 8 + static_cast<size_t>(2) * slots * 8 + 16;
 }
 
 namespace {

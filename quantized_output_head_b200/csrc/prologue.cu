@@ -66,10 +66,18 @@ __global__ void __launch_bounds__(256) prologue_kernel(const PrologueParams p) {
         for (int e = 0; e < 16; ++e) acc = fmaf(static_cast<float>(c8[e]), hf[e], acc);
       } else {
         const uint16_t* sb = p.s_B + static_cast<size_t>(k) * ngB;
+        const int g0 = j / p.g_B;
+        if (g0 == (j + 15) / p.g_B) {   // the 16 columns share one group scale
+          float part = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float sc = __half2float(__ushort_as_half(sb[(j + e) / p.g_B]));
-          acc = fmaf(sc * static_cast<float>(c8[e]), hf[e], acc);
+          for (int e = 0; e < 16; ++e) part = fmaf(static_cast<float>(c8[e]), hf[e], part);
+          acc = fmaf(__half2float(__ushort_as_half(sb[g0])), part, acc);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float sc = __half2float(__ushort_as_half(sb[(j + e) / p.g_B]));
+            acc = fmaf(sc * static_cast<float>(c8[e]), hf[e], acc);
+          }
         }
       }
     }
