@@ -116,17 +116,9 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   for (int t0 = 0; t0 < T; t0 += kDecodeTokens) {
     dp.t0 = t0;
     dp.nt = (T - t0 < kDecodeTokens) ? (T - t0) : kDecodeTokens;
-    // Eight fixed-point logit slots (at most 8 KB); the rest of shared memory
-    // holds m-tile buffers (at most kMaxStages).
-    const int slots = 8;
-    const size_t fixed = decode_smem_bytes(0, slots, L.mblk_bytes, h->nw_work, dp.nt);
-    const size_t per_stage = decode_smem_bytes(1, slots, L.mblk_bytes, h->nw_work, dp.nt) - fixed;
-    int stages = static_cast<int>((static_cast<size_t>(h->smem_optin) - fixed) / per_stage);
-    stages = stages < kMaxStages ? stages : kMaxStages;
-    dp.stages = stages;
-    dp.slots = slots;
-    e = launch_decode(L.g_steps, dp, h->grid, decode_smem_bytes(stages, slots, L.mblk_bytes, h->nw_work, dp.nt),
-                      stream);
+    dp.slots = kSlots;
+    decode_smem_plan(dp, L.g_steps);
+    e = launch_decode(L.g_steps, dp, h->grid, decode_smem_bytes(dp), stream);
     if (e != cudaSuccess) return set_cuda_error(e);
   }
   if (h->ev_after != nullptr) {

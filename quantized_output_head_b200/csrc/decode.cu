@@ -6,35 +6,33 @@
 //          + s_L[v] sum_k L[v,k] z_c[t,k]                         core (Eq. 3)
 //          + s_A[v] sum_k A[v,k] z_r[t,k]                         correction (Eq. 4-6)
 // with z_c, z_r from the prologue kernel.  Codes are unpacked in registers to
-// exact fp16 values (bias + offset code) and multiplied on the tensor cores
-// (m16n8k16: vocabulary rows as M, tokens as N, fp32 accumulation).  The bias
-// is removed once per scale group in fp32 with a per-token constant computed
-// from the same fp16 operands, and the fp16 group / row scales multiply fp32
-// partial sums, so no scaled weight is ever rounded.  h enters as fp16 scaled
-// by a per-token power of two (exact for bf16 inputs); z as an fp16 pair
-// (high part + remainder) under its own power of two.
+// exact fp16 integers (offset code, plus 64 in half of the columns) and
+// multiplied on the tensor cores (m16n8k16: vocabulary rows as M, tokens as
+// N, fp32 accumulation).  The constant part is removed once per scale group in
+// fp32 with a per-token sum of the same fp16 operands, and the fp16 group /
+// row scales multiply fp32 partial sums, so no scaled weight is ever rounded.
+// h enters as fp16 scaled by a per-token power of two (exact for bf16 inputs);
+// z as an fp16 pair (high part + remainder) under its own power of two.
 //
-// Block organisation (one block per SM, persistent over m-tiles; no block-wide
-// barrier after setup):
-//   warp 0            producer: bulk-copies whole m-tile blocks HBM -> SMEM
-//                     into a ring of `stages` buffers (full[s]); a buffer is
-//                     refilled as soon as every compute warp has read it
-//                     (empty[s]), independent of the epilogue
-//   warp 1            epilogue: takes the summed 16 x nt logit tile of a slot
-//                     (reduced[r]), pushes each logit into a running
-//                     log-sum-exp / argmax state, writes logits when asked,
-//                     clears the slot and frees it                (redfree[r])
-//   residual warps    each owns 16 k16 steps of d for every m-tile; the fp16
-//                     h fragments of its columns stay in registers
-//   core warps        each owns kCL 64-column chunks of r_c'
-//   correction warps  each owns kCA 32-column chunks of r_r'
-// Each compute warp adds its 16 x nt partial logits into a fixed-point slot
-// tile (integer adds: same bits in any order) and signals the epilogue warp;
-// no warp ever waits for another to finish an m-tile.  At the end every block writes one partial per token; the last block to
-// finish (atomic ticket, no spinning) merges them into LSE, argmax and CE.
-// Every wait on an mbarrier is bounded (kWaitLimitNs); on expiry the block
-// raises ARCHEAD_STATUS_WAIT_TIMEOUT, skips the remaining work and drains its
-// copies before exiting.
+// Work split (one block per SM, persistent over the m-tiles m = block,
+// block + grid, ...): every compute warp owns a fixed slice of every m-tile
+// block, so it streams its own bytes:
+//   residual warps    16 k16 steps of d each; their fp16 h fragments stay in
+//                     registers for the whole launch
+//   core warps        kCL 64-column chunks of r_c' each
+//   correction warps  kCA 32-column chunks of r_r' each
+// Each compute warp prefetches its slice of the next kRing m-tiles into a
+// private shared-memory ring with cp.async (16 B per lane, L2 only) and waits
+// only on its own copies: no producer warp and no block-wide synchronisation.
+// After an m-tile the warp adds its 16 x nt partial logits into a fixed-point
+// slot tile (int64, shared atomics; identical bits in any order) and arrives
+// on reduced[r].  Warp 0, the epilogue, takes each finished tile, pushes the
+// logits into a running log-sum-exp / argmax state, writes logits when asked,
+// clears the slot and frees it (redfree[r]).  At the end every block writes one
+// partial per token; the last block to finish (atomic ticket, no spinning)
+// merges them into LSE, argmax and CE.  Every mbarrier wait is bounded
+// (kWaitLimitNs); on expiry the block raises ARCHEAD_STATUS_WAIT_TIMEOUT and
+// skips the remaining work.
 #include <cuda_runtime.h>
 
 #include "device.cuh"
@@ -47,23 +45,18 @@ namespace {
 constexpr int kEpiSlots = 4;     // 16 rows x 8 tokens / 32 lanes
 
 struct SmemView {
-  uint8_t* stages;
-  unsigned long long* tsum;  // [slots][nt][16 rows] fixed-point logit sums
-  uint64_t* full;      // [stages] producer -> compute warps (bytes landed)
-  uint64_t* empty;     // [stages] compute warps -> producer (stage read)
-  uint64_t* reduced;   // [slots]  compute warps -> epilogue warp
-  uint64_t* redfree;   // [slots]  epilogue warp -> compute warps
-  int* flags;          // [0] abort
+  uint8_t* rings;                // per compute warp: kRing slices
+  unsigned long long* tsum;      // [slots][nt][16 rows] fixed-point logit sums
+  uint64_t* reduced;             // [slots] compute warps -> epilogue warp
+  uint64_t* redfree;             // [slots] epilogue warp -> compute warps
+  int* flags;                    // [0] abort
 };
 
 __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams& p) {
   SmemView v;
-  const size_t tile = static_cast<size_t>(p.nt) * 16;
-  v.stages = smem;
-  v.tsum = reinterpret_cast<unsigned long long*>(smem + static_cast<size_t>(p.stages) * p.mblk_bytes);
-  v.full = reinterpret_cast<uint64_t*>(v.tsum + static_cast<size_t>(p.slots) * tile);
-  v.empty = v.full + p.stages;
-  v.reduced = v.empty + p.stages;
+  v.rings = smem;
+  v.tsum = reinterpret_cast<unsigned long long*>(smem + p.ring_bytes);
+  v.reduced = reinterpret_cast<uint64_t*>(v.tsum + static_cast<size_t>(p.slots) * p.nt * 16);
   v.redfree = v.reduced + p.slots;
   v.flags = reinterpret_cast<int*>(v.redfree + p.slots);
   return v;
@@ -87,34 +80,17 @@ __device__ __forceinline__ bool warp_wait(const SmemView& sv, uint64_t* bar, uin
   return ok;
 }
 
-__device__ __forceinline__ int mtile_of(int i) { return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x); }
+__device__ __forceinline__ int mtile_of(int i) {
+  return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+}
 
-// ----------------------------------------------------------------- producer
-__device__ void producer(const DecodeParams& p, const SmemView& sv, int n_my) {
-  const int S = p.stages;
-  int issued = 0;
-  for (int i = 0; i < n_my; ++i) {
-    const int s = i % S;
-    const int u = i / S;
-    if (aborted(sv)) break;
-    if (u > 0 && !mbar_wait(smem_addr(&sv.empty[s]), (u - 1) & 1)) {
-      raise_timeout(sv, p.status);
-      break;
-    }
-    const uint32_t full = smem_addr(&sv.full[s]);
-    mbar_arrive_expect_tx(full, p.mblk_bytes);
-    const uint8_t* src = p.mtiles + static_cast<size_t>(mtile_of(i)) * p.mblk_bytes;
-    const uint32_t dst = smem_addr(sv.stages + static_cast<size_t>(s) * p.mblk_bytes);
-    for (uint32_t off = 0; off < p.mblk_bytes; off += 16384u) {
-      const uint32_t n = min(16384u, p.mblk_bytes - off);
-      bulk_copy_g2s(dst + off, src + off, n, full);
-    }
-    ++issued;
-  }
-  // Every issued copy must have landed before this block may exit.
-  for (int i = max(0, issued - S); i < issued; ++i) {
-    if (!mbar_wait(smem_addr(&sv.full[i % S]), (i / S) & 1)) raise_timeout(sv, p.status);
-  }
+__device__ __forceinline__ const uint8_t* mtile_block(const DecodeParams& p, int i) {
+  return p.mtiles + static_cast<size_t>(mtile_of(i)) * p.mblk_bytes;
+}
+
+// Copy `bytes` (a multiple of 16) from global to shared memory, 16 B per lane.
+__device__ __forceinline__ void warp_copy(uint8_t* dst, const uint8_t* src, uint32_t bytes, int lane) {
+  for (uint32_t o = lane * 16u; o < bytes; o += 512u) cp_async16(smem_addr(dst + o), src + o);
 }
 
 // B-operand fragment (16 x 8, column = token) from the fp16 row of token gr:
@@ -132,7 +108,7 @@ __device__ __forceinline__ void load_b_frag_f16(const uint16_t* base, int k0, in
   }
 }
 
-// sum over the fp16 pair of bias_lo * (x + y) for b0 and bias_hi * (x + y) for b1.
+// bias_lo * (x + y) over the pair b0 plus bias_hi * (x + y) over the pair b1.
 __device__ __forceinline__ float bias_dot(uint32_t b0, uint32_t b1, float bias_lo, float bias_hi) {
   const float2 f0 = half2_bits_to_float2(b0);
   const float2 f1 = half2_bits_to_float2(b1);
@@ -163,10 +139,9 @@ __device__ __forceinline__ void add_partial(const SmemView& sv, const DecodePara
                                             const float (&acc)[4]) {
   const int gr = lane >> 2, cc = lane & 3;
   unsigned long long* tile = sv.tsum + static_cast<size_t>(r) * p.nt * 16;
-  const int t0 = 2 * cc;
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const int t = t0 + j;
+    const int t = 2 * cc + j;
     if (t < p.nt) {
       const long long lo = __float2ll_rn(acc[j] * kFixScale);
       const long long hi = __float2ll_rn(acc[2 + j] * kFixScale);
@@ -176,13 +151,10 @@ __device__ __forceinline__ void add_partial(const SmemView& sv, const DecodePara
   }
 }
 
-// End of one m-tile for a compute warp: release the stage buffer, add the
-// partial logits into slot r (after the epilogue has drained the slot's
-// previous use) and report to the epilogue warp.
-__device__ __forceinline__ void finish_mtile(const SmemView& sv, const DecodeParams& p, int i, int s, int lane,
+// End of m-tile i for a compute warp: add its partial logits into slot r
+// (after the epilogue has drained the slot's previous use) and report.
+__device__ __forceinline__ void finish_mtile(const SmemView& sv, const DecodeParams& p, int i, int lane,
                                              const float (&acc)[4]) {
-  __syncwarp();
-  if (lane == 0) mbar_arrive(smem_addr(&sv.empty[s]));
   const int r = i % p.slots;
   if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
   add_partial(sv, p, r, lane, acc);
@@ -191,17 +163,49 @@ __device__ __forceinline__ void finish_mtile(const SmemView& sv, const DecodePar
 }
 
 // ------------------------------------------------------------ residual warps
+// Ring slice: [kCRes chunks x 512 B of codes][groups x 32 B of scales].
+struct ResSlice {
+  int chunk0, nchunks;     // residual chunks of this warp
+  int grp0, ng;            // scale groups its columns touch
+};
+
+__device__ __forceinline__ ResSlice res_slice(const DecodeParams& p, int wres) {
+  ResSlice r;
+  r.chunk0 = wres * kCRes;
+  r.nchunks = min(kCRes, p.n_res - r.chunk0);
+  const int col0 = r.chunk0 * kResChunkK, col1 = col0 + r.nchunks * kResChunkK - 1;
+  r.grp0 = col0 >> (p.g_steps_log2 + 4);
+  r.ng = (col1 >> (p.g_steps_log2 + 4)) - r.grp0 + 1;
+  return r;
+}
+
+__device__ __forceinline__ void issue_res(const DecodeParams& p, const ResSlice& rs, uint8_t* slot, int i, int lane) {
+  const uint8_t* blk = mtile_block(p, i);
+  warp_copy(slot, blk + p.off_res + rs.chunk0 * kResChunkBytes, rs.nchunks * kResChunkBytes, lane);
+  warp_copy(slot + kCRes * kResChunkBytes, blk + p.off_sres + rs.grp0 * kSresGroupBytes, rs.ng * kSresGroupBytes,
+            lane);
+}
+
 // G = k16 steps per scale group within the warp's 16 steps (16 when a group
 // spans the whole warp range or more).
 template <int G>
-__device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wres, int cw, int lane) {
+__device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wres, int lane) {
   constexpr int kNG = 16 / G;    // local scale groups
   const int gr = lane >> 2;
-  const int S = p.stages;
+  const ResSlice rs = res_slice(p, wres);
+  const uint32_t sbytes = p.res_slice_bytes;
+  uint8_t* ring = sv.rings + static_cast<size_t>(wres) * kRing * sbytes;
+  // Start streaming before the prologue's results are needed.
+#pragma unroll
+  for (int k = 0; k < kRing; ++k) {
+    if (k < n_my) issue_res(p, rs, ring + k * sbytes, k, lane);
+    cp_async_commit();
+  }
+  grid_dependency_wait();
   const bool tok = gr < p.nt;
   float hs = 0.f;
   if (tok) hs = ldexpf(1.f, kScaleExp - p.escale[p.t0 + gr]);
-  // fp16 h fragments of this warp's columns, and the bias constant of each
+  // fp16 h fragments of this warp's columns, and the constant-part sum of each
   // local group for token gr.
   uint32_t hf[kCRes][4][2];
   float cg[kNG];
@@ -210,12 +214,11 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
   const uint16_t* hrow = p.hidden + static_cast<size_t>(p.t0 + (tok ? gr : 0)) * p.d;
 #pragma unroll
   for (int c = 0; c < kCRes; ++c) {
-    const int chunk = wres * kCRes + c;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
       uint32_t b[2] = {0u, 0u};
-      if (tok && chunk < p.n_res) {
-        const uint16_t* r = hrow + chunk * kResChunkK + s * 16 + 2 * (lane & 3);
+      if (tok && c < rs.nchunks) {
+        const uint16_t* r = hrow + (rs.chunk0 + c) * kResChunkK + s * 16 + 2 * (lane & 3);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const uint32_t bits = *reinterpret_cast<const uint32_t*>(r + 8 * j);
@@ -233,21 +236,22 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
 #pragma unroll
   for (int g = 0; g < kNG; ++g) cgc[g] = column_pair(quad_sum(cg[g]), lane);
   const float2 unscale = column_pair(tok ? 1.f / hs : 0.f, lane);
-  const int last_step = min(16, (p.n_res - wres * kCRes) * 4) - 1;
+  const int last_step = rs.nchunks * 4 - 1;
   const int step0 = wres * 16;
 
   for (int i = 0; i < n_my; ++i) {
-    const int s = i % S;
+    uint8_t* slot = ring + (i % kRing) * sbytes;
+    cp_async_wait<kRing - 1>();
+    __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (warp_wait(sv, &sv.full[s], (i / S) & 1, p.status, lane)) {
-      const uint8_t* stg = sv.stages + static_cast<size_t>(s) * p.mblk_bytes;
+    {
       float t0[4] = {0.f, 0.f, 0.f, 0.f};
       float t1[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint8_t* sres = slot + kCRes * kResChunkBytes;
 #pragma unroll
       for (int c = 0; c < kCRes; ++c) {
-        const int chunk = wres * kCRes + c;
-        if (chunk < p.n_res) {
-          const uint4 nib = *reinterpret_cast<const uint4*>(stg + p.off_res + chunk * kResChunkBytes + lane * 16);
+        if (c < rs.nchunks) {
+          const uint4 nib = *reinterpret_cast<const uint4*>(slot + c * kResChunkBytes + lane * 16);
           const uint32_t wv[4] = {nib.x, nib.y, nib.z, nib.w};
 #pragma unroll
           for (int st = 0; st < 4; ++st) {
@@ -258,9 +262,9 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
             unpack_int4_biased(wv[st], a);
             mma_f16_16816(tmp, a, hf[c][st][0], hf[c][st][1]);
             if ((step + 1) % G == 0 || (G == 16 && step == last_step)) {
-              const int grp = (step0 + step) >> p.g_steps_log2;
-              const float2 sc = half2_bits_to_float2(
-                  *reinterpret_cast<const uint32_t*>(stg + p.off_sres + grp * kSresGroupBytes + gr * 4));
+              const int grp = ((step0 + step) >> p.g_steps_log2) - rs.grp0;
+              const float2 sc =
+                  half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(sres + grp * kSresGroupBytes + gr * 4));
               acc[0] = fmaf(sc.x, tmp[0] - cgc[lg].x, acc[0]);
               acc[1] = fmaf(sc.x, tmp[1] - cgc[lg].y, acc[1]);
               acc[2] = fmaf(sc.y, tmp[2] - cgc[lg].x, acc[2]);
@@ -275,14 +279,36 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
       acc[2] *= unscale.x;
       acc[3] *= unscale.y;
     }
-    finish_mtile(sv, p, i, s, lane, acc);
+    __syncwarp();   // every lane is done reading the slot
+    if (i + kRing < n_my) issue_res(p, rs, slot, i + kRing, lane);
+    cp_async_commit();
+    finish_mtile(sv, p, i, lane, acc);
   }
+  cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------- core warps
-__device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wl, int cw, int lane) {
+// Ring slice: [kCL x 512 B nibbles][kCL x 128 B fifth bits][32 B s_L].
+__device__ __forceinline__ void issue_core(const DecodeParams& p, int chunk0, int nch, uint8_t* slot, int i,
+                                           int lane) {
+  const uint8_t* blk = mtile_block(p, i);
+  warp_copy(slot, blk + p.off_Lnib + chunk0 * kLNibChunkBytes, nch * kLNibChunkBytes, lane);
+  warp_copy(slot + kCL * kLNibChunkBytes, blk + p.off_Lhi + chunk0 * kLHiChunkBytes, nch * kLHiChunkBytes, lane);
+  warp_copy(slot + kCL * (kLNibChunkBytes + kLHiChunkBytes), blk + p.off_sL, 32, lane);
+}
+
+__device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wl, int lane) {
   const int gr = lane >> 2;
-  const int S = p.stages;
+  const int chunk0 = wl * kCL;
+  const int nch = min(kCL, p.n_L - chunk0);
+  const uint32_t sbytes = p.core_slice_bytes;
+  uint8_t* ring = sv.rings + p.core_ring_off + static_cast<size_t>(wl) * kRing * sbytes;
+#pragma unroll
+  for (int k = 0; k < kRing; ++k) {
+    if (k < n_my) issue_core(p, chunk0, nch, ring + k * sbytes, k, lane);
+    cp_async_commit();
+  }
+  grid_dependency_wait();
   const bool tok = gr < p.nt;
   uint32_t zf[kCL][4][2][2];
   float cb = 0.f;
@@ -290,11 +316,10 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
   const uint16_t* zl = p.zlo + static_cast<size_t>(p.t0 + (tok ? gr : 0)) * p.Kz;
 #pragma unroll
   for (int c = 0; c < kCL; ++c) {
-    const int chunk = wl * kCL + c;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      const int k0 = chunk * kLChunkK + s * 16;
-      const bool ok = tok && chunk < p.n_L;
+      const int k0 = (chunk0 + c) * kLChunkK + s * 16;
+      const bool ok = tok && c < nch;
       load_b_frag_f16(zh, k0, lane, ok, zf[c][s][0][0], zf[c][s][0][1]);
       load_b_frag_f16(zl, k0, lane, ok, zf[c][s][1][0], zf[c][s][1][1]);
       cb += bias_dot(zf[c][s][0][0], zf[c][s][0][1], kBiasLo + 16.f, kBiasHi + 16.f);
@@ -306,49 +331,66 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
   const float2 unscale = column_pair(zs, lane);
 
   for (int i = 0; i < n_my; ++i) {
-    const int s = i % S;
+    uint8_t* slot = ring + (i % kRing) * sbytes;
+    cp_async_wait<kRing - 1>();
+    __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (warp_wait(sv, &sv.full[s], (i / S) & 1, p.status, lane)) {
-      const uint8_t* stg = sv.stages + static_cast<size_t>(s) * p.mblk_bytes;
-      bool any = false;
 #pragma unroll
-      for (int c = 0; c < kCL; ++c) {
-        const int chunk = wl * kCL + c;
-        if (chunk < p.n_L) {
-          any = true;
-          const uint4 nib = *reinterpret_cast<const uint4*>(stg + p.off_Lnib + chunk * kLNibChunkBytes + lane * 16);
-          const uint32_t hb = *reinterpret_cast<const uint32_t*>(stg + p.off_Lhi + chunk * kLHiChunkBytes + lane * 4);
-          uint32_t a[4];
-          unpack_int5_biased<0>(nib.x, hb, a);
-          mma_f16_16816(acc, a, zf[c][0][0][0], zf[c][0][0][1]);
-          mma_f16_16816(acc, a, zf[c][0][1][0], zf[c][0][1][1]);
-          unpack_int5_biased<1>(nib.y, hb, a);
-          mma_f16_16816(acc, a, zf[c][1][0][0], zf[c][1][0][1]);
-          mma_f16_16816(acc, a, zf[c][1][1][0], zf[c][1][1][1]);
-          unpack_int5_biased<2>(nib.z, hb, a);
-          mma_f16_16816(acc, a, zf[c][2][0][0], zf[c][2][0][1]);
-          mma_f16_16816(acc, a, zf[c][2][1][0], zf[c][2][1][1]);
-          unpack_int5_biased<3>(nib.w, hb, a);
-          mma_f16_16816(acc, a, zf[c][3][0][0], zf[c][3][0][1]);
-          mma_f16_16816(acc, a, zf[c][3][1][0], zf[c][3][1][1]);
-        }
-      }
-      if (any) {
-        const float2 sc = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(stg + p.off_sL + gr * 4));
-        acc[0] = (acc[0] - cbc.x) * (sc.x * unscale.x);
-        acc[1] = (acc[1] - cbc.y) * (sc.x * unscale.y);
-        acc[2] = (acc[2] - cbc.x) * (sc.y * unscale.x);
-        acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
+    for (int c = 0; c < kCL; ++c) {
+      if (c < nch) {
+        const uint4 nib = *reinterpret_cast<const uint4*>(slot + c * kLNibChunkBytes + lane * 16);
+        const uint32_t hb =
+            *reinterpret_cast<const uint32_t*>(slot + kCL * kLNibChunkBytes + c * kLHiChunkBytes + lane * 4);
+        uint32_t a[4];
+        unpack_int5_biased<0>(nib.x, hb, a);
+        mma_f16_16816(acc, a, zf[c][0][0][0], zf[c][0][0][1]);
+        mma_f16_16816(acc, a, zf[c][0][1][0], zf[c][0][1][1]);
+        unpack_int5_biased<1>(nib.y, hb, a);
+        mma_f16_16816(acc, a, zf[c][1][0][0], zf[c][1][0][1]);
+        mma_f16_16816(acc, a, zf[c][1][1][0], zf[c][1][1][1]);
+        unpack_int5_biased<2>(nib.z, hb, a);
+        mma_f16_16816(acc, a, zf[c][2][0][0], zf[c][2][0][1]);
+        mma_f16_16816(acc, a, zf[c][2][1][0], zf[c][2][1][1]);
+        unpack_int5_biased<3>(nib.w, hb, a);
+        mma_f16_16816(acc, a, zf[c][3][0][0], zf[c][3][0][1]);
+        mma_f16_16816(acc, a, zf[c][3][1][0], zf[c][3][1][1]);
       }
     }
-    finish_mtile(sv, p, i, s, lane, acc);
+    const float2 sc = half2_bits_to_float2(
+        *reinterpret_cast<const uint32_t*>(slot + kCL * (kLNibChunkBytes + kLHiChunkBytes) + gr * 4));
+    acc[0] = (acc[0] - cbc.x) * (sc.x * unscale.x);
+    acc[1] = (acc[1] - cbc.y) * (sc.x * unscale.y);
+    acc[2] = (acc[2] - cbc.x) * (sc.y * unscale.x);
+    acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
+    __syncwarp();
+    if (i + kRing < n_my) issue_core(p, chunk0, nch, slot, i + kRing, lane);
+    cp_async_commit();
+    finish_mtile(sv, p, i, lane, acc);
   }
+  cp_async_wait_all();
 }
 
 // ---------------------------------------------------------- correction warps
-__device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wa, int cw, int lane) {
+// Ring slice: [kCA x 512 B codes][32 B s_A].
+__device__ __forceinline__ void issue_corr(const DecodeParams& p, int chunk0, int nch, uint8_t* slot, int i,
+                                           int lane) {
+  const uint8_t* blk = mtile_block(p, i);
+  warp_copy(slot, blk + p.off_A + chunk0 * kAChunkBytes, nch * kAChunkBytes, lane);
+  warp_copy(slot + kCA * kAChunkBytes, blk + p.off_sA, 32, lane);
+}
+
+__device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wa, int lane) {
   const int gr = lane >> 2;
-  const int S = p.stages;
+  const int chunk0 = wa * kCA;
+  const int nch = min(kCA, p.n_A - chunk0);
+  const uint32_t sbytes = p.corr_slice_bytes;
+  uint8_t* ring = sv.rings + p.corr_ring_off + static_cast<size_t>(wa) * kRing * sbytes;
+#pragma unroll
+  for (int k = 0; k < kRing; ++k) {
+    if (k < n_my) issue_corr(p, chunk0, nch, ring + k * sbytes, k, lane);
+    cp_async_commit();
+  }
+  grid_dependency_wait();
   const bool tok = gr < p.nt;
   uint32_t zf[kCA][2][2][2];
   float cb = 0.f;
@@ -356,11 +398,10 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
   const uint16_t* zl = p.zlo + static_cast<size_t>(p.t0 + (tok ? gr : 0)) * p.Kz;
 #pragma unroll
   for (int c = 0; c < kCA; ++c) {
-    const int chunk = wa * kCA + c;
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
-      const int k0 = p.rcp + chunk * kAChunkK + s * 16;
-      const bool ok = tok && chunk < p.n_A;
+      const int k0 = p.rcp + (chunk0 + c) * kAChunkK + s * 16;
+      const bool ok = tok && c < nch;
       load_b_frag_f16(zh, k0, lane, ok, zf[c][s][0][0], zf[c][s][0][1]);
       load_b_frag_f16(zl, k0, lane, ok, zf[c][s][1][0], zf[c][s][1][1]);
       cb += bias_dot(zf[c][s][0][0], zf[c][s][0][1], kBiasLo + 128.f, kBiasLo + 128.f);
@@ -372,40 +413,40 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
   const float2 unscale = column_pair(zs, lane);
 
   for (int i = 0; i < n_my; ++i) {
-    const int s = i % S;
+    uint8_t* slot = ring + (i % kRing) * sbytes;
+    cp_async_wait<kRing - 1>();
+    __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (warp_wait(sv, &sv.full[s], (i / S) & 1, p.status, lane)) {
-      const uint8_t* stg = sv.stages + static_cast<size_t>(s) * p.mblk_bytes;
-      bool any = false;
 #pragma unroll
-      for (int c = 0; c < kCA; ++c) {
-        const int chunk = wa * kCA + c;
-        if (chunk < p.n_A) {
-          any = true;
-          const uint4 w = *reinterpret_cast<const uint4*>(stg + p.off_A + chunk * kAChunkBytes + lane * 16);
-          uint32_t a[4];
-          unpack_int8_biased(w.x, w.y, a);
-          mma_f16_16816(acc, a, zf[c][0][0][0], zf[c][0][0][1]);
-          mma_f16_16816(acc, a, zf[c][0][1][0], zf[c][0][1][1]);
-          unpack_int8_biased(w.z, w.w, a);
-          mma_f16_16816(acc, a, zf[c][1][0][0], zf[c][1][0][1]);
-          mma_f16_16816(acc, a, zf[c][1][1][0], zf[c][1][1][1]);
-        }
-      }
-      if (any) {
-        const float2 sc = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(stg + p.off_sA + gr * 4));
-        acc[0] = (acc[0] - cbc.x) * (sc.x * unscale.x);
-        acc[1] = (acc[1] - cbc.y) * (sc.x * unscale.y);
-        acc[2] = (acc[2] - cbc.x) * (sc.y * unscale.x);
-        acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
+    for (int c = 0; c < kCA; ++c) {
+      if (c < nch) {
+        const uint4 w = *reinterpret_cast<const uint4*>(slot + c * kAChunkBytes + lane * 16);
+        uint32_t a[4];
+        unpack_int8_biased(w.x, w.y, a);
+        mma_f16_16816(acc, a, zf[c][0][0][0], zf[c][0][0][1]);
+        mma_f16_16816(acc, a, zf[c][0][1][0], zf[c][0][1][1]);
+        unpack_int8_biased(w.z, w.w, a);
+        mma_f16_16816(acc, a, zf[c][1][0][0], zf[c][1][0][1]);
+        mma_f16_16816(acc, a, zf[c][1][1][0], zf[c][1][1][1]);
       }
     }
-    finish_mtile(sv, p, i, s, lane, acc);
+    const float2 sc =
+        half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(slot + kCA * kAChunkBytes + gr * 4));
+    acc[0] = (acc[0] - cbc.x) * (sc.x * unscale.x);
+    acc[1] = (acc[1] - cbc.y) * (sc.x * unscale.y);
+    acc[2] = (acc[2] - cbc.x) * (sc.y * unscale.x);
+    acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
+    __syncwarp();
+    if (i + kRing < n_my) issue_corr(p, chunk0, nch, slot, i + kRing, lane);
+    cp_async_commit();
+    finish_mtile(sv, p, i, lane, acc);
   }
+  cp_async_wait_all();
 }
 
 // ------------------------------------------------------------ epilogue warp
 __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int lane) {
+  grid_dependency_wait();   // the workspace is shared with the previous launch
   const int nel = 16 * p.nt;
   LseState st[kEpiSlots];
   int target[kEpiSlots];
@@ -492,44 +533,46 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
   const int n_my = (p.n_mtiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < p.stages; ++s) {
-      mbar_init(smem_addr(&sv.full[s]), 1);
-      mbar_init(smem_addr(&sv.empty[s]), p.nw_work);
-    }
     for (int r = 0; r < p.slots; ++r) {
       mbar_init(smem_addr(&sv.reduced[r]), p.nw_work);
       mbar_init(smem_addr(&sv.redfree[r]), 1);
     }
-    for (int e = 0; e < p.slots * p.nt * 16; ++e) sv.tsum[e] = 0ull;
     sv.flags[0] = 0;
     mbar_fence_init();
   }
+  for (int e = threadIdx.x; e < p.slots * p.nt * 16; e += blockDim.x) sv.tsum[e] = 0ull;
   __syncthreads();
 
   if (warp == 0) {
-    if (lane == 0) producer(p, sv, n_my);
-    return;
-  }
-  // Everything below reads the prologue's output or the workspace.
-  grid_dependency_wait();
-  if (warp == 1) {
     epilogue_warp(p, sv, n_my, lane);
     return;
   }
-  const int cw = warp - 2;
+  const int cw = warp - 1;
   if (cw < p.nw_res) {
-    residual_warp<G>(p, sv, n_my, cw, cw, lane);
+    residual_warp<G>(p, sv, n_my, cw, lane);
   } else if (cw < p.nw_res + p.nw_L) {
-    core_warp(p, sv, n_my, cw - p.nw_res, cw, lane);
+    core_warp(p, sv, n_my, cw - p.nw_res, lane);
   } else if (cw < p.nw_work) {
-    correction_warp(p, sv, n_my, cw - p.nw_res - p.nw_L, cw, lane);
+    correction_warp(p, sv, n_my, cw - p.nw_res - p.nw_L, lane);
   }
 }
 
-size_t decode_smem_bytes(int stages, int slots, uint32_t mblk_bytes, int nw_work, int nt) {
-  (void)nw_work;
-  return static_cast<size_t>(stages) * mblk_bytes + static_cast<size_t>(slots) * nt * 16 * 8 +
-         static_cast<size_t>(2) * stages * 8 + static_cast<size_t>(2) * slots * 8 + 16;
+// Shared-memory plan of one launch (host side): ring slices per role.
+void decode_smem_plan(DecodeParams& p, int g_steps) {
+  const int g = g_steps * 16;
+  const int span = kCRes * kResChunkK;                       // columns of one residual warp
+  const int ng = (g >= span) ? 2 : span / g;                 // groups a warp's columns can touch
+  p.res_slice_bytes = kCRes * kResChunkBytes + ng * kSresGroupBytes;
+  p.core_slice_bytes = kCL * (kLNibChunkBytes + kLHiChunkBytes) + 32;
+  p.corr_slice_bytes = kCA * kAChunkBytes + 32;
+  p.core_ring_off = static_cast<uint32_t>(p.nw_res) * kRing * p.res_slice_bytes;
+  p.corr_ring_off = p.core_ring_off + static_cast<uint32_t>(p.nw_L) * kRing * p.core_slice_bytes;
+  p.ring_bytes = p.corr_ring_off + static_cast<uint32_t>(p.nw_A) * kRing * p.corr_slice_bytes;
+}
+
+size_t decode_smem_bytes(const DecodeParams& p) {
+  return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nt * 16 * 8 +
+         static_cast<size_t>(2) * p.slots * 8 + 16;
 }
 
 namespace {
@@ -556,7 +599,7 @@ cudaError_t decode_set_attributes(int g_steps, size_t smem) {
 cudaError_t launch_decode(int g_steps, const DecodeParams& p, int grid, size_t smem, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3((2 + p.nw_work) * 32);
+  cfg.blockDim = dim3((1 + p.nw_work) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -69,6 +69,16 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
       : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared through L2 only (LSU path); the
+// calling thread tracks completion with commit / wait groups.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // ------------------------------------------------- programmatic launch order
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() {
@@ -109,47 +119,57 @@ __device__ __forceinline__ uint32_t shift_to(uint32_t x) {
   else return x << (-kShift);
 }
 
-// fp16 fragment unpacking with a bias.  A 4-bit field placed under the fp16
-// exponent of 1024 (0x6400, mantissa step 1 at bit 0) reads as 1024 + u; the
-// same field at bits 4-7 under the exponent of 64 (0x5400, mantissa step 1 at
-// bit 4) reads as 64 + u.  Both are exact, so the tensor core sees
-// (bias + code + offset) and the bias is removed once per scale group in fp32.
-// Per k16 step the A columns 2cc, 2cc+1 (registers a0, a1) carry the 1024 bias
-// and the columns 2cc+8, 2cc+9 (a2, a3) the 64 bias.
-constexpr float kBiasLo = 1024.f;
+// fp16 fragment unpacking.  A 4-bit field placed under the fp16 exponent of
+// 1024 (0x6400, mantissa step 1 at bit 0) reads as 1024 + u, and one exact fp16
+// subtraction of 1024 leaves u; the field at bits 4-7 under the exponent of 64
+// (0x5400, mantissa step 1 at bit 4) reads as 64 + u with no shift at all.  So
+// per k16 step the A columns 2cc, 2cc+1 (registers a0, a1) carry the bare
+// offset code and the columns 2cc+8, 2cc+9 (a2, a3) the code plus 64; the
+// tensor core sees exact small integers and the constant part (offset, and
+// 64 for the high columns) is removed once per scale group in fp32.
+constexpr float kBiasLo = 0.f;
 constexpr float kBiasHi = 64.f;
+constexpr uint32_t kHalf1024x2 = 0x64006400u;
+
+__device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
 
 // Offset-binary INT4 word: nibbles of (a0, a2, a1, a3) at bits 0, 4, 8, 12 (low
 // columns) and 16, 20, 24, 28 (high columns).
 __device__ __forceinline__ void unpack_int4_biased(uint32_t w, uint32_t (&a)[4]) {
   const uint32_t w8 = w >> 8;
-  a[0] = and_or<0x000F000Fu, 0x64006400u>(w);
+  a[0] = hsub2_bits(and_or<0x000F000Fu, 0x64006400u>(w), kHalf1024x2);
   a[2] = and_or<0x00F000F0u, 0x54005400u>(w);
-  a[1] = and_or<0x000F000Fu, 0x64006400u>(w8);
+  a[1] = hsub2_bits(and_or<0x000F000Fu, 0x64006400u>(w8), kHalf1024x2);
   a[3] = and_or<0x00F000F0u, 0x54005400u>(w8);
 }
 
 // Offset-binary INT5 codes of k16 step S: low nibbles as for INT4 in w, the
 // fifth bit of the low / high column of position q (q = 0..3 for a0, a2, a1,
-// a3) at bits 4S+q / 4S+q+16 of hb.  The fifth bit goes to bit 4 (1024 bias)
-// or bit 8 (64 bias, whose mantissa step is at bit 4).
+// a3) at bits 4S+q / 4S+q+16 of hb.  The fifth bit goes to bit 4 (under 1024)
+// or bit 8 (under 64, whose mantissa step is at bit 4).
 template <int S>
 __device__ __forceinline__ void unpack_int5_biased(uint32_t w, uint32_t hb, uint32_t (&a)[4]) {
   const uint32_t w8 = w >> 8;
-  a[0] = and_or_r(shift_to<4 * S + 0 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w));
+  a[0] = hsub2_bits(and_or_r(shift_to<4 * S + 0 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w)),
+                    kHalf1024x2);
   a[2] = and_or_r(shift_to<4 * S + 1 - 8>(hb), 0x01000100u, and_or<0x00F000F0u, 0x54005400u>(w));
-  a[1] = and_or_r(shift_to<4 * S + 2 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w8));
+  a[1] = hsub2_bits(and_or_r(shift_to<4 * S + 2 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w8)),
+                    kHalf1024x2);
   a[3] = and_or_r(shift_to<4 * S + 3 - 8>(hb), 0x01000100u, and_or<0x00F000F0u, 0x54005400u>(w8));
 }
 
 // Offset-binary INT8 bytes (row gr col c, row gr col c+1, row gr+8 col c,
 // row gr+8 col c+1) of w0 (columns c) and w1 (columns c+8): one byte permute
-// per pair puts each byte under the exponent of 1024.
+// per pair puts each byte under the exponent of 1024, one subtraction removes it.
 __device__ __forceinline__ void unpack_int8_biased(uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
-  a[0] = __byte_perm(w0, 0x64646464u, 0x4140u);
-  a[1] = __byte_perm(w0, 0x64646464u, 0x4342u);
-  a[2] = __byte_perm(w1, 0x64646464u, 0x4140u);
-  a[3] = __byte_perm(w1, 0x64646464u, 0x4342u);
+  a[0] = hsub2_bits(__byte_perm(w0, 0x64646464u, 0x4140u), kHalf1024x2);
+  a[1] = hsub2_bits(__byte_perm(w0, 0x64646464u, 0x4342u), kHalf1024x2);
+  a[2] = hsub2_bits(__byte_perm(w1, 0x64646464u, 0x4140u), kHalf1024x2);
+  a[3] = hsub2_bits(__byte_perm(w1, 0x64646464u, 0x4342u), kHalf1024x2);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {

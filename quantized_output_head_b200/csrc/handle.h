@@ -51,7 +51,8 @@ inline WsLayout ws_layout(const archead_handle& h, int T) {
 }
 
 // Kernel launchers and attributes (decode.cu, prologue.cu).
-size_t decode_smem_bytes(int stages, int slots, uint32_t mblk_bytes, int nw_work, int nt);
+void decode_smem_plan(DecodeParams& p, int g_steps);
+size_t decode_smem_bytes(const DecodeParams& p);
 cudaError_t decode_set_attributes(int g_steps, size_t smem);
 cudaError_t launch_decode(int g_steps, const DecodeParams& p, int grid, size_t smem, cudaStream_t stream);
 cudaError_t launch_prologue(const PrologueParams& p, cudaStream_t stream);

@@ -138,9 +138,17 @@ bool plan_decode(archead_handle* h, int smem_optin) {
   const int nw_L = (L.n_L + kCL - 1) / kCL;
   const int nw_A = (L.n_A + kCA - 1) / kCA;
   const int nw_work = nw_res + nw_L + nw_A;
-  if (2 + nw_work > kMaxDecodeWarps) return false;
-  // Two stages at the widest launch (8 tokens) must fit.
-  if (decode_smem_bytes(2, 2, L.mblk_bytes, nw_work, kDecodeTokens) > static_cast<size_t>(smem_optin)) return false;
+  if (1 + nw_work > kMaxDecodeWarps) return false;
+  // The rings and slots of the widest launch (8 tokens) must fit.
+  DecodeParams dp{};
+  dp.nw_res = nw_res;
+  dp.nw_L = nw_L;
+  dp.nw_A = nw_A;
+  dp.nw_work = nw_work;
+  dp.nt = kDecodeTokens;
+  dp.slots = kSlots;
+  decode_smem_plan(dp, L.g_steps);
+  if (decode_smem_bytes(dp) > static_cast<size_t>(smem_optin)) return false;
   h->nw_res = nw_res;
   h->nw_L = nw_L;
   h->nw_A = nw_A;
