@@ -88,11 +88,6 @@ __device__ __forceinline__ const uint8_t* mtile_block(const DecodeParams& p, int
   return p.mtiles + static_cast<size_t>(mtile_of(i)) * p.mblk_bytes;
 }
 
-// Copy `bytes` (a multiple of 16) from global to shared memory, 16 B per lane.
-__device__ __forceinline__ void warp_copy(uint8_t* dst, const uint8_t* src, uint32_t bytes, int lane) {
-  for (uint32_t o = lane * 16u; o < bytes; o += 512u) cp_async16(smem_addr(dst + o), src + o);
-}
-
 // B-operand fragment (16 x 8, column = token) from the fp16 row of token gr:
 // lane (gr, cc) holds rows k0 + 2cc, +1 and k0 + 2cc + 8, +9.
 __device__ __forceinline__ void load_b_frag_f16(const uint16_t* base, int k0, int lane, bool valid,
@@ -138,7 +133,7 @@ constexpr float kFixScale = 4294967296.0f;   // 2^32
 __device__ __forceinline__ void add_partial(const SmemView& sv, const DecodeParams& p, int r, int lane,
                                             const float (&acc)[4]) {
   const int gr = lane >> 2, cc = lane & 3;
-  unsigned long long* tile = sv.tsum + static_cast<size_t>(r) * p.nt * 16;
+  unsigned long long* tile = sv.tsum + r * p.nt * 16;
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     const int t = 2 * cc + j;
@@ -155,8 +150,8 @@ __device__ __forceinline__ void add_partial(const SmemView& sv, const DecodePara
 // (after the epilogue has drained the slot's previous use) and report.
 __device__ __forceinline__ void finish_mtile(const SmemView& sv, const DecodeParams& p, int i, int lane,
                                              const float (&acc)[4]) {
-  const int r = i % p.slots;
-  if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i / p.slots) - 1) & 1, p.status, lane);
+  const int r = i & (kSlots - 1);
+  if (i >= kSlots) warp_wait(sv, &sv.redfree[r], ((i / kSlots) - 1) & 1, p.status, lane);
   add_partial(sv, p, r, lane, acc);
   __syncwarp();
   if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[r]));
@@ -181,9 +176,50 @@ __device__ __forceinline__ ResSlice res_slice(const DecodeParams& p, int wres) {
 
 __device__ __forceinline__ void issue_res(const DecodeParams& p, const ResSlice& rs, uint8_t* slot, int i, int lane) {
   const uint8_t* blk = mtile_block(p, i);
-  warp_copy(slot, blk + p.off_res + rs.chunk0 * kResChunkBytes, rs.nchunks * kResChunkBytes, lane);
-  warp_copy(slot + kCRes * kResChunkBytes, blk + p.off_sres + rs.grp0 * kSresGroupBytes, rs.ng * kSresGroupBytes,
-            lane);
+  const uint8_t* codes = blk + p.off_res + rs.chunk0 * kResChunkBytes + lane * 16;
+  const uint32_t dst = smem_addr(slot) + lane * 16;
+#pragma unroll
+  for (int c = 0; c < kCRes; ++c)
+    if (c < rs.nchunks) cp_async16(dst + c * kResChunkBytes, codes + c * kResChunkBytes);
+  if (lane * 16 < rs.ng * kSresGroupBytes)
+    cp_async16(dst + kCRes * kResChunkBytes, blk + p.off_sres + rs.grp0 * kSresGroupBytes + lane * 16);
+}
+
+// One m-tile of a residual warp: 16 k16 steps over its 4 chunks, flushing
+// each scale group into acc.  kFull: all 4 chunks present (no guards).
+template <int G, bool kFull>
+__device__ __forceinline__ void residual_tile(const uint8_t* slot, const ResSlice& rs,
+                                              const uint32_t (&hf)[kCRes][4][2], const float2 (&cgc)[16 / G],
+                                              int step0, int last_step, int g_log2, int lane, float (&acc)[4]) {
+  const int gr = lane >> 2;
+  float t0[4] = {0.f, 0.f, 0.f, 0.f};
+  float t1[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint8_t* sres = slot + kCRes * kResChunkBytes + gr * 4;
+#pragma unroll
+  for (int c = 0; c < kCRes; ++c) {
+    if (kFull || c < rs.nchunks) {
+      const uint4 nib = *reinterpret_cast<const uint4*>(slot + c * kResChunkBytes + lane * 16);
+      const uint32_t wv[4] = {nib.x, nib.y, nib.z, nib.w};
+#pragma unroll
+      for (int st = 0; st < 4; ++st) {
+        const int step = 4 * c + st;
+        const int lg = step / G;
+        float(&tmp)[4] = (lg & 1) ? t1 : t0;
+        uint32_t a[4];
+        unpack_int4_biased(wv[st], a);
+        mma_f16_16816(tmp, a, hf[c][st][0], hf[c][st][1]);
+        if ((step + 1) % G == 0 || (G == 16 && step == last_step)) {
+          const int grp = ((step0 + step) >> g_log2) - rs.grp0;
+          const float2 sc = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(sres + grp * kSresGroupBytes));
+          acc[0] = fmaf(sc.x, tmp[0] - cgc[lg].x, acc[0]);
+          acc[1] = fmaf(sc.x, tmp[1] - cgc[lg].y, acc[1]);
+          acc[2] = fmaf(sc.y, tmp[2] - cgc[lg].x, acc[2]);
+          acc[3] = fmaf(sc.y, tmp[3] - cgc[lg].y, acc[3]);
+          tmp[0] = tmp[1] = tmp[2] = tmp[3] = 0.f;
+        }
+      }
+    }
+  }
 }
 
 // G = k16 steps per scale group within the warp's 16 steps (16 when a group
@@ -244,41 +280,14 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
     cp_async_wait<kRing - 1>();
     __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    {
-      float t0[4] = {0.f, 0.f, 0.f, 0.f};
-      float t1[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint8_t* sres = slot + kCRes * kResChunkBytes;
-#pragma unroll
-      for (int c = 0; c < kCRes; ++c) {
-        if (c < rs.nchunks) {
-          const uint4 nib = *reinterpret_cast<const uint4*>(slot + c * kResChunkBytes + lane * 16);
-          const uint32_t wv[4] = {nib.x, nib.y, nib.z, nib.w};
-#pragma unroll
-          for (int st = 0; st < 4; ++st) {
-            const int step = 4 * c + st;
-            const int lg = step / G;
-            float(&tmp)[4] = (lg & 1) ? t1 : t0;
-            uint32_t a[4];
-            unpack_int4_biased(wv[st], a);
-            mma_f16_16816(tmp, a, hf[c][st][0], hf[c][st][1]);
-            if ((step + 1) % G == 0 || (G == 16 && step == last_step)) {
-              const int grp = ((step0 + step) >> p.g_steps_log2) - rs.grp0;
-              const float2 sc =
-                  half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(sres + grp * kSresGroupBytes + gr * 4));
-              acc[0] = fmaf(sc.x, tmp[0] - cgc[lg].x, acc[0]);
-              acc[1] = fmaf(sc.x, tmp[1] - cgc[lg].y, acc[1]);
-              acc[2] = fmaf(sc.y, tmp[2] - cgc[lg].x, acc[2]);
-              acc[3] = fmaf(sc.y, tmp[3] - cgc[lg].y, acc[3]);
-              tmp[0] = tmp[1] = tmp[2] = tmp[3] = 0.f;
-            }
-          }
-        }
-      }
-      acc[0] *= unscale.x;
-      acc[1] *= unscale.y;
-      acc[2] *= unscale.x;
-      acc[3] *= unscale.y;
-    }
+    if (rs.nchunks == kCRes)
+      residual_tile<G, true>(slot, rs, hf, cgc, step0, kCRes * 4 - 1, p.g_steps_log2, lane, acc);
+    else
+      residual_tile<G, false>(slot, rs, hf, cgc, step0, last_step, p.g_steps_log2, lane, acc);
+    acc[0] *= unscale.x;
+    acc[1] *= unscale.y;
+    acc[2] *= unscale.x;
+    acc[3] *= unscale.y;
     __syncwarp();   // every lane is done reading the slot
     if (i + kRing < n_my) issue_res(p, rs, slot, i + kRing, lane);
     cp_async_commit();
@@ -292,9 +301,15 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
 __device__ __forceinline__ void issue_core(const DecodeParams& p, int chunk0, int nch, uint8_t* slot, int i,
                                            int lane) {
   const uint8_t* blk = mtile_block(p, i);
-  warp_copy(slot, blk + p.off_Lnib + chunk0 * kLNibChunkBytes, nch * kLNibChunkBytes, lane);
-  warp_copy(slot + kCL * kLNibChunkBytes, blk + p.off_Lhi + chunk0 * kLHiChunkBytes, nch * kLHiChunkBytes, lane);
-  warp_copy(slot + kCL * (kLNibChunkBytes + kLHiChunkBytes), blk + p.off_sL, 32, lane);
+  const uint32_t dst = smem_addr(slot) + lane * 16;
+  const uint8_t* nib = blk + p.off_Lnib + chunk0 * kLNibChunkBytes + lane * 16;
+#pragma unroll
+  for (int c = 0; c < kCL; ++c)
+    if (c < nch) cp_async16(dst + c * kLNibChunkBytes, nib + c * kLNibChunkBytes);
+  // fifth-bit planes (128 B per chunk) and the 32 B of row scales
+  if (lane * 16 < nch * kLHiChunkBytes)
+    cp_async16(dst + kCL * kLNibChunkBytes, blk + p.off_Lhi + chunk0 * kLHiChunkBytes + lane * 16);
+  if (lane < 2) cp_async16(dst + kCL * (kLNibChunkBytes + kLHiChunkBytes), blk + p.off_sL + lane * 16);
 }
 
 __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wl, int lane) {
@@ -375,8 +390,12 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
 __device__ __forceinline__ void issue_corr(const DecodeParams& p, int chunk0, int nch, uint8_t* slot, int i,
                                            int lane) {
   const uint8_t* blk = mtile_block(p, i);
-  warp_copy(slot, blk + p.off_A + chunk0 * kAChunkBytes, nch * kAChunkBytes, lane);
-  warp_copy(slot + kCA * kAChunkBytes, blk + p.off_sA, 32, lane);
+  const uint32_t dst = smem_addr(slot) + lane * 16;
+  const uint8_t* codes = blk + p.off_A + chunk0 * kAChunkBytes + lane * 16;
+#pragma unroll
+  for (int c = 0; c < kCA; ++c)
+    if (c < nch) cp_async16(dst + c * kAChunkBytes, codes + c * kAChunkBytes);
+  if (lane < 2) cp_async16(dst + kCA * kAChunkBytes, blk + p.off_sA + lane * 16);
 }
 
 __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wa, int lane) {
@@ -457,8 +476,8 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     target[k] = (e < nel && p.targets != nullptr) ? p.targets[p.t0 + (e >> 4)] : -1;
   }
   for (int i = 0; i < n_my; ++i) {
-    const int r = i % p.slots;
-    const bool ok = warp_wait(sv, &sv.reduced[r], (i / p.slots) & 1, p.status, lane);
+    const int r = i & (kSlots - 1);
+    const bool ok = warp_wait(sv, &sv.reduced[r], (i / kSlots) & 1, p.status, lane);
     unsigned long long* tsum = sv.tsum + static_cast<size_t>(r) * nel;
     const int vbase = mtile_of(i) * kMT;
 #pragma unroll

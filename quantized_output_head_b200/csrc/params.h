@@ -13,7 +13,7 @@ constexpr int kCA = 2;
 constexpr int kMaxDecodeWarps = 24;      // launch bound of the decode kernel
 constexpr int kDecodeTokens = 8;         // N of one m16n8k16 fragment
 constexpr int kRing = 4;                 // m-tiles in flight per compute warp
-constexpr int kSlots = 8;                // fixed-point logit slots
+constexpr int kSlots = 8;                // fixed-point logit slots (a power of two)
 // h is scaled per token by 2^(kScaleExp - E_t), E_t the binary exponent of
 // max|h_t| (max|h_t| < 2^E_t), so the fp16 copy is below 2^kScaleExp.
 constexpr int kScaleExp = 14;
