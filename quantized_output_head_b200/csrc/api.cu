@@ -116,7 +116,9 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   for (int t0 = 0; t0 < T; t0 += kDecodeTokens) {
     dp.t0 = t0;
     dp.nt = (T - t0 < kDecodeTokens) ? (T - t0) : kDecodeTokens;
-    dp.slots = kSlots;
+    // Partial-logit slots: 8 while the tiles are small, 4 at the widest launch.
+    dp.slots = dp.nt <= 4 ? 8 : 4;
+    dp.slots_log2 = dp.nt <= 4 ? 3 : 2;
     decode_smem_plan(dp, L.g_steps);
     e = launch_decode(L.g_steps, dp, h->grid, decode_smem_bytes(dp), stream);
     if (e != cudaSuccess) return set_cuda_error(e);

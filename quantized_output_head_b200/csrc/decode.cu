@@ -24,11 +24,11 @@
 // Each compute warp prefetches its slice of the next kRing m-tiles into a
 // private shared-memory ring with cp.async (16 B per lane, L2 only) and waits
 // only on its own copies: no producer warp and no block-wide synchronisation.
-// After an m-tile the warp adds its 16 x nt partial logits into a fixed-point
-// slot tile (int64, shared atomics; identical bits in any order) and arrives
-// on reduced[r].  Warp 0, the epilogue, takes each finished tile, pushes the
-// logits into a running log-sum-exp / argmax state, writes logits when asked,
-// clears the slot and frees it (redfree[r]).  At the end every block writes one
+// After an m-tile the warp stores its 16 x nt partial logits in its own region
+// of a slot and arrives on reduced[r].  Warp 0, the epilogue, sums each slot's
+// regions in warp order (deterministic), pushes the logits into a running
+// log-sum-exp / argmax state, writes logits when asked, and frees the slot
+// (redfree[r]).  At the end every block writes one
 // partial per token; the last block to finish (atomic ticket, no spinning)
 // merges them into LSE, argmax and CE.  Every mbarrier wait is bounded
 // (kWaitLimitNs); on expiry the block raises ARCHEAD_STATUS_WAIT_TIMEOUT and
@@ -46,7 +46,7 @@ constexpr int kEpiSlots = 4;     // 16 rows x 8 tokens / 32 lanes
 
 struct SmemView {
   uint8_t* rings;                // per compute warp: kRing slices
-  unsigned long long* tsum;      // [slots][nt][16 rows] fixed-point logit sums
+  float* part;                   // [slots][nw_work][nt][16 rows] per-warp partial logits
   uint64_t* reduced;             // [slots] compute warps -> epilogue warp
   uint64_t* redfree;             // [slots] epilogue warp -> compute warps
   int* flags;                    // [0] abort
@@ -55,8 +55,8 @@ struct SmemView {
 __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams& p) {
   SmemView v;
   v.rings = smem;
-  v.tsum = reinterpret_cast<unsigned long long*>(smem + p.ring_bytes);
-  v.reduced = reinterpret_cast<uint64_t*>(v.tsum + static_cast<size_t>(p.slots) * p.nt * 16);
+  v.part = reinterpret_cast<float*>(smem + p.ring_bytes);
+  v.reduced = reinterpret_cast<uint64_t*>(v.part + static_cast<size_t>(p.slots) * p.nw_work * p.nt * 16);
   v.redfree = v.reduced + p.slots;
   v.flags = reinterpret_cast<int*>(v.redfree + p.slots);
   return v;
@@ -123,36 +123,25 @@ __device__ __forceinline__ float quad_sum(float v) {
   return v;
 }
 
-// Logit partial sums of the compute warps meet in a fixed-point tile: each
-// value is rounded to a multiple of 2^-32 (error <= 2^-33, far below the
-// logit tolerance) and added as a 64-bit integer.  Integer addition is
-// associative, so the tile holds the same bits whatever the order in which the
-// warps arrive.  |partial| < 2^31 is assumed (the conversion saturates).
-constexpr float kFixScale = 4294967296.0f;   // 2^32
-
-__device__ __forceinline__ void add_partial(const SmemView& sv, const DecodeParams& p, int r, int lane,
-                                            const float (&acc)[4]) {
-  const int gr = lane >> 2, cc = lane & 3;
-  unsigned long long* tile = sv.tsum + r * p.nt * 16;
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int t = 2 * cc + j;
-    if (t < p.nt) {
-      const long long lo = __float2ll_rn(acc[j] * kFixScale);
-      const long long hi = __float2ll_rn(acc[2 + j] * kFixScale);
-      atomicAdd(tile + t * 16 + gr, static_cast<unsigned long long>(lo));
-      atomicAdd(tile + t * 16 + gr + 8, static_cast<unsigned long long>(hi));
-    }
-  }
-}
-
-// End of m-tile i for a compute warp: add its partial logits into slot r
-// (after the epilogue has drained the slot's previous use) and report.
-__device__ __forceinline__ void finish_mtile(const SmemView& sv, const DecodeParams& p, int i, int lane,
+// End of m-tile i for compute warp cw: store its 16 x nt partial logits in
+// its own region of slot r (after the epilogue has drained the slot's previous
+// use) and report.  The epilogue sums the regions in warp order, so the result
+// does not depend on arrival order.
+__device__ __forceinline__ void finish_mtile(const SmemView& sv, const DecodeParams& p, int i, int cw, int lane,
                                              const float (&acc)[4]) {
-  const int r = i & (kSlots - 1);
-  if (i >= kSlots) warp_wait(sv, &sv.redfree[r], ((i / kSlots) - 1) & 1, p.status, lane);
-  add_partial(sv, p, r, lane, acc);
+  const int r = i & (p.slots - 1);
+  if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i >> p.slots_log2) - 1) & 1, p.status, lane);
+  const int gr = lane >> 2, cc = lane & 3;
+  float* tile = sv.part + (r * p.nw_work + cw) * p.nt * 16;
+  const int t0 = 2 * cc, t1 = 2 * cc + 1;
+  if (t0 < p.nt) {
+    tile[t0 * 16 + gr] = acc[0];
+    tile[t0 * 16 + gr + 8] = acc[2];
+  }
+  if (t1 < p.nt) {
+    tile[t1 * 16 + gr] = acc[1];
+    tile[t1 * 16 + gr + 8] = acc[3];
+  }
   __syncwarp();
   if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[r]));
 }
@@ -225,7 +214,7 @@ __device__ __forceinline__ void residual_tile(const uint8_t* slot, const ResSlic
 // G = k16 steps per scale group within the warp's 16 steps (16 when a group
 // spans the whole warp range or more).
 template <int G>
-__device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wres, int lane) {
+__device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wres, int cw, int lane) {
   constexpr int kNG = 16 / G;    // local scale groups
   const int gr = lane >> 2;
   const ResSlice rs = res_slice(p, wres);
@@ -291,7 +280,7 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
     __syncwarp();   // every lane is done reading the slot
     if (i + kRing < n_my) issue_res(p, rs, slot, i + kRing, lane);
     cp_async_commit();
-    finish_mtile(sv, p, i, lane, acc);
+    finish_mtile(sv, p, i, cw, lane, acc);
   }
   cp_async_wait_all();
 }
@@ -312,7 +301,7 @@ __device__ __forceinline__ void issue_core(const DecodeParams& p, int chunk0, in
   if (lane < 2) cp_async16(dst + kCL * (kLNibChunkBytes + kLHiChunkBytes), blk + p.off_sL + lane * 16);
 }
 
-__device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wl, int lane) {
+__device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wl, int cw, int lane) {
   const int gr = lane >> 2;
   const int chunk0 = wl * kCL;
   const int nch = min(kCL, p.n_L - chunk0);
@@ -380,7 +369,7 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
     __syncwarp();
     if (i + kRing < n_my) issue_core(p, chunk0, nch, slot, i + kRing, lane);
     cp_async_commit();
-    finish_mtile(sv, p, i, lane, acc);
+    finish_mtile(sv, p, i, cw, lane, acc);
   }
   cp_async_wait_all();
 }
@@ -398,7 +387,7 @@ __device__ __forceinline__ void issue_corr(const DecodeParams& p, int chunk0, in
   if (lane < 2) cp_async16(dst + kCA * kAChunkBytes, blk + p.off_sA + lane * 16);
 }
 
-__device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wa, int lane) {
+__device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wa, int cw, int lane) {
   const int gr = lane >> 2;
   const int chunk0 = wa * kCA;
   const int nch = min(kCA, p.n_A - chunk0);
@@ -458,7 +447,7 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
     __syncwarp();
     if (i + kRing < n_my) issue_corr(p, chunk0, nch, slot, i + kRing, lane);
     cp_async_commit();
-    finish_mtile(sv, p, i, lane, acc);
+    finish_mtile(sv, p, i, cw, lane, acc);
   }
   cp_async_wait_all();
 }
@@ -476,18 +465,25 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     target[k] = (e < nel && p.targets != nullptr) ? p.targets[p.t0 + (e >> 4)] : -1;
   }
   for (int i = 0; i < n_my; ++i) {
-    const int r = i & (kSlots - 1);
-    const bool ok = warp_wait(sv, &sv.reduced[r], (i / kSlots) & 1, p.status, lane);
-    unsigned long long* tsum = sv.tsum + static_cast<size_t>(r) * nel;
+    const int r = i & (p.slots - 1);
+    const bool ok = warp_wait(sv, &sv.reduced[r], (i >> p.slots_log2) & 1, p.status, lane);
+    const float* part = sv.part + r * p.nw_work * nel;
     const int vbase = mtile_of(i) * kMT;
 #pragma unroll
     for (int k = 0; k < kEpiSlots; ++k) {
       const int e = lane + 32 * k;
-      if (e < nel) {
-        const long long fx = static_cast<long long>(tsum[e]);
-        tsum[e] = 0ull;   // ready for the slot's next use
-        if (!ok) continue;
-        const float y = __ll2float_rn(fx) * (1.0f / kFixScale);
+      if (ok && e < nel) {
+        // warp-order sum with four independent chains
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        int w = 0;
+        for (; w + 4 <= p.nw_work; w += 4) {
+          y0 += part[(w + 0) * nel + e];
+          y1 += part[(w + 1) * nel + e];
+          y2 += part[(w + 2) * nel + e];
+          y3 += part[(w + 3) * nel + e];
+        }
+        for (; w < p.nw_work; ++w) y0 += part[w * nel + e];
+        const float y = (y0 + y1) + (y2 + y3);
         const int row = e & 15, t = e >> 4;
         const int v = vbase + row;
         if (v < p.V) {
@@ -559,7 +555,6 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
     sv.flags[0] = 0;
     mbar_fence_init();
   }
-  for (int e = threadIdx.x; e < p.slots * p.nt * 16; e += blockDim.x) sv.tsum[e] = 0ull;
   __syncthreads();
 
   if (warp == 0) {
@@ -568,11 +563,11 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
   }
   const int cw = warp - 1;
   if (cw < p.nw_res) {
-    residual_warp<G>(p, sv, n_my, cw, lane);
+    residual_warp<G>(p, sv, n_my, cw, cw, lane);
   } else if (cw < p.nw_res + p.nw_L) {
-    core_warp(p, sv, n_my, cw - p.nw_res, lane);
+    core_warp(p, sv, n_my, cw - p.nw_res, cw, lane);
   } else if (cw < p.nw_work) {
-    correction_warp(p, sv, n_my, cw - p.nw_res - p.nw_L, lane);
+    correction_warp(p, sv, n_my, cw - p.nw_res - p.nw_L, cw, lane);
   }
 }
 
@@ -590,7 +585,7 @@ void decode_smem_plan(DecodeParams& p, int g_steps) {
 }
 
 size_t decode_smem_bytes(const DecodeParams& p) {
-  return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nt * 16 * 8 +
+  return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nw_work * p.nt * 16 * 4 +
          static_cast<size_t>(2) * p.slots * 8 + 16;
 }
 

@@ -13,7 +13,6 @@ constexpr int kCA = 2;
 constexpr int kMaxDecodeWarps = 24;      // launch bound of the decode kernel
 constexpr int kDecodeTokens = 8;         // N of one m16n8k16 fragment
 constexpr int kRing = 4;                 // m-tiles in flight per compute warp
-constexpr int kSlots = 8;                // fixed-point logit slots (a power of two)
 // h is scaled per token by 2^(kScaleExp - E_t), E_t the binary exponent of
 // max|h_t| (max|h_t| < 2^E_t), so the fp16 copy is below 2^kScaleExp.
 constexpr int kScaleExp = 14;
@@ -38,7 +37,7 @@ struct DecodeParams {
   int32_t n_res, n_L, n_A, n_mtiles, g_steps_log2;
   uint32_t off_res, off_Lnib, off_Lhi, off_A, off_sres, off_sL, off_sA, mblk_bytes;
   int32_t nw_res, nw_L, nw_A, nw_work;   // compute warps by role
-  int32_t slots;               // fixed-point logit slots between compute and epilogue warps
+  int32_t slots, slots_log2;   // partial-logit slots between compute and epilogue warps (power of two)
   // Shared-memory rings: one per compute warp, kRing slices each.
   uint32_t res_slice_bytes, core_slice_bytes, corr_slice_bytes;
   uint32_t core_ring_off, corr_ring_off, ring_bytes;
