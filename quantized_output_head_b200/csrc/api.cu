@@ -116,9 +116,11 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   for (int t0 = 0; t0 < T; t0 += kDecodeTokens) {
     dp.t0 = t0;
     dp.nt = (T - t0 < kDecodeTokens) ? (T - t0) : kDecodeTokens;
-    // Partial-logit slots: 8 while the tiles are small, 4 at the widest launch.
-    dp.slots = dp.nt <= 4 ? 8 : 4;
-    dp.slots_log2 = dp.nt <= 4 ? 3 : 2;
+    // Partial logits move in groups of mg m-tiles with mg * nt <= 8; four slots.
+    dp.mg_log2 = dp.nt <= 1 ? 3 : dp.nt <= 2 ? 2 : dp.nt <= 4 ? 1 : 0;
+    dp.mg = 1 << dp.mg_log2;
+    dp.slots = 4;
+    dp.slots_log2 = 2;
     decode_smem_plan(dp, L.g_steps);
     e = launch_decode(L.g_steps, dp, h->grid, decode_smem_bytes(dp), stream);
     if (e != cudaSuccess) return set_cuda_error(e);

@@ -42,11 +42,12 @@ namespace archead {
 
 namespace {
 
-constexpr int kEpiSlots = 4;     // 16 rows x 8 tokens / 32 lanes
+constexpr int kEpiSlots = 4;     // kGroupTile x 16 logits / 32 lanes
+constexpr int kGroupTile = 8;    // m-tiles x tokens per partial-logit group (mg * nt)
 
 struct SmemView {
   uint8_t* rings;                // per compute warp: kRing slices
-  float* part;                   // [slots][nw_work][nt][16 rows] per-warp partial logits
+  float* part;                   // [slots][nw_work][mg][nt][16 rows] per-warp partial logits
   uint64_t* reduced;             // [slots] compute warps -> epilogue warp
   uint64_t* redfree;             // [slots] epilogue warp -> compute warps
   int* flags;                    // [0] abort
@@ -56,7 +57,7 @@ __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams&
   SmemView v;
   v.rings = smem;
   v.part = reinterpret_cast<float*>(smem + p.ring_bytes);
-  v.reduced = reinterpret_cast<uint64_t*>(v.part + static_cast<size_t>(p.slots) * p.nw_work * p.nt * 16);
+  v.reduced = reinterpret_cast<uint64_t*>(v.part + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16);
   v.redfree = v.reduced + p.slots;
   v.flags = reinterpret_cast<int*>(v.redfree + p.slots);
   return v;
@@ -82,10 +83,6 @@ __device__ __forceinline__ bool warp_wait(const SmemView& sv, uint64_t* bar, uin
 
 __device__ __forceinline__ int mtile_of(int i) {
   return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
-}
-
-__device__ __forceinline__ const uint8_t* mtile_block(const DecodeParams& p, int i) {
-  return p.mtiles + static_cast<size_t>(mtile_of(i)) * p.mblk_bytes;
 }
 
 // B-operand fragment (16 x 8, column = token) from the fp16 row of token gr:
@@ -123,27 +120,39 @@ __device__ __forceinline__ float quad_sum(float v) {
   return v;
 }
 
-// End of m-tile i for compute warp cw: store its 16 x nt partial logits in
-// its own region of slot r (after the epilogue has drained the slot's previous
-// use) and report.  The epilogue sums the regions in warp order, so the result
-// does not depend on arrival order.
-__device__ __forceinline__ void finish_mtile(const SmemView& sv, const DecodeParams& p, int i, int cw, int lane,
-                                             const float (&acc)[4]) {
-  const int r = i & (p.slots - 1);
-  if (i >= p.slots) warp_wait(sv, &sv.redfree[r], ((i >> p.slots_log2) - 1) & 1, p.status, lane);
+// Partial logits travel in groups of p.mg consecutive m-tiles of this block
+// (p.mg * p.nt = 8): slot r = group & (slots - 1) holds, per compute warp, a
+// [mg][nt][16] tile.  A compute warp checks once per group that the epilogue
+// has drained the slot's previous group, stores each m-tile's partial tile
+// with plain stores, and arrives on reduced[r] once per group.  The epilogue
+// sums the warps' tiles in warp order, so results do not depend on timing.
+__device__ __forceinline__ float* group_begin(const SmemView& sv, const DecodeParams& p, int i, int cw, int lane) {
+  const int grp = i >> p.mg_log2;
+  const int r = grp & (p.slots - 1);
+  if (grp >= p.slots) warp_wait(sv, &sv.redfree[r], ((grp >> p.slots_log2) - 1) & 1, p.status, lane);
+  return sv.part + (r * p.nw_work + cw) * (kGroupTile * 16);
+}
+
+__device__ __forceinline__ void store_partial(float* tile, const DecodeParams& p, int i, int lane,
+                                              const float (&acc)[4]) {
   const int gr = lane >> 2, cc = lane & 3;
-  float* tile = sv.part + (r * p.nw_work + cw) * p.nt * 16;
+  float* t = tile + (i & (p.mg - 1)) * p.nt * 16;
   const int t0 = 2 * cc, t1 = 2 * cc + 1;
   if (t0 < p.nt) {
-    tile[t0 * 16 + gr] = acc[0];
-    tile[t0 * 16 + gr + 8] = acc[2];
+    t[t0 * 16 + gr] = acc[0];
+    t[t0 * 16 + gr + 8] = acc[2];
   }
   if (t1 < p.nt) {
-    tile[t1 * 16 + gr] = acc[1];
-    tile[t1 * 16 + gr + 8] = acc[3];
+    t[t1 * 16 + gr] = acc[1];
+    t[t1 * 16 + gr + 8] = acc[3];
   }
-  __syncwarp();
-  if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[r]));
+}
+
+__device__ __forceinline__ void group_end(const SmemView& sv, const DecodeParams& p, int i, int n_my, int lane) {
+  if ((i & (p.mg - 1)) == p.mg - 1 || i == n_my - 1) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sv.reduced[(i >> p.mg_log2) & (p.slots - 1)]));
+  }
 }
 
 // ------------------------------------------------------------ residual warps
@@ -163,15 +172,16 @@ __device__ __forceinline__ ResSlice res_slice(const DecodeParams& p, int wres) {
   return r;
 }
 
-__device__ __forceinline__ void issue_res(const DecodeParams& p, const ResSlice& rs, uint8_t* slot, int i, int lane) {
-  const uint8_t* blk = mtile_block(p, i);
-  const uint8_t* codes = blk + p.off_res + rs.chunk0 * kResChunkBytes + lane * 16;
-  const uint32_t dst = smem_addr(slot) + lane * 16;
+// Copy this lane's 16-byte pieces of one m-tile's residual slice: codes at
+// `codes` (already offset to the lane), scales at `scales` (lanes that own a
+// piece only).  kFull: all kCRes chunks present.
+template <bool kFull>
+__device__ __forceinline__ void issue_res(uint32_t dst, const uint8_t* codes, const uint8_t* scales, int nchunks,
+                                          bool scale_lane) {
 #pragma unroll
   for (int c = 0; c < kCRes; ++c)
-    if (c < rs.nchunks) cp_async16(dst + c * kResChunkBytes, codes + c * kResChunkBytes);
-  if (lane * 16 < rs.ng * kSresGroupBytes)
-    cp_async16(dst + kCRes * kResChunkBytes, blk + p.off_sres + rs.grp0 * kSresGroupBytes + lane * 16);
+    if (kFull || c < nchunks) cp_async16(dst + c * kResChunkBytes, codes + c * kResChunkBytes);
+  if (scale_lane) cp_async16(dst + kCRes * kResChunkBytes, scales);
 }
 
 // One m-tile of a residual warp: 16 k16 steps over its 4 chunks, flushing
@@ -220,12 +230,25 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
   const ResSlice rs = res_slice(p, wres);
   const uint32_t sbytes = p.res_slice_bytes;
   uint8_t* ring = sv.rings + static_cast<size_t>(wres) * kRing * sbytes;
+  const uint32_t ring_s = smem_addr(ring) + lane * 16;
+  // Global pieces of m-tile 0 of this block; m-tile i is `stride` bytes further per step.
+  const size_t stride = static_cast<size_t>(gridDim.x) * p.mblk_bytes;
+  const uint8_t* base = p.mtiles + static_cast<size_t>(blockIdx.x) * p.mblk_bytes;
+  const uint8_t* g_codes = base + p.off_res + rs.chunk0 * kResChunkBytes + lane * 16;
+  const uint8_t* g_scales = base + p.off_sres + rs.grp0 * kSresGroupBytes + lane * 16;
+  const bool scale_lane = lane * 16 < rs.ng * kSresGroupBytes;
+  const bool full = rs.nchunks == kCRes;
   // Start streaming before the prologue's results are needed.
 #pragma unroll
   for (int k = 0; k < kRing; ++k) {
-    if (k < n_my) issue_res(p, rs, ring + k * sbytes, k, lane);
+    if (k < n_my) {
+      if (full) issue_res<true>(ring_s + k * sbytes, g_codes + k * stride, g_scales + k * stride, rs.nchunks, scale_lane);
+      else issue_res<false>(ring_s + k * sbytes, g_codes + k * stride, g_scales + k * stride, rs.nchunks, scale_lane);
+    }
     cp_async_commit();
   }
+  g_codes += kRing * stride;
+  g_scales += kRing * stride;
   grid_dependency_wait();
   const bool tok = gr < p.nt;
   float hs = 0.f;
@@ -264,12 +287,15 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
   const int last_step = rs.nchunks * 4 - 1;
   const int step0 = wres * 16;
 
+  float* tile = nullptr;
   for (int i = 0; i < n_my; ++i) {
-    uint8_t* slot = ring + (i % kRing) * sbytes;
+    if ((i & (p.mg - 1)) == 0) tile = group_begin(sv, p, i, cw, lane);
+    const uint32_t k = static_cast<uint32_t>(i) & (kRing - 1);
+    const uint8_t* slot = ring + k * sbytes;
     cp_async_wait<kRing - 1>();
     __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (rs.nchunks == kCRes)
+    if (full)
       residual_tile<G, true>(slot, rs, hf, cgc, step0, kCRes * 4 - 1, p.g_steps_log2, lane, acc);
     else
       residual_tile<G, false>(slot, rs, hf, cgc, step0, last_step, p.g_steps_log2, lane, acc);
@@ -278,27 +304,31 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
     acc[2] *= unscale.x;
     acc[3] *= unscale.y;
     __syncwarp();   // every lane is done reading the slot
-    if (i + kRing < n_my) issue_res(p, rs, slot, i + kRing, lane);
+    if (i + kRing < n_my) {
+      if (full) issue_res<true>(ring_s + k * sbytes, g_codes, g_scales, rs.nchunks, scale_lane);
+      else issue_res<false>(ring_s + k * sbytes, g_codes, g_scales, rs.nchunks, scale_lane);
+    }
+    g_codes += stride;
+    g_scales += stride;
     cp_async_commit();
-    finish_mtile(sv, p, i, cw, lane, acc);
+    store_partial(tile, p, i, lane, acc);
+    group_end(sv, p, i, n_my, lane);
   }
   cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------- core warps
 // Ring slice: [kCL x 512 B nibbles][kCL x 128 B fifth bits][32 B s_L].
-__device__ __forceinline__ void issue_core(const DecodeParams& p, int chunk0, int nch, uint8_t* slot, int i,
-                                           int lane) {
-  const uint8_t* blk = mtile_block(p, i);
-  const uint32_t dst = smem_addr(slot) + lane * 16;
-  const uint8_t* nib = blk + p.off_Lnib + chunk0 * kLNibChunkBytes + lane * 16;
+// One m-tile's core slice for this lane: nibble planes, fifth-bit planes
+// (lanes below nch * 8) and row scales (lanes 0, 1).  Global pointers are
+// already offset to the lane.
+__device__ __forceinline__ void issue_core(uint32_t dst, const uint8_t* g_nib, const uint8_t* g_hi,
+                                           const uint8_t* g_sl, int nch, bool hi_lane, bool sl_lane) {
 #pragma unroll
   for (int c = 0; c < kCL; ++c)
-    if (c < nch) cp_async16(dst + c * kLNibChunkBytes, nib + c * kLNibChunkBytes);
-  // fifth-bit planes (128 B per chunk) and the 32 B of row scales
-  if (lane * 16 < nch * kLHiChunkBytes)
-    cp_async16(dst + kCL * kLNibChunkBytes, blk + p.off_Lhi + chunk0 * kLHiChunkBytes + lane * 16);
-  if (lane < 2) cp_async16(dst + kCL * (kLNibChunkBytes + kLHiChunkBytes), blk + p.off_sL + lane * 16);
+    if (c < nch) cp_async16(dst + c * kLNibChunkBytes, g_nib + c * kLNibChunkBytes);
+  if (hi_lane) cp_async16(dst + kCL * kLNibChunkBytes, g_hi);
+  if (sl_lane) cp_async16(dst + kCL * (kLNibChunkBytes + kLHiChunkBytes), g_sl);
 }
 
 __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wl, int cw, int lane) {
@@ -307,11 +337,22 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
   const int nch = min(kCL, p.n_L - chunk0);
   const uint32_t sbytes = p.core_slice_bytes;
   uint8_t* ring = sv.rings + p.core_ring_off + static_cast<size_t>(wl) * kRing * sbytes;
+  const uint32_t ring_s = smem_addr(ring) + lane * 16;
+  const size_t stride = static_cast<size_t>(gridDim.x) * p.mblk_bytes;
+  const uint8_t* base = p.mtiles + static_cast<size_t>(blockIdx.x) * p.mblk_bytes;
+  const uint8_t* g_nib = base + p.off_Lnib + chunk0 * kLNibChunkBytes + lane * 16;
+  const uint8_t* g_hi = base + p.off_Lhi + chunk0 * kLHiChunkBytes + lane * 16;
+  const uint8_t* g_sl = base + p.off_sL + lane * 16;
+  const bool hi_lane = lane * 16 < nch * kLHiChunkBytes, sl_lane = lane < 2;
 #pragma unroll
   for (int k = 0; k < kRing; ++k) {
-    if (k < n_my) issue_core(p, chunk0, nch, ring + k * sbytes, k, lane);
+    if (k < n_my) issue_core(ring_s + k * sbytes, g_nib + k * stride, g_hi + k * stride, g_sl + k * stride, nch,
+                             hi_lane, sl_lane);
     cp_async_commit();
   }
+  g_nib += kRing * stride;
+  g_hi += kRing * stride;
+  g_sl += kRing * stride;
   grid_dependency_wait();
   const bool tok = gr < p.nt;
   uint32_t zf[kCL][4][2][2];
@@ -334,8 +375,11 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
   const float zs = tok ? ldexpf(1.f, p.escale[p.t0 + gr] + p.e_B - kScaleExp) : 0.f;
   const float2 unscale = column_pair(zs, lane);
 
+  float* tile = nullptr;
   for (int i = 0; i < n_my; ++i) {
-    uint8_t* slot = ring + (i % kRing) * sbytes;
+    if ((i & (p.mg - 1)) == 0) tile = group_begin(sv, p, i, cw, lane);
+    const uint32_t k = static_cast<uint32_t>(i) & (kRing - 1);
+    const uint8_t* slot = ring + k * sbytes;
     cp_async_wait<kRing - 1>();
     __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -367,24 +411,26 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
     acc[2] = (acc[2] - cbc.x) * (sc.y * unscale.x);
     acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
     __syncwarp();
-    if (i + kRing < n_my) issue_core(p, chunk0, nch, slot, i + kRing, lane);
+    if (i + kRing < n_my) issue_core(ring_s + k * sbytes, g_nib, g_hi, g_sl, nch, hi_lane, sl_lane);
+    g_nib += stride;
+    g_hi += stride;
+    g_sl += stride;
     cp_async_commit();
-    finish_mtile(sv, p, i, cw, lane, acc);
+    store_partial(tile, p, i, lane, acc);
+    group_end(sv, p, i, n_my, lane);
   }
   cp_async_wait_all();
 }
 
 // ---------------------------------------------------------- correction warps
 // Ring slice: [kCA x 512 B codes][32 B s_A].
-__device__ __forceinline__ void issue_corr(const DecodeParams& p, int chunk0, int nch, uint8_t* slot, int i,
-                                           int lane) {
-  const uint8_t* blk = mtile_block(p, i);
-  const uint32_t dst = smem_addr(slot) + lane * 16;
-  const uint8_t* codes = blk + p.off_A + chunk0 * kAChunkBytes + lane * 16;
+// One m-tile's correction slice for this lane: codes and row scales (lanes 0, 1).
+__device__ __forceinline__ void issue_corr(uint32_t dst, const uint8_t* g_codes, const uint8_t* g_sa, int nch,
+                                           bool sa_lane) {
 #pragma unroll
   for (int c = 0; c < kCA; ++c)
-    if (c < nch) cp_async16(dst + c * kAChunkBytes, codes + c * kAChunkBytes);
-  if (lane < 2) cp_async16(dst + kCA * kAChunkBytes, blk + p.off_sA + lane * 16);
+    if (c < nch) cp_async16(dst + c * kAChunkBytes, g_codes + c * kAChunkBytes);
+  if (sa_lane) cp_async16(dst + kCA * kAChunkBytes, g_sa);
 }
 
 __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wa, int cw, int lane) {
@@ -393,11 +439,19 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
   const int nch = min(kCA, p.n_A - chunk0);
   const uint32_t sbytes = p.corr_slice_bytes;
   uint8_t* ring = sv.rings + p.corr_ring_off + static_cast<size_t>(wa) * kRing * sbytes;
+  const uint32_t ring_s = smem_addr(ring) + lane * 16;
+  const size_t stride = static_cast<size_t>(gridDim.x) * p.mblk_bytes;
+  const uint8_t* base = p.mtiles + static_cast<size_t>(blockIdx.x) * p.mblk_bytes;
+  const uint8_t* g_codes = base + p.off_A + chunk0 * kAChunkBytes + lane * 16;
+  const uint8_t* g_sa = base + p.off_sA + lane * 16;
+  const bool sa_lane = lane < 2;
 #pragma unroll
   for (int k = 0; k < kRing; ++k) {
-    if (k < n_my) issue_corr(p, chunk0, nch, ring + k * sbytes, k, lane);
+    if (k < n_my) issue_corr(ring_s + k * sbytes, g_codes + k * stride, g_sa + k * stride, nch, sa_lane);
     cp_async_commit();
   }
+  g_codes += kRing * stride;
+  g_sa += kRing * stride;
   grid_dependency_wait();
   const bool tok = gr < p.nt;
   uint32_t zf[kCA][2][2][2];
@@ -420,8 +474,11 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
   const float zs = tok ? ldexpf(1.f, p.escale[p.t0 + gr] + p.e_B - kScaleExp) : 0.f;
   const float2 unscale = column_pair(zs, lane);
 
+  float* tile = nullptr;
   for (int i = 0; i < n_my; ++i) {
-    uint8_t* slot = ring + (i % kRing) * sbytes;
+    if ((i & (p.mg - 1)) == 0) tile = group_begin(sv, p, i, cw, lane);
+    const uint32_t k = static_cast<uint32_t>(i) & (kRing - 1);
+    const uint8_t* slot = ring + k * sbytes;
     cp_async_wait<kRing - 1>();
     __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -445,9 +502,12 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
     acc[2] = (acc[2] - cbc.x) * (sc.y * unscale.x);
     acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
     __syncwarp();
-    if (i + kRing < n_my) issue_corr(p, chunk0, nch, slot, i + kRing, lane);
+    if (i + kRing < n_my) issue_corr(ring_s + k * sbytes, g_codes, g_sa, nch, sa_lane);
+    g_codes += stride;
+    g_sa += stride;
     cp_async_commit();
-    finish_mtile(sv, p, i, cw, lane, acc);
+    store_partial(tile, p, i, lane, acc);
+    group_end(sv, p, i, n_my, lane);
   }
   cp_async_wait_all();
 }
@@ -455,37 +515,40 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
 // ------------------------------------------------------------ epilogue warp
 __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int lane) {
   grid_dependency_wait();   // the workspace is shared with the previous launch
-  const int nel = 16 * p.nt;
+  // Lane l, slot k holds element e = l + 32k of every group tile (fixed token).
   LseState st[kEpiSlots];
   int target[kEpiSlots];
 #pragma unroll
   for (int k = 0; k < kEpiSlots; ++k) {
     st[k] = lse_init();
     const int e = lane + 32 * k;
-    target[k] = (e < nel && p.targets != nullptr) ? p.targets[p.t0 + (e >> 4)] : -1;
+    target[k] = p.targets != nullptr ? p.targets[p.t0 + (e >> 4) % p.nt] : -1;
   }
-  for (int i = 0; i < n_my; ++i) {
-    const int r = i & (p.slots - 1);
-    const bool ok = warp_wait(sv, &sv.reduced[r], (i >> p.slots_log2) & 1, p.status, lane);
-    const float* part = sv.part + r * p.nw_work * nel;
-    const int vbase = mtile_of(i) * kMT;
+  const int ngroups = (n_my + p.mg - 1) >> p.mg_log2;
+  for (int grp = 0; grp < ngroups; ++grp) {
+    const int r = grp & (p.slots - 1);
+    const bool ok = warp_wait(sv, &sv.reduced[r], (grp >> p.slots_log2) & 1, p.status, lane);
+    const float* part = sv.part + r * p.nw_work * (kGroupTile * 16);
+    const int i0 = grp << p.mg_log2;
 #pragma unroll
     for (int k = 0; k < kEpiSlots; ++k) {
+      // element e = (m * nt + t) * 16 + row of this group's tile
       const int e = lane + 32 * k;
-      if (ok && e < nel) {
+      const int m = e / (16 * p.nt);
+      if (ok && m < p.mg && i0 + m < n_my) {
         // warp-order sum with four independent chains
         float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
         int w = 0;
         for (; w + 4 <= p.nw_work; w += 4) {
-          y0 += part[(w + 0) * nel + e];
-          y1 += part[(w + 1) * nel + e];
-          y2 += part[(w + 2) * nel + e];
-          y3 += part[(w + 3) * nel + e];
+          y0 += part[(w + 0) * (kGroupTile * 16) + e];
+          y1 += part[(w + 1) * (kGroupTile * 16) + e];
+          y2 += part[(w + 2) * (kGroupTile * 16) + e];
+          y3 += part[(w + 3) * (kGroupTile * 16) + e];
         }
-        for (; w < p.nw_work; ++w) y0 += part[w * nel + e];
+        for (; w < p.nw_work; ++w) y0 += part[w * (kGroupTile * 16) + e];
         const float y = (y0 + y1) + (y2 + y3);
-        const int row = e & 15, t = e >> 4;
-        const int v = vbase + row;
+        const int row = e & 15, t = (e >> 4) - m * p.nt;
+        const int v = mtile_of(i0 + m) * kMT + row;
         if (v < p.V) {
           lse_push(st[k], y, v);
           if (p.logits != nullptr) p.logits[static_cast<size_t>(p.t0 + t) * p.V + v] = y;
@@ -496,15 +559,26 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&sv.redfree[r]));
   }
-  // Block partial per token: slot k of lanes 16h..16h+15 holds token 2k + h.
+  // Block partial per token: the 16 lanes of half-warp h in slot k hold
+  // element rows of token ((32k + 16h) / 16) mod nt; merge per half-warp,
+  // then gather the half-warps of each token through shared memory order.
 #pragma unroll
   for (int k = 0; k < kEpiSlots; ++k) {
 #pragma unroll
     for (int m = 8; m >= 1; m >>= 1) st[k] = lse_merge(st[k], lse_shfl_xor(st[k], m));
-    const int t = 2 * k + (lane >> 4);
-    if ((lane & 15) == 0 && t < p.nt)
+  }
+  for (int t = 0; t < p.nt; ++t) {
+    // half-warp q = 2k + (lane >> 4) carries token q mod nt
+    LseState a = lse_init();
+#pragma unroll
+    for (int k = 0; k < kEpiSlots; ++k) {
+      const LseState lo = lse_shfl_idx(st[k], 0), hi = lse_shfl_idx(st[k], 16);
+      if ((2 * k) % p.nt == t) a = lse_merge(a, lo);
+      if ((2 * k + 1) % p.nt == t) a = lse_merge(a, hi);
+    }
+    if (lane == 0)
       p.partials[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] =
-          make_float4(st[k].m, st[k].s, __int_as_float(st[k].idx), 0.f);
+          make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
   }
   __threadfence();
   __syncwarp();
@@ -585,7 +659,7 @@ void decode_smem_plan(DecodeParams& p, int g_steps) {
 }
 
 size_t decode_smem_bytes(const DecodeParams& p) {
-  return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nw_work * p.nt * 16 * 4 +
+  return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16 * 4 +
          static_cast<size_t>(2) * p.slots * 8 + 16;
 }
 

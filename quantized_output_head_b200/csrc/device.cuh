@@ -214,6 +214,13 @@ __device__ __forceinline__ LseState lse_merge(const LseState& a, const LseState&
   else r.idx = min(a.idx, b.idx);
   return r;
 }
+__device__ __forceinline__ LseState lse_shfl_idx(const LseState& a, int src) {
+  LseState o;
+  o.m = __shfl_sync(0xffffffffu, a.m, src);
+  o.s = __shfl_sync(0xffffffffu, a.s, src);
+  o.idx = __shfl_sync(0xffffffffu, a.idx, src);
+  return o;
+}
 __device__ __forceinline__ LseState lse_shfl_xor(const LseState& a, int mask) {
   LseState o;
   o.m = __shfl_xor_sync(0xffffffffu, a.m, mask);

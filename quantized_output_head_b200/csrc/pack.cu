@@ -147,6 +147,7 @@ bool plan_decode(archead_handle* h, int smem_optin) {
   dp.nw_work = nw_work;
   dp.nt = kDecodeTokens;
   dp.slots = 4;
+  dp.mg = 1;
   decode_smem_plan(dp, L.g_steps);
   if (decode_smem_bytes(dp) > static_cast<size_t>(smem_optin)) return false;
   h->nw_res = nw_res;

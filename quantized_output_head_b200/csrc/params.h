@@ -38,6 +38,7 @@ struct DecodeParams {
   uint32_t off_res, off_Lnib, off_Lhi, off_A, off_sres, off_sL, off_sA, mblk_bytes;
   int32_t nw_res, nw_L, nw_A, nw_work;   // compute warps by role
   int32_t slots, slots_log2;   // partial-logit slots between compute and epilogue warps (power of two)
+  int32_t mg, mg_log2;         // m-tiles per partial-logit group (mg * nt <= 8, power of two)
   // Shared-memory rings: one per compute warp, kRing slices each.
   uint32_t res_slice_bytes, core_slice_bytes, corr_slice_bytes;
   uint32_t core_ring_off, corr_ring_off, ring_bytes;
