@@ -159,6 +159,24 @@ ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint
                                         int32_t* argmax_host, float* ce_host, void* workspace,
                                         size_t workspace_bytes, archead_stream_t stream);
 
+/* Allocation-free form of archead_logits_lse_argmax, for callers that may not
+ * allocate device memory when they run the head (for example while a CUDA
+ * graph is being captured under an allocator that forbids it, or inside a
+ * host framework that owns all device memory).  Same arguments and results,
+ * without the workspace: scratch comes from a fixed array of
+ * archead_static_workspace_capacity() bytes (2 MiB) in the library's own device
+ * memory, held by every GPU that loads the library until the process exits.
+ * The first call on a device, with that device current, looks the array up
+ * (cudaGetSymbolAddress) and clears its status word, so make that first call
+ * before any stream capture.  All calls on a device share the array: calls
+ * that may overlap on the GPU race.  A T whose workspace would not fit the
+ * array returns ARCHEAD_ENOMEM.  (No counterpart in the paper: a library
+ * convenience.) */
+ARCHEAD_API size_t archead_static_workspace_capacity(void);
+ARCHEAD_API int archead_logits_lse_argmax_static(const archead_handle* handle, const uint16_t* hidden,
+                                                 int32_t T, const int32_t* targets, float* lse,
+                                                 int32_t* argmax, float* ce, archead_stream_t stream);
+
 /* Read (and with clear != 0, reset) the device status word of a workspace:
  * a bitwise OR of ARCHEAD_STATUS_* since the last clear.  Synchronises the
  * stream.  Returns ARCHEAD_ETIMEOUT if ARCHEAD_STATUS_WAIT_TIMEOUT is set. */

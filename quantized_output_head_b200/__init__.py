@@ -32,7 +32,7 @@ EXPORTED = (
     "archead_workspace_bytes",
     "archead_logits", "archead_logits_lse_argmax", "archead_host_workspace_bytes", "archead_lse_argmax_host",
     "archead_workspace_status", "archead_set_profile_events", "archead_free", "archead_last_cuda_error",
-    "archead_status_string",
+    "archead_status_string", "archead_static_workspace_capacity", "archead_logits_lse_argmax_static",
 )
 
 
@@ -59,6 +59,8 @@ _sig = {
     "archead_lse_argmax_host": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "archead_workspace_status": (ctypes.c_int, [_vp, ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "archead_set_profile_events": (ctypes.c_int, [_vp, _vp, _vp]),
+    "archead_static_workspace_capacity": (_sz, []),
+    "archead_logits_lse_argmax_static": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "archead_free": (None, [_vp]),
     "archead_last_cuda_error": (ctypes.c_int, []),
     "archead_status_string": (ctypes.c_char_p, [ctypes.c_int]),

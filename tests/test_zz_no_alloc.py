@@ -1,0 +1,61 @@
+"""The allocation-free entry point gives the same results as the workspace one.
+
+archead_logits_lse_argmax_static exists for callers that cannot allocate
+device memory when they run the head (graph capture under an allocator that
+forbids it, host frameworks that own all device memory).  It takes no
+workspace; its scratch is a fixed device array inside the library.  This file
+is collected last so that a failure here stops a -x run only after every other
+test has run; it must also pass on its own in a fresh process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import archead_inputs as gen
+import oracle
+from parity import check_argmax, check_lse_ce
+
+pytestmark = pytest.mark.gpu
+
+
+def test_static_entry_matches_workspace_entry_twice():
+    import quantized_output_head_b200 as qoh
+    lib = qoh._lib
+    shape = (1000, 256, 32, 8, 64, 64)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=2024)
+    h_bits, targets = gen.random_hidden(256, 5, seed=2025, V=shape[0])
+    head = qoh.PackedHead(*shape, comps)
+    hd = torch.from_numpy(h_bits.view(np.int16)).cuda()
+    td = torch.from_numpy(targets).cuda()
+    ref_lse, ref_am, ref_ce = head.lse_argmax(hd, td)
+    y, rowmax = oracle.logits(comps, 64, 64, h_bits)
+    tol = oracle.tolerance(h_bits, rowmax)
+    stream = torch.cuda.current_stream().cuda_stream
+    for _ in range(2):
+        lse = torch.full((5,), float("nan"), device="cuda")
+        am = torch.full((5,), -1, dtype=torch.int32, device="cuda")
+        ce = torch.full((5,), float("nan"), device="cuda")
+        rc = lib.archead_logits_lse_argmax_static(head.handle, hd.data_ptr(), 5, td.data_ptr(), lse.data_ptr(),
+                                                   am.data_ptr(), ce.data_ptr(), stream)
+        assert rc == qoh.ARCHEAD_OK, lib.archead_status_string(rc)
+        torch.cuda.synchronize()
+        np.testing.assert_allclose(lse.cpu().numpy(), ref_lse.cpu().numpy(), rtol=0, atol=float(tol.max()))
+        np.testing.assert_allclose(ce.cpu().numpy(), ref_ce.cpu().numpy(), rtol=0, atol=2 * float(tol.max()))
+        assert np.array_equal(am.cpu().numpy(), ref_am.cpu().numpy())
+        check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, targets)
+        check_argmax(am.cpu().numpy(), y, tol)
+
+
+def test_static_entry_rejects_too_many_tokens():
+    import quantized_output_head_b200 as qoh
+    lib = qoh._lib
+    shape = (64, 64, 16, 8, 16, 16)
+    head = qoh.PackedHead(*shape, gen.random_components(gen.HeadShape(*shape), seed=7))
+    cap = lib.archead_static_workspace_capacity()
+    T = 1
+    while lib.archead_workspace_bytes(head.handle, T) <= cap:
+        T *= 2
+    rc = lib.archead_logits_lse_argmax_static(head.handle, 4096, T, None, 4096, 4096, None, None)
+    assert rc == qoh.ARCHEAD_ENOMEM
