@@ -99,10 +99,14 @@ def vocab_pass_bytes_per_launch(shape, nt, op, Kz):
             + 4 * nt * (op["argmax"] + op["lse"] + op["ce"]))
 
 
+DECODE_SOURCES = ("decode.cu", "device.cuh", "params.h", "layout.h")
+
+
 def source_hash():
+    """Hash of the sources the vocabulary-pass kernel is compiled from."""
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "quantized_output_head_b200", "csrc")
-    for f in sorted(os.listdir(cs)):
+    for f in DECODE_SOURCES:
         h.update(open(os.path.join(cs, f), "rb").read())
     return h.hexdigest()[:16]
 
