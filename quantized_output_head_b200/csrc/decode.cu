@@ -221,6 +221,52 @@ __device__ __forceinline__ void residual_tile(const uint8_t* slot, const ResSlic
   }
 }
 
+// Two m-tiles of a residual warp at once (all 4 chunks present): the two
+// independent MMA chains interleave, so the warp has work while one waits.
+template <int G>
+__device__ __forceinline__ void residual_tile_pair(const uint8_t* slot_a, const uint8_t* slot_b, const ResSlice& rs,
+                                                   const uint32_t (&hf)[kCRes][4][2], const float2 (&cgc)[16 / G],
+                                                   int step0, int g_log2, int lane, float (&acc_a)[4],
+                                                   float (&acc_b)[4]) {
+  const int gr = lane >> 2;
+  float ta[4] = {0.f, 0.f, 0.f, 0.f};
+  float tb[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint8_t* sres_a = slot_a + kCRes * kResChunkBytes + gr * 4;
+  const uint8_t* sres_b = slot_b + kCRes * kResChunkBytes + gr * 4;
+#pragma unroll
+  for (int c = 0; c < kCRes; ++c) {
+    const uint4 na = *reinterpret_cast<const uint4*>(slot_a + c * kResChunkBytes + lane * 16);
+    const uint4 nb = *reinterpret_cast<const uint4*>(slot_b + c * kResChunkBytes + lane * 16);
+    const uint32_t wa[4] = {na.x, na.y, na.z, na.w};
+    const uint32_t wb[4] = {nb.x, nb.y, nb.z, nb.w};
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+      const int step = 4 * c + st;
+      uint32_t a[4];
+      unpack_int4_biased(wa[st], a);
+      mma_f16_16816(ta, a, hf[c][st][0], hf[c][st][1]);
+      unpack_int4_biased(wb[st], a);
+      mma_f16_16816(tb, a, hf[c][st][0], hf[c][st][1]);
+      if ((step + 1) % G == 0) {
+        const int lg = step / G;
+        const int grp = ((step0 + step) >> g_log2) - rs.grp0;
+        const float2 sa = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(sres_a + grp * kSresGroupBytes));
+        const float2 sb = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(sres_b + grp * kSresGroupBytes));
+        acc_a[0] = fmaf(sa.x, ta[0] - cgc[lg].x, acc_a[0]);
+        acc_a[1] = fmaf(sa.x, ta[1] - cgc[lg].y, acc_a[1]);
+        acc_a[2] = fmaf(sa.y, ta[2] - cgc[lg].x, acc_a[2]);
+        acc_a[3] = fmaf(sa.y, ta[3] - cgc[lg].y, acc_a[3]);
+        acc_b[0] = fmaf(sb.x, tb[0] - cgc[lg].x, acc_b[0]);
+        acc_b[1] = fmaf(sb.x, tb[1] - cgc[lg].y, acc_b[1]);
+        acc_b[2] = fmaf(sb.y, tb[2] - cgc[lg].x, acc_b[2]);
+        acc_b[3] = fmaf(sb.y, tb[3] - cgc[lg].y, acc_b[3]);
+        ta[0] = ta[1] = ta[2] = ta[3] = 0.f;
+        tb[0] = tb[1] = tb[2] = tb[3] = 0.f;
+      }
+    }
+  }
+}
+
 // G = k16 steps per scale group within the warp's 16 steps (16 when a group
 // spans the whole warp range or more).
 template <int G>
@@ -288,7 +334,43 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
   const int step0 = wres * 16;
 
   float* tile = nullptr;
-  for (int i = 0; i < n_my; ++i) {
+  int i = 0;
+  if (full && G == 8) {
+    // Pairs of m-tiles (two scale groups per warp range; smaller groups keep
+    // too many per-group sums live for two tiles).
+    for (; i + 1 < n_my; i += 2) {
+      const uint32_t k = static_cast<uint32_t>(i) & (kRing - 1);   // even: k, k + 1 < kRing
+      const uint8_t* slot = ring + k * sbytes;
+      cp_async_wait<kRing - 2>();
+      __syncwarp();
+      float acc_a[4] = {0.f, 0.f, 0.f, 0.f};
+      float acc_b[4] = {0.f, 0.f, 0.f, 0.f};
+      residual_tile_pair<G>(slot, slot + sbytes, rs, hf, cgc, step0, p.g_steps_log2, lane, acc_a, acc_b);
+      acc_a[0] *= unscale.x;
+      acc_a[1] *= unscale.y;
+      acc_a[2] *= unscale.x;
+      acc_a[3] *= unscale.y;
+      acc_b[0] *= unscale.x;
+      acc_b[1] *= unscale.y;
+      acc_b[2] *= unscale.x;
+      acc_b[3] *= unscale.y;
+      __syncwarp();   // every lane is done reading both slots
+      if (i + kRing < n_my) issue_res<true>(ring_s + k * sbytes, g_codes, g_scales, kCRes, scale_lane);
+      cp_async_commit();
+      if (i + 1 + kRing < n_my)
+        issue_res<true>(ring_s + (k + 1) * sbytes, g_codes + stride, g_scales + stride, kCRes, scale_lane);
+      cp_async_commit();
+      g_codes += 2 * stride;
+      g_scales += 2 * stride;
+      if ((i & (p.mg - 1)) == 0) tile = group_begin(sv, p, i, cw, lane);
+      store_partial(tile, p, i, lane, acc_a);
+      group_end(sv, p, i, n_my, lane);
+      if (((i + 1) & (p.mg - 1)) == 0) tile = group_begin(sv, p, i + 1, cw, lane);
+      store_partial(tile, p, i + 1, lane, acc_b);
+      group_end(sv, p, i + 1, n_my, lane);
+    }
+  }
+  for (; i < n_my; ++i) {
     if ((i & (p.mg - 1)) == 0) tile = group_begin(sv, p, i, cw, lane);
     const uint32_t k = static_cast<uint32_t>(i) & (kRing - 1);
     const uint8_t* slot = ring + k * sbytes;
