@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libarchead.so")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
-SOURCES = ["pack.cu", "api.cu", "decode.cu", "prologue.cu", "static_ws.cu"]
+SOURCES = ["pack.cu", "api.cu", "decode.cu", "prologue.cu", "static_ws.cu", "actprep.cu", "tcgemm.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-Xptxas", "-v",
          "--expt-relaxed-constexpr"]

@@ -1,0 +1,238 @@
+// Activation operand of the tensor-core forward (ARCHead paper, §3.2 Eq. 7:
+// the factored form h·R^T then L, and the correction h·B^T then A).
+//
+// For a tile of 16 tokens the kernel computes, per token t,
+//   E_t with max_j |h[t,j]| < 2^E_t and c_t = kScaleExp - E_t + mseg,
+// and writes one fp16 row of the concatenated activation matrix
+//   X[t] = [ h[t]·2^(c_t-alpha) | z_c[t]·2^(c_t-beta) | z_r[t]·2^(c_t-gamma) ],
+//   z_c[t,k] = s_R[k] sum_j R[k,j] h[t,j],   z_r[t,k] = sum_j s_B[k,j/g_B] B[k,j] h[t,j].
+// alpha, beta, gamma put the largest dequantised weight of each segment just
+// below 2^kScaleExp; mseg = min(alpha, beta - e_B, gamma - e_B) keeps every
+// entry of X below 2^kScaleExp as well (2^e_B bounds the L1 norm of each
+// dequantised R and B row), so the product of the two sides is
+// y[t,v]·2^c_t with no fp16 overflow.
+//
+// grid.y = Kz'/64 + 1: blocks y < Kz'/64 compute 64 entries of z for the 16
+// tokens with m16n8k16 MMAs (tokens as M, z rows as N, fp16 h scaled by
+// 2^(kScaleExp - E_t), exact int8 codes as fp16, fp32 accumulation; the
+// group scales of B are applied in fp32 at each group end); block y = last
+// converts h.  Within every 16-column block X is stored in the column order
+// of the dequantised weights in tensor memory (tc_kpos).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "device.cuh"
+#include "params.h"
+#include "tc_params.h"
+#include "tcgen05.cuh"
+
+namespace archead {
+
+namespace {
+
+// bf16 pair -> fp16 pair times 2^e (exact while the result is a normal fp16).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t bits, float scale) {
+  const float lo = __uint_as_float(bits << 16) * scale;
+  const float hi = __uint_as_float(bits & 0xFFFF0000u) * scale;
+  return pack_half2(lo, hi);
+}
+
+// int8 quadruple (columns c..c+3) -> exact fp16 pairs (c, c+1) and (c+2, c+3).
+__device__ __forceinline__ void int8x4_to_f16(uint32_t w, uint32_t& b0, uint32_t& b1) {
+  const uint32_t u = w ^ 0x80808080u;   // offset binary: code + 128
+  b0 = hsub2_bits(__byte_perm(u, 0x64646464u, 0x4140u), kH2_1152);
+  b1 = hsub2_bits(__byte_perm(u, 0x64646464u, 0x4342u), kH2_1152);
+}
+
+// One warp's share of the 16-token x 64-row block of z, over 64-column blocks
+// [b0, b1) of d.  kCorr: rows of B with group scales (flushed in fp32 at every
+// group end); otherwise rows of R (row scale applied by the caller).
+// The k order inside an MMA is a permutation of the columns that A and B
+// share: lane cc covers columns 16cc..16cc+15 of each 64-column block, step st
+// columns 16cc + 4st + 0..3.
+template <bool kCorr>
+__device__ __forceinline__ void z_block(const ActParams& p, int n0, int b0, int b1, const float (&hs)[2],
+                                        const uint16_t* hrow_a, const uint16_t* hrow_b, int lane,
+                                        float (&acc)[8][4]) {
+  const int gr = lane >> 2, cc = lane & 3;
+  const int ngB = p.d / p.g_B;
+  float tmp[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) tmp[n][e] = 0.f;
+  const int8_t* rows[8];
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const int zr = n0 + 8 * n + gr;
+    rows[n] = nullptr;
+    if (zr < p.Kz) rows[n] = kCorr ? p.B + static_cast<size_t>(zr - p.rcp) * p.d : p.R + static_cast<size_t>(zr) * p.d;
+  }
+  for (int blk = b0; blk < b1; ++blk) {
+    const int c0 = blk * 64 + 16 * cc;
+    uint32_t ha[4][4];
+    {
+      uint4 a0 = make_uint4(0, 0, 0, 0), a1 = a0, b0v = a0, b1v = a0;
+      if (hrow_a != nullptr) {
+        a0 = *reinterpret_cast<const uint4*>(hrow_a + c0);
+        a1 = *reinterpret_cast<const uint4*>(hrow_a + c0 + 8);
+      }
+      if (hrow_b != nullptr) {
+        b0v = *reinterpret_cast<const uint4*>(hrow_b + c0);
+        b1v = *reinterpret_cast<const uint4*>(hrow_b + c0 + 8);
+      }
+      const uint32_t pa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint32_t pb[8] = {b0v.x, b0v.y, b0v.z, b0v.w, b1v.x, b1v.y, b1v.z, b1v.w};
+#pragma unroll
+      for (int st = 0; st < 4; ++st) {
+        ha[st][0] = bf16x2_to_f16x2(pa[2 * st], hs[0]);
+        ha[st][2] = bf16x2_to_f16x2(pa[2 * st + 1], hs[0]);
+        ha[st][1] = bf16x2_to_f16x2(pb[2 * st], hs[1]);
+        ha[st][3] = bf16x2_to_f16x2(pb[2 * st + 1], hs[1]);
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      uint4 rv = make_uint4(0, 0, 0, 0);
+      if (rows[n] != nullptr) rv = *reinterpret_cast<const uint4*>(rows[n] + c0);
+      const uint32_t wv[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+      for (int st = 0; st < 4; ++st) {
+        uint32_t bb0, bb1;
+        int8x4_to_f16(wv[st], bb0, bb1);
+        if constexpr (kCorr) mma_f16_16816(tmp[n], ha[st], bb0, bb1);
+        else mma_f16_16816(acc[n], ha[st], bb0, bb1);
+      }
+    }
+    if (kCorr && (((blk + 1) * 64) % p.g_B == 0 || blk + 1 == b1)) {
+      const int grp = (blk * 64) / p.g_B;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const int zc = n0 + 8 * n + 2 * cc;
+        const float s0 = zc < p.Kz ? __half2float(__ushort_as_half(p.s_B[static_cast<size_t>(zc - p.rcp) * ngB + grp])) : 0.f;
+        const float s1 =
+            zc + 1 < p.Kz ? __half2float(__ushort_as_half(p.s_B[static_cast<size_t>(zc + 1 - p.rcp) * ngB + grp])) : 0.f;
+        acc[n][0] = fmaf(s0, tmp[n][0], acc[n][0]);
+        acc[n][1] = fmaf(s1, tmp[n][1], acc[n][1]);
+        acc[n][2] = fmaf(s0, tmp[n][2], acc[n][2]);
+        acc[n][3] = fmaf(s1, tmp[n][3], acc[n][3]);
+        tmp[n][0] = tmp[n][1] = tmp[n][2] = tmp[n][3] = 0.f;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(256) act_prep_kernel(const ActParams p) {
+  __shared__ float red[8][16][64];
+  __shared__ int s_E[16];
+  // The tensor-core kernel may start streaming the packed head right away; it
+  // waits (griddepcontrol.wait) before it reads anything written here.
+  grid_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * 16;
+  if (p.targets != nullptr && blockIdx.x == 0 && blockIdx.y == 0) {
+    for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
+      const int v = p.targets[t];
+      if (v < 0 || v >= p.V) atomicOr(p.status, static_cast<uint32_t>(ARCHEAD_STATUS_BAD_TARGET));
+    }
+  }
+  // E_t of the tile's tokens: |bf16| orders like its bit pattern without the sign.
+  for (int tt = 0; tt < 2; ++tt) {
+    const int tl = 2 * warp + tt, t = t0 + tl;
+    uint32_t mx = 0;
+    if (t < p.T) {
+      const uint4* row = reinterpret_cast<const uint4*>(p.hidden + static_cast<size_t>(t) * p.d);
+      for (int i = lane; i < p.d / 8; i += 32) {
+        const uint4 v = row[i];
+        mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.w & 0x7FFF7FFFu);
+      }
+    }
+    const uint32_t m16 = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
+    if (lane == 0) {
+      int E = 0;
+      if (m16 != 0) frexpf(__uint_as_float(m16 << 16), &E);   // max|h_t| < 2^E
+      s_E[tl] = E;
+    }
+  }
+  __syncthreads();
+
+  if (blockIdx.y == gridDim.y - 1) {
+    // h segment: X[t, j] = h[t, j]·2^(c_t - alpha), c_t = kScaleExp - E_t + mseg.
+    if (threadIdx.x < 16 && t0 + static_cast<int>(threadIdx.x) < p.T)
+      p.cexp[t0 + threadIdx.x] = kScaleExp - s_E[threadIdx.x] + p.mseg;
+    const int nb16 = p.d / 16;
+    for (int item = threadIdx.x; item < 16 * nb16; item += blockDim.x) {
+      const int tl = item / nb16, b = item - tl * nb16, t = t0 + tl;
+      if (t >= p.T) break;
+      const float sc = ldexpf(1.f, kScaleExp - s_E[tl] + p.mseg - p.alpha);
+      const uint4* src = reinterpret_cast<const uint4*>(p.hidden + static_cast<size_t>(t) * p.d + b * 16);
+      const uint4 lo = src[0], hi = src[1];
+      const uint32_t in[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};   // column pairs 2i, 2i+1
+      uint32_t out[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) out[jj] = bf16x2_to_f16x2(in[(jj >> 1) + 4 * (jj & 1)], sc);
+      uint4* dst = reinterpret_cast<uint4*>(p.xop + static_cast<size_t>(t) * p.Kc + b * 16);
+      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+    return;
+  }
+
+  // z segment: rows n0 .. n0 + 63 of (R | B), all of one kind (r_c' is a multiple of 64).
+  const int n0 = blockIdx.y * 64;
+  const int gr = lane >> 2;
+  const int nb = p.d / 64;
+  const int b0 = warp * nb / 8, b1 = (warp + 1) * nb / 8;
+  const int ta = t0 + gr, tb = t0 + gr + 8;
+  const float hs[2] = {ta < p.T ? ldexpf(1.f, kScaleExp - s_E[gr]) : 0.f,
+                       tb < p.T ? ldexpf(1.f, kScaleExp - s_E[gr + 8]) : 0.f};
+  const uint16_t* hrow_a = ta < p.T ? p.hidden + static_cast<size_t>(ta) * p.d : nullptr;
+  const uint16_t* hrow_b = tb < p.T ? p.hidden + static_cast<size_t>(tb) * p.d : nullptr;
+  float acc[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+  const bool corr = n0 >= p.rcp;
+  if (corr) z_block<true>(p, n0, b0, b1, hs, hrow_a, hrow_b, lane, acc);
+  else z_block<false>(p, n0, b0, b1, hs, hrow_a, hrow_b, lane, acc);
+  const int cc = lane & 3;
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    red[warp][gr][8 * n + 2 * cc] = acc[n][0];
+    red[warp][gr][8 * n + 2 * cc + 1] = acc[n][1];
+    red[warp][gr + 8][8 * n + 2 * cc] = acc[n][2];
+    red[warp][gr + 8][8 * n + 2 * cc + 1] = acc[n][3];
+  }
+  __syncthreads();
+  // X[t, d + n] = z·2^(c_t - beta|gamma): with c_t = kScaleExp - E_t + mseg the
+  // token exponent cancels against the 2^(kScaleExp - E_t) of h.
+  const float sc_core = ldexpf(1.f, p.mseg - p.beta);
+  const float sc_corr = ldexpf(1.f, p.mseg - p.gamma);
+  for (int idx = threadIdx.x; idx < 16 * 64; idx += blockDim.x) {
+    const int tl = idx >> 6, c = idx & 63, t = t0 + tl, n = n0 + c;
+    if (t >= p.T) continue;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[w][tl][c];
+    float val = 0.f;
+    if (n < p.rcp) val = s * __half2float(__ushort_as_half(p.s_R[n])) * sc_core;
+    else if (n < p.Kz) val = s * sc_corr;
+    const int col = p.d + (n & ~15) + tc_kpos(n & 15);
+    p.xop[static_cast<size_t>(t) * p.Kc + col] = __half_as_ushort(__float2half_rn(val));
+  }
+}
+
+cudaError_t launch_act_prep(const ActParams& p, cudaStream_t stream) {
+  const dim3 grid((p.T + 15) / 16, (p.Kc - p.d) / 64 + 1);
+  act_prep_kernel<<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace archead

@@ -4,6 +4,7 @@
 // on the caller's stream, with no host synchronisation.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstring>
 
 #include "handle.h"
@@ -24,6 +25,100 @@ int check_device(const archead_handle* h) {
   return dev == h->device ? ARCHEAD_OK : ARCHEAD_EINVAL;
 }
 
+// Tensor-core path: activation operand, the tensor-core kernel, and the
+// per-token fold of its partials.
+int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const int32_t* targets, float* logits,
+               int32_t* argmax, float* lse, float* ce, uint8_t* wb, const WsLayout& w, cudaStream_t stream) {
+  const Layout& L = h->L;
+  const int Kc = tc_kc(L);
+  uint32_t* status = reinterpret_cast<uint32_t*>(wb + w.status);
+  int32_t* cexp = reinterpret_cast<int32_t*>(wb + w.cexp);
+  uint16_t* xop = reinterpret_cast<uint16_t*>(wb + w.xop);
+  float4* partials = reinterpret_cast<float4*>(wb + w.tpartials);
+  float* tgt = reinterpret_cast<float*>(wb + w.tgt);
+
+  ActParams ap{};
+  ap.hidden = hidden;
+  ap.R = reinterpret_cast<const int8_t*>(h->arena + L.off_R);
+  ap.s_R = reinterpret_cast<const uint16_t*>(h->arena + L.off_sR);
+  ap.B = reinterpret_cast<const int8_t*>(h->arena + L.off_B);
+  ap.s_B = reinterpret_cast<const uint16_t*>(h->arena + L.off_sB);
+  ap.targets = targets;
+  ap.status = status;
+  ap.xop = xop;
+  ap.cexp = cexp;
+  ap.T = T;
+  ap.d = L.d;
+  ap.rcp = L.rcp;
+  ap.Kz = L.Kz;
+  ap.Kc = Kc;
+  ap.g_B = L.g_B;
+  ap.V = L.V;
+  ap.alpha = h->tc_alpha;
+  ap.beta = h->tc_beta;
+  ap.gamma = h->tc_gamma;
+  ap.mseg = h->tc_mseg;
+  cudaError_t e = launch_act_prep(ap, stream);
+  if (e != cudaSuccess) return set_cuda_error(e);
+
+  TcParams tp{};
+  tp.mtiles = h->arena;
+  tp.targets = targets;
+  tp.cexp = cexp;
+  tp.logits = logits;
+  tp.partials = partials;
+  tp.tgt = tgt;
+  tp.status = status;
+  tp.T = T;
+  tp.V = L.V;
+  tp.n_nt = (T + kTcMaxBN - 1) / kTcMaxBN;
+  const int per = (T + tp.n_nt - 1) / tp.n_nt;
+  tp.BN = (per + 15) / 16 * 16;
+  tp.n_mt128 = tc_n_mt128(L);
+  tp.n_units = tp.n_mt128 * tp.n_nt;
+  tp.n_res = L.n_res;
+  tp.n_L = L.n_L;
+  tp.n_A = L.n_A;
+  tp.n_mtiles = L.n_mtiles;
+  int lg = 0;
+  while ((1 << lg) < L.g) ++lg;
+  tp.g_log2 = lg;
+  tp.ks_core = L.n_res;
+  tp.ks_corr = L.n_res + L.n_L;
+  tp.n_ks = Kc / kTcBK;
+  tp.off_res = L.off_res;
+  tp.off_Lnib = L.off_Lnib;
+  tp.off_Lhi = L.off_Lhi;
+  tp.off_A = L.off_A;
+  tp.off_sres = L.off_sres;
+  tp.off_sL = L.off_sL;
+  tp.off_sA = L.off_sA;
+  tp.mblk_bytes = L.mblk_bytes;
+  tp.sc_res = std::ldexp(1.f, h->tc_alpha);
+  tp.sc_L = std::ldexp(1.f, h->tc_beta);
+  tp.sc_A = std::ldexp(1.f, h->tc_gamma);
+  tc_smem_plan(tp);
+  CUtensorMap map;
+  e = tc_encode_xmap(&map, xop, T, Kc, tp.BN);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  const int grid = tp.n_units < h->num_sms ? tp.n_units : h->num_sms;
+  if (h->ev_before != nullptr) {
+    e = cudaEventRecord(h->ev_before, stream);
+    if (e != cudaSuccess) return set_cuda_error(e);
+  }
+  e = launch_tc(tp, map, grid, stream);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  if (h->ev_after != nullptr) {
+    e = cudaEventRecord(h->ev_after, stream);
+    if (e != cudaSuccess) return set_cuda_error(e);
+  }
+  if (argmax != nullptr || lse != nullptr || ce != nullptr) {
+    e = launch_tc_merge(partials, tp.n_mt128, T, targets, tgt, L.V, lse, argmax, ce, stream);
+    if (e != cudaSuccess) return set_cuda_error(e);
+  }
+  return ARCHEAD_OK;
+}
+
 int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const int32_t* targets, float* logits,
             int32_t* argmax, float* lse, float* ce, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (h == nullptr || hidden == nullptr || ws == nullptr) return ARCHEAD_EINVAL;
@@ -39,6 +134,7 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   if (dc != ARCHEAD_OK) return dc;
 
   uint8_t* wb = static_cast<uint8_t*>(ws);
+  if (use_tc(*h, T)) return forward_tc(h, hidden, T, targets, logits, argmax, lse, ce, wb, w, stream);
   const Layout& L = h->L;
   uint32_t* counter = reinterpret_cast<uint32_t*>(wb + w.counter);
   uint32_t* status = reinterpret_cast<uint32_t*>(wb + w.status);

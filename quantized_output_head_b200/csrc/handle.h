@@ -1,10 +1,12 @@
 // Host-side handle of a packed head loaded into a caller-owned device arena.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
 #include "layout.h"
 #include "params.h"
+#include "tc_params.h"
 
 struct archead_handle {
   archead::Layout L;
@@ -15,15 +17,30 @@ struct archead_handle {
   int nw_res, nw_L, nw_A, nw_work;   // decode compute warps by role
   int smem_optin;           // shared memory a block may use on this device
   int e_B;                  // 2^e_B bounds the L1 norm of every dequantised R / B row
+  // Tensor-core path (tc_params.h): per-segment weight exponents and whether
+  // the shape can take it.
+  bool tc_ok;
+  int tc_alpha, tc_beta, tc_gamma, tc_mseg;
   cudaEvent_t ev_before;    // optional profiling events (not owned)
   cudaEvent_t ev_after;
 };
 
 namespace archead {
 
+// Calls with at least kTcMinTokens tokens take the tensor-core path when the
+// shape allows it; smaller ones the decode kernel.
+inline bool use_tc(const archead_handle& h, int T) { return h.tc_ok && T >= kTcMinTokens; }
+
+// K columns of the tensor-core path: d + r_c' + r_r' rounded up to 64.
+inline int tc_kc(const Layout& L) { return L.d + L.rcp + static_cast<int>(round_up(L.rrp, 64)); }
+inline int tc_n_mt128(const Layout& L) { return (L.n_mtiles + 7) / 8; }
+
 // Workspace regions of one forward call with T tokens.
 struct WsLayout {
-  size_t counter, status, escale, zhi, zlo, partials, tgt, total;
+  size_t counter, status;
+  size_t escale, zhi, zlo, partials;   // decode path
+  size_t cexp, xop, tpartials;         // tensor-core path
+  size_t tgt, total;
   // host-buffer form only
   size_t h_hidden, h_targets, h_lse, h_argmax, h_ce, host_total;
 };
@@ -35,10 +52,16 @@ inline WsLayout ws_layout(const archead_handle& h, int T) {
   w.counter = 0;
   w.status = 4;
   o = 256;
-  w.escale = o;   o += round_up(t * 4, 256);
-  w.zhi = o;      o += round_up(t * h.L.Kz * 2, 256);
-  w.zlo = o;      o += round_up(t * h.L.Kz * 2, 256);
-  w.partials = o; o += round_up(t * h.grid * 16, 256);
+  if (use_tc(h, T)) {
+    w.cexp = o;      o += round_up(t * 4, 256);
+    w.xop = o;       o += round_up(t * tc_kc(h.L) * 2, 256);
+    w.tpartials = o; o += round_up(t * tc_n_mt128(h.L) * 16, 256);
+  } else {
+    w.escale = o;   o += round_up(t * 4, 256);
+    w.zhi = o;      o += round_up(t * h.L.Kz * 2, 256);
+    w.zlo = o;      o += round_up(t * h.L.Kz * 2, 256);
+    w.partials = o; o += round_up(t * h.grid * 16, 256);
+  }
   w.tgt = o;      o += round_up(t * 4, 256);
   w.total = o;
   w.h_hidden = o;  o += round_up(t * h.L.d * 2, 256);
@@ -56,6 +79,17 @@ size_t decode_smem_bytes(const DecodeParams& p);
 cudaError_t decode_set_attributes(int g_steps, size_t smem);
 cudaError_t launch_decode(int g_steps, const DecodeParams& p, int grid, size_t smem, cudaStream_t stream);
 cudaError_t launch_prologue(const PrologueParams& p, cudaStream_t stream);
+
+// Tensor-core path (actprep.cu, tcgemm.cu).
+cudaError_t launch_act_prep(const ActParams& p, cudaStream_t stream);
+void tc_smem_plan(TcParams& p);
+size_t tc_smem_bytes(const TcParams& p);
+size_t tc_smem_max();
+cudaError_t tc_set_attributes();
+cudaError_t tc_encode_xmap(CUtensorMap* map, const uint16_t* xop, int T, int Kc, int BN);
+cudaError_t launch_tc(const TcParams& p, const CUtensorMap& map, int grid, cudaStream_t stream);
+cudaError_t launch_tc_merge(const float4* partials, int n_mt128, int T, const int32_t* targets, const float* tgt,
+                            int V, float* lse, int32_t* argmax, float* ce, cudaStream_t stream);
 
 // Thread-local record of the last CUDA error (api.cu).
 int set_cuda_error(cudaError_t e);

@@ -180,6 +180,37 @@ int row_norm_exponent(const Layout& L, const archead_host_components& C) {
   return e;
 }
 
+// Smallest e with x < 2^e (x > 0); 0 for x == 0.
+int exp_above(double x) {
+  if (!(x > 0.0)) return 0;
+  int e = 0;
+  std::frexp(x, &e);
+  return e;
+}
+
+double max_abs_half(const uint16_t* s, size_t n) {
+  double m = 0.0;
+  for (size_t i = 0; i < n; ++i) m = std::max(m, std::abs(half_to_double(s[i])));
+  return m;
+}
+
+// Weight exponents of the tensor-core path: each dequantised segment times
+// 2^alpha|beta|gamma stays below 2^kScaleExp (|q| <= 8, |L| <= 16, |A| <= 128),
+// and mseg keeps the activation side below 2^kScaleExp too (z rows are bounded
+// by 2^(E_t + e_B)).
+void plan_tc(archead_handle* h, const archead_host_components& C, int smem_optin) {
+  const Layout& L = h->L;
+  h->tc_alpha = kScaleExp - exp_above(8.0 * max_abs_half(C.s_res, static_cast<size_t>(L.V) * L.n_groups));
+  h->tc_beta = L.r_c > 0 ? kScaleExp - exp_above(16.0 * max_abs_half(C.s_L, L.V)) : 0;
+  h->tc_gamma = L.r_r > 0 ? kScaleExp - exp_above(128.0 * max_abs_half(C.s_A, L.V)) : 0;
+  int m = h->tc_alpha;
+  if (L.r_c > 0) m = std::min(m, h->tc_beta - h->e_B);
+  if (L.r_r > 0) m = std::min(m, h->tc_gamma - h->e_B);
+  h->tc_mseg = m;
+  // The activation kernel folds the group scales of B at 64-column block ends.
+  h->tc_ok = (L.g_B % kTcBK == 0) && tc_smem_max() <= static_cast<size_t>(smem_optin);
+}
+
 }  // namespace
 }  // namespace archead
 
@@ -286,7 +317,9 @@ extern "C" ARCHEAD_API int archead_pack_load(const archead_desc* desc, const arc
     return ARCHEAD_EUNSUP;
   }
   h->e_B = row_norm_exponent(L, *comps);
+  plan_tc(h, *comps, optin);
   e = decode_set_attributes(L.g_steps, static_cast<size_t>(optin));
+  if (e == cudaSuccess && h->tc_ok) e = tc_set_attributes();
   if (e != cudaSuccess) {
     delete h;
     return set_cuda_error(e);

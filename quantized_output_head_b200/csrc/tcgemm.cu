@@ -1,0 +1,527 @@
+// Tensor-core forward for many tokens (ARCHead paper, §3.2 Eq. 7 with the
+// residual of §3.1 and the correction of Eq. 4-6), on the 5th-generation
+// tensor cores of sm_100a.
+//
+// Work unit: 128 vocabulary rows (8 m-tile blocks) x BN tokens.  One CTA per
+// SM walks its units; per unit the K axis is the concatenation
+//   [ residual: d columns | core: r_c' columns | correction: r_r' columns ]
+// in k-steps of 64 columns.  Roles:
+//   warps 0-7   dequantise: warp w owns m-tile block j = 2(w%4) + w/4 of the
+//               unit (TMEM lanes 16j..16j+15, inside the warp's lane quarter).
+//               It streams its block's packed bytes through a private
+//               cp.async ring, turns each k-step into signed fp16 times the
+//               scale (one rounding: s * 2^alpha * q), and stores the 16 x 64
+//               tile into the stage's TMEM columns (tcgen05.st 16x256b).
+//   warp 8      TMA: the BN x 64 tile of the activation operand X (fp16,
+//               128-byte swizzle) into the stage's shared-memory buffer.
+//   warp 9      MMA: one thread issues tcgen05.mma kind::f16 (M=128, N=BN,
+//               K=16 x 4) with A from TMEM and B from shared memory into one
+//               of two fp32 TMEM accumulators, commits each stage back to the
+//               producers and each finished unit to the epilogue.
+//   warps 10-13 epilogue: tcgen05.ld of the accumulator (warp lane quarter =
+//               32 rows), times 2^-c_t per token, optional logits, target
+//               logit, and per-token (max, sum exp, first argmax) over the
+//               128 rows, written as one partial per (token, 128-row tile).
+// A merge kernel folds the partials into LSE, argmax and cross-entropy.
+// Every mbarrier wait is bounded (kWaitLimitNs); on expiry the CTA raises
+// ARCHEAD_STATUS_WAIT_TIMEOUT, skips its remaining work and frees its TMEM.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "device.cuh"
+#include "tc_params.h"
+#include "tcgen05.cuh"
+
+namespace archead {
+
+namespace {
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccStride = 128;            // TMEM columns per accumulator
+constexpr uint32_t kAcol0 = 2 * kAccStride;     // first column of the A stages
+static_assert(kAcol0 + kTcStages * 32 <= kTmemCols, "TMEM plan");
+static_assert(kTcRing == 8, "ring index mask");
+
+struct TcSmem {
+  uint8_t* bst;        // [kTcStages][bstage_bytes], 1024-byte aligned
+  uint8_t* rings;      // [kTcDeqWarps][kTcRing][kTcSlotBytes]
+  float4* epi;         // [4][kTcMaxBN] per-warp (max, sum, idx) of the current unit
+  uint64_t* full;      // [kTcStages] dequant warps + TMA -> MMA
+  uint64_t* empty;     // [kTcStages] MMA -> dequant warps + TMA
+  uint64_t* accf;      // [2] MMA -> epilogue
+  uint64_t* acce;      // [2] epilogue -> MMA
+  uint32_t* tmem;      // TMEM base address
+  int* abort_flag;
+};
+
+__device__ __forceinline__ TcSmem tc_smem(uint8_t* base, const TcParams& p) {
+  TcSmem s;
+  s.bst = base;
+  s.rings = base + p.ring_off;
+  s.epi = reinterpret_cast<float4*>(base + p.epi_off);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + p.bar_off);
+  s.full = bars;
+  s.empty = bars + kTcStages;
+  s.accf = bars + 2 * kTcStages;
+  s.acce = bars + 2 * kTcStages + 2;
+  s.tmem = reinterpret_cast<uint32_t*>(bars + 2 * kTcStages + 4);
+  s.abort_flag = reinterpret_cast<int*>(s.tmem + 1);
+  return s;
+}
+
+__device__ __forceinline__ bool tc_aborted(const TcSmem& s) {
+  return *reinterpret_cast<volatile int*>(s.abort_flag) != 0;
+}
+
+// Bounded wait of one thread; on expiry raises the timeout status.
+__device__ __forceinline__ bool tc_wait(const TcSmem& s, uint64_t* bar, uint32_t parity, uint32_t* status) {
+  if (tc_aborted(s)) return false;
+  if (mbar_wait(smem_addr(bar), parity)) return true;
+  *reinterpret_cast<volatile int*>(s.abort_flag) = 1;
+  atomicOr(status, static_cast<uint32_t>(ARCHEAD_STATUS_WAIT_TIMEOUT));
+  return false;
+}
+
+// Warp-uniform form.
+__device__ __forceinline__ bool tc_wait_warp(const TcSmem& s, uint64_t* bar, uint32_t parity, uint32_t* status) {
+  bool ok = true;
+  if (tc_aborted(s)) ok = false;
+  else ok = mbar_wait(smem_addr(bar), parity);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && (threadIdx.x & 31) == 0 && !tc_aborted(s)) {
+    *reinterpret_cast<volatile int*>(s.abort_flag) = 1;
+    atomicOr(status, static_cast<uint32_t>(ARCHEAD_STATUS_WAIT_TIMEOUT));
+  }
+  return ok;
+}
+
+// ------------------------------------------------------- dequantising warps
+// Packed bytes of one k-step of one m-tile block -> ring slot:
+//   residual  [0,512) codes, [1024, ...) group scales of the 64 columns
+//   core      [0,512) low nibbles, [512,640) fifth bits, [1024,1056) s_L
+//   correction [0,1024) two 32-column chunks, [1024,1056) s_A
+__device__ __forceinline__ void issue_step(const TcParams& p, uint32_t dst, const uint8_t* blk, int ks, int lane) {
+  if (ks < p.ks_core) {
+    cp_async16(dst + lane * 16, blk + p.off_res + ks * kResChunkBytes + lane * 16);
+    const int gsh = p.g_log2;
+    const int g0 = (ks * kTcBK) >> gsh;
+    const int nbytes = (gsh >= 6 ? 1 : (kTcBK >> gsh)) * kSresGroupBytes;
+    if (lane * 16 < nbytes) cp_async16(dst + 1024 + lane * 16, blk + p.off_sres + g0 * kSresGroupBytes + lane * 16);
+  } else if (ks < p.ks_corr) {
+    const int c = ks - p.ks_core;
+    cp_async16(dst + lane * 16, blk + p.off_Lnib + c * kLNibChunkBytes + lane * 16);
+    if (lane < 8) cp_async16(dst + 512 + lane * 16, blk + p.off_Lhi + c * kLHiChunkBytes + lane * 16);
+    if (lane < 2) cp_async16(dst + 1024 + lane * 16, blk + p.off_sL + lane * 16);
+  } else {
+    const int a = 2 * (ks - p.ks_corr);
+    cp_async16(dst + lane * 16, blk + p.off_A + a * kAChunkBytes + lane * 16);
+    if (a + 1 < p.n_A) cp_async16(dst + 512 + lane * 16, blk + p.off_A + (a + 1) * kAChunkBytes + lane * 16);
+    if (lane < 2) cp_async16(dst + 1024 + lane * 16, blk + p.off_sA + lane * 16);
+  }
+}
+
+// Scale pair (row gr, row gr + 8) of a slot -> two half2 (s, s) times 2^e.
+__device__ __forceinline__ void scale_pair(const uint8_t* at, float mul, uint32_t& s0, uint32_t& s1) {
+  const float2 f = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(at));
+  s0 = pack_half2(f.x * mul, f.x * mul);
+  s1 = pack_half2(f.y * mul, f.y * mul);
+}
+
+// Fragment registers (p order) of one k16 step -> tcgen05.st order, scaled.
+__device__ __forceinline__ void place(const uint32_t (&a)[4], uint32_t s0, uint32_t s1, uint32_t* r) {
+  r[0] = hmul2_bits(a[0], s0);   // lane gr,     column 2cc     (k 2cc, 2cc+1)
+  r[1] = hmul2_bits(a[2], s0);   // lane gr,     column 2cc + 1 (k 2cc+8, 2cc+9)
+  r[2] = hmul2_bits(a[1], s1);   // lane gr + 8, column 2cc
+  r[3] = hmul2_bits(a[3], s1);   // lane gr + 8, column 2cc + 1
+}
+
+__device__ __forceinline__ void dequant_residual(const TcParams& p, const uint8_t* slot, int ks, int lane,
+                                                 uint32_t (&r)[16]) {
+  const int gr = lane >> 2;
+  const uint4 c = *reinterpret_cast<const uint4*>(slot + lane * 16);
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  const int gsh = p.g_log2;
+  uint32_t s0 = 0, s1 = 0;
+#pragma unroll
+  for (int st = 0; st < 4; ++st) {
+    // local group of this k16 step (groups are >= 16 columns, powers of two)
+    const int lg = ((ks * kTcBK + 16 * st) >> gsh) - ((ks * kTcBK) >> gsh);
+    if (st == 0 || gsh < 6) scale_pair(slot + 1024 + lg * kSresGroupBytes + gr * 4, p.sc_res, s0, s1);
+    uint32_t a[4];
+    unpack_int4_signed(w[st], a);
+    place(a, s0, s1, r + 4 * st);
+  }
+}
+
+__device__ __forceinline__ void dequant_core(const TcParams& p, const uint8_t* slot, int lane, uint32_t (&r)[16]) {
+  const int gr = lane >> 2;
+  const uint4 n = *reinterpret_cast<const uint4*>(slot + lane * 16);
+  const uint32_t hb = *reinterpret_cast<const uint32_t*>(slot + 512 + lane * 4);
+  uint32_t s0, s1;
+  scale_pair(slot + 1024 + gr * 4, p.sc_L, s0, s1);
+  uint32_t a[4];
+  unpack_int5_signed<0>(n.x, hb, a);
+  place(a, s0, s1, r + 0);
+  unpack_int5_signed<1>(n.y, hb, a);
+  place(a, s0, s1, r + 4);
+  unpack_int5_signed<2>(n.z, hb, a);
+  place(a, s0, s1, r + 8);
+  unpack_int5_signed<3>(n.w, hb, a);
+  place(a, s0, s1, r + 12);
+}
+
+__device__ __forceinline__ void dequant_corr(const TcParams& p, const uint8_t* slot, bool second, int lane,
+                                             uint32_t (&r)[16]) {
+  const int gr = lane >> 2;
+  uint32_t s0, s1;
+  scale_pair(slot + 1024 + gr * 4, p.sc_A, s0, s1);
+  const uint4 c0 = *reinterpret_cast<const uint4*>(slot + lane * 16);
+  uint32_t a[4];
+  unpack_int8_signed(c0.x, c0.y, a);
+  place(a, s0, s1, r + 0);
+  unpack_int8_signed(c0.z, c0.w, a);
+  place(a, s0, s1, r + 4);
+  if (second) {
+    const uint4 c1 = *reinterpret_cast<const uint4*>(slot + 512 + lane * 16);
+    unpack_int8_signed(c1.x, c1.y, a);
+    place(a, s0, s1, r + 8);
+    unpack_int8_signed(c1.z, c1.w, a);
+    place(a, s0, s1, r + 12);
+  } else {
+#pragma unroll
+    for (int i = 8; i < 16; ++i) r[i] = 0u;
+  }
+}
+
+__device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int w, int lane) {
+  const int j = 2 * (w & 3) + (w >> 2);
+  const uint32_t ring_s = smem_addr(sm.rings) + static_cast<uint32_t>(w) * kTcRing * kTcSlotBytes;
+  const uint8_t* ring = sm.rings + static_cast<size_t>(w) * kTcRing * kTcSlotBytes;
+  const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                   static_cast<int>(gridDim.x);
+  // Prefetch cursor: unit ordinal pi, k-step pks.
+  int pi = 0, pks = 0;
+  auto issue_next = [&](uint32_t slot) {
+    if (pi < n_my) {
+      const int u = static_cast<int>(blockIdx.x) + pi * static_cast<int>(gridDim.x);
+      const int mt16 = (u / p.n_nt) * 8 + j;
+      if (mt16 < p.n_mtiles)
+        issue_step(p, ring_s + slot * kTcSlotBytes, p.mtiles + static_cast<size_t>(mt16) * p.mblk_bytes, pks, lane);
+      if (++pks == p.n_ks) {
+        pks = 0;
+        ++pi;
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll 1
+  for (uint32_t k = 0; k < kTcRing; ++k) issue_next(k);
+
+  const uint32_t tmem_row = tmem_base + (static_cast<uint32_t>(16 * j) << 16) + kAcol0;
+  int s = 0;
+  uint32_t ph = 0;
+  uint32_t it = 0;
+  for (int ui = 0; ui < n_my; ++ui) {
+    const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
+    const bool valid = (u / p.n_nt) * 8 + j < p.n_mtiles;
+    for (int ks = 0; ks < p.n_ks; ++ks, ++it) {
+      if (!tc_wait_warp(sm, &sm.empty[s], ph ^ 1u, p.status)) {
+        cp_async_wait_all();
+        return;
+      }
+      tc_fence_after();
+      const uint32_t rs = it & (kTcRing - 1);
+      const uint8_t* slot = ring + rs * kTcSlotBytes;
+      cp_async_wait<kTcRing - 1>();
+      __syncwarp();
+      uint32_t r[16];
+      if (!valid) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = 0u;
+      } else if (ks < p.ks_core) {
+        dequant_residual(p, slot, ks, lane, r);
+      } else if (ks < p.ks_corr) {
+        dequant_core(p, slot, lane, r);
+      } else {
+        dequant_corr(p, slot, 2 * (ks - p.ks_corr) + 1 < p.n_A, lane, r);
+      }
+      __syncwarp();   // every lane is done reading the slot
+      issue_next(rs);
+      tmem_st_16x256b_x4(tmem_row + static_cast<uint32_t>(s) * 32u, r);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&sm.full[s]));
+      if (++s == kTcStages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+  }
+  cp_async_wait_all();
+}
+
+// ---------------------------------------------------------------- TMA warp
+__device__ void tma_warp(const TcParams& p, const TcSmem& sm, const CUtensorMap* xmap, int lane) {
+  if (lane != 0) return;
+  grid_dependency_wait();   // X and c_t come from the activation kernel
+  const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                   static_cast<int>(gridDim.x);
+  const uint32_t bst = smem_addr(sm.bst);
+  int s = 0;
+  uint32_t ph = 0;
+  for (int ui = 0; ui < n_my; ++ui) {
+    const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
+    const int y = (u % p.n_nt) * p.BN;
+    for (int ks = 0; ks < p.n_ks; ++ks) {
+      if (!tc_wait(sm, &sm.empty[s], ph ^ 1u, p.status)) return;
+      const uint32_t bar = smem_addr(&sm.full[s]);
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(p.BN) * 128u);
+      tma_load_2d(bst + static_cast<uint32_t>(s) * p.bstage_bytes, xmap, ks * kTcBK, y, bar);
+      if (++s == kTcStages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- MMA warp
+__device__ void mma_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int lane) {
+  if (lane != 0) return;
+  const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                   static_cast<int>(gridDim.x);
+  const uint32_t idesc = tc_idesc_f16(kTcBM, p.BN);
+  const uint32_t bst = smem_addr(sm.bst);
+  int s = 0;
+  uint32_t ph = 0;
+  for (int ui = 0; ui < n_my; ++ui) {
+    const uint32_t a = static_cast<uint32_t>(ui) & 1u;
+    if (!tc_wait(sm, &sm.acce[a], ((static_cast<uint32_t>(ui) >> 1) & 1u) ^ 1u, p.status)) return;
+    tc_fence_after();
+    const uint32_t d_tmem = tmem_base + a * kAccStride;
+    for (int ks = 0; ks < p.n_ks; ++ks) {
+      if (!tc_wait(sm, &sm.full[s], ph, p.status)) return;
+      tc_fence_after();
+      const uint64_t bdesc = smem_desc_k128(bst + static_cast<uint32_t>(s) * p.bstage_bytes);
+      const uint32_t a_tmem = tmem_base + kAcol0 + static_cast<uint32_t>(s) * 32u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        tc_mma_ts(d_tmem, a_tmem + 8u * i, bdesc + 2u * i, idesc, (ks | i) != 0 ? 1u : 0u);
+      tc_commit(smem_addr(&sm.empty[s]));
+      if (++s == kTcStages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    tc_commit(smem_addr(&sm.accf[a]));
+  }
+}
+
+// ----------------------------------------------------------- epilogue warps
+__device__ void epilogue_warps(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int ew, int lane) {
+  grid_dependency_wait();   // c_t, and the previous call's readers of the outputs
+  const int q = (kTcDeqWarps + 2 + ew) & 3;   // TMEM lane quarter of this warp
+  const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                   static_cast<int>(gridDim.x);
+  bool ok = true;
+  for (int ui = 0; ui < n_my; ++ui) {
+    const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
+    const int mt = u / p.n_nt, tb = (u % p.n_nt) * p.BN;
+    const uint32_t a = static_cast<uint32_t>(ui) & 1u;
+    if (ok) ok = tc_wait_warp(sm, &sm.accf[a], (static_cast<uint32_t>(ui) >> 1) & 1u, p.status);
+    if (ok) {
+      tc_fence_after();
+      const int v = mt * kTcBM + 32 * q + lane;
+      const bool v_ok = v < p.V;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * kAccStride;
+      const int ncol = min(p.BN, p.T - tb);
+      for (int c0 = 0; c0 < ncol; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c0), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int col = c0 + jj;
+          if (col >= ncol) break;
+          const int t = tb + col;
+          const float inv = ldexpf(1.f, -__ldg(p.cexp + t));
+          const float y = v_ok ? __uint_as_float(r[jj]) * inv : -INFINITY;
+          if (v_ok) {
+            if (p.logits != nullptr) p.logits[static_cast<size_t>(t) * p.V + v] = y;
+            if (p.targets != nullptr && __ldg(p.targets + t) == v) p.tgt[t] = y;
+          }
+          float m = y;
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          float e = v_ok ? __expf(y - m) : 0.f;
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+          const uint32_t ball = __ballot_sync(0xffffffffu, v_ok && y == m);
+          if (lane == 0) {
+            const int idx = ball != 0u ? mt * kTcBM + 32 * q + __ffs(ball) - 1 : 0x7fffffff;
+            sm.epi[q * kTcMaxBN + col] = make_float4(m, e, __int_as_float(idx), 0.f);
+          }
+        }
+      }
+      tc_fence_before();
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sm.acce[a]));
+    // The four warps' states of each token -> one partial per (token, tile).
+    named_bar_sync(1, 128);
+    const int col = ew * 32 + lane;
+    if (ok && col < p.BN && tb + col < p.T) {
+      LseState st = lse_init();
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float4 e = sm.epi[w * kTcMaxBN + col];
+        st = lse_merge(st, LseState{e.x, e.y, __float_as_int(e.z)});
+      }
+      p.partials[static_cast<size_t>(tb + col) * p.n_mt128 + mt] = make_float4(st.m, st.s, __int_as_float(st.idx), 0.f);
+    }
+    named_bar_sync(1, 128);
+  }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kTcWarps * 32, 1)
+    tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap xmap) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const TcSmem sm = tc_smem(base, p);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(smem_addr(&sm.full[s]), kTcDeqWarps + 1);
+      mbar_init(smem_addr(&sm.empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_addr(&sm.accf[a]), 1);
+      mbar_init(smem_addr(&sm.acce[a]), 4);
+    }
+    *sm.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kTcDeqWarps + 1) {
+    tmem_alloc(smem_addr(sm.tmem), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *sm.tmem;
+
+  if (warp < kTcDeqWarps) dequant_warp(p, sm, tmem_base, warp, lane);
+  else if (warp == kTcDeqWarps) tma_warp(p, sm, &xmap, lane);
+  else if (warp == kTcDeqWarps + 1) mma_warp(p, sm, tmem_base, lane);
+  else epilogue_warps(p, sm, tmem_base, warp - kTcDeqWarps - 2, lane);
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kTcDeqWarps + 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Per-token fold of the partials: LSE, first argmax, cross-entropy.
+__global__ void __launch_bounds__(256) tc_merge_kernel(const float4* partials, int n_mt128, int T,
+                                                       const int32_t* targets, const float* tgt, int V, float* lse,
+                                                       int32_t* argmax, float* ce) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  grid_dependency_wait();
+  if (t >= T) return;
+  LseState a = lse_init();
+  for (int m = lane; m < n_mt128; m += 32) {
+    const float4 q = partials[static_cast<size_t>(t) * n_mt128 + m];
+    a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) a = lse_merge(a, lse_shfl_xor(a, o));
+  if (lane == 0) {
+    const float l = a.m + logf(a.s);
+    if (lse != nullptr) lse[t] = l;
+    if (argmax != nullptr) argmax[t] = a.idx;
+    if (ce != nullptr) {
+      const int tg = targets[t];
+      ce[t] = (tg >= 0 && tg < V) ? l - tgt[t] : __int_as_float(0x7fc00000);
+    }
+  }
+}
+
+// ------------------------------------------------------------------- host
+void tc_smem_plan(TcParams& p) {
+  p.bstage_bytes = static_cast<uint32_t>(p.BN) * 128u;   // multiple of 2048 (BN % 16 == 0)
+  p.ring_off = kTcStages * p.bstage_bytes;
+  p.epi_off = p.ring_off + kTcDeqWarps * kTcRing * kTcSlotBytes;
+  p.bar_off = p.epi_off + 4 * kTcMaxBN * 16;
+}
+
+size_t tc_smem_bytes(const TcParams& p) { return static_cast<size_t>(p.bar_off) + 256 + 1024; }
+
+size_t tc_smem_max() {
+  TcParams p{};
+  p.BN = kTcMaxBN;
+  tc_smem_plan(p);
+  return tc_smem_bytes(p);
+}
+
+cudaError_t tc_set_attributes() {
+  return cudaFuncSetAttribute(reinterpret_cast<const void*>(&tc_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(tc_smem_max()));
+}
+
+namespace {
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiled g_encode = nullptr;
+std::once_flag g_encode_once;
+}  // namespace
+
+// Tensor map of X [T, Kc] fp16: boxes of 64 columns x BN rows, 128-byte swizzle.
+cudaError_t tc_encode_xmap(CUtensorMap* map, const uint16_t* xop, int T, int Kc, int BN) {
+  std::call_once(g_encode_once, []() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiled>(fn);
+  });
+  if (g_encode == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Kc), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Kc) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcBK), static_cast<cuuint32_t>(BN)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(xop), dims, strides,
+                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_tc(const TcParams& p, const CUtensorMap& map, int grid, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kTcWarps * 32);
+  cfg.dynamicSmemBytes = tc_smem_bytes(p);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[] = {const_cast<TcParams*>(&p), const_cast<CUtensorMap*>(&map)};
+  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&tc_kernel), args);
+}
+
+cudaError_t launch_tc_merge(const float4* partials, int n_mt128, int T, const int32_t* targets, const float* tgt,
+                            int V, float* lse, int32_t* argmax, float* ce, cudaStream_t stream) {
+  tc_merge_kernel<<<(T + 7) / 8, 256, 0, stream>>>(partials, n_mt128, T, targets, tgt, V, lse, argmax, ce);
+  return cudaGetLastError();
+}
+
+}  // namespace archead

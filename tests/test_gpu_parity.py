@@ -190,6 +190,23 @@ def test_small_shapes(qoh, V, d, r_c, r_r, g, g_B, T):
     assert np.array_equal(am.cpu().numpy(), am2.cpu().numpy())
 
 
+# Calls of >= 16 tokens take the tensor-core kernel when g_B is a multiple of 64.
+SMALL_TC = [
+    # V,    d,   r_c, r_r, g,   g_B, T
+    (1000, 320, 32, 8, 64, 64, 16),       # ragged vocabulary, one 32-column correction chunk
+    (2000, 256, 0, 0, 16, 64, 33),        # residual only, g = 16, ragged token tile
+    (1500, 512, 64, 0, 32, 64, 130),      # no correction, g = 32, two token tiles
+    (4099, 512, 128, 64, 256, 128, 40),   # g = 256, last 128-row tile nearly empty
+    (300, 128, 64, 32, 128, 128, 200),    # three 128-row tiles, the last partial
+    (1003, 320, 100, 40, 16, 10, 20),     # g_B = 10: 16+ tokens through the decode kernel
+]
+
+
+@pytest.mark.parametrize("V,d,r_c,r_r,g,g_B,T", SMALL_TC)
+def test_small_shapes_many_tokens(qoh, V, d, r_c, r_r, g, g_B, T):
+    test_small_shapes(qoh, V, d, r_c, r_r, g, g_B, T)
+
+
 def test_zero_residual_and_correction_is_core_product(qoh):
     shape = (512, 256, 64, 32, 64, 64)
     comps = gen.random_components(gen.HeadShape(*shape), seed=99)
