@@ -64,11 +64,13 @@ def parse_args():
 
 
 def peaks():
+    """HBM GB/s, dense bf16 TFLOP/s (burst, sustained) and where they come from."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+        burst = float(d["bf16_tflops"])
+        return float(d["hbm_gbs"]), burst, float(d.get("bf16_tflops_sustained", burst)), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def workload(cfg, T):
@@ -99,28 +101,43 @@ def vocab_pass_bytes_per_launch(shape, nt, op, Kz):
             + 4 * nt * (op["argmax"] + op["lse"] + op["ce"]))
 
 
-DECODE_SOURCES = ("decode.cu", "device.cuh", "params.h", "layout.h")
+def tc_pass_bytes_flops(shape, T, op):
+    """Algorithmic bytes and flops of one tensor-core launch: the per-row packed
+    payload read once, the fp16 activation operand [h | z] (T x Kc), the
+    per-(token, 128-row tile) partials and target logits written, logits if asked."""
+    V, d, r_c, r_r = shape[0], shape[1], shape[2], shape[3]
+    kc = d + -(-r_c // 64) * 64 + -(-r_r // 64) * 64
+    n_mt128 = -(-V // 128)
+    b = (V * row_bytes(shape) + 2 * T * kc + 16 * T * n_mt128 + 4 * T + (4 * T * V if op["logits"] else 0))
+    return b, 2 * T * V * (d + r_c + r_r)
 
 
-def source_hash():
+KERNEL_SOURCES = {
+    "decode": ("decode.cu", "device.cuh", "params.h", "layout.h"),
+    "tensor_core": ("tcgemm.cu", "tcgen05.cuh", "tc_params.h", "device.cuh", "layout.h"),
+}
+PROFILE_STEM = {"decode": "decode_kernel", "tensor_core": "tc_kernel"}
+
+
+def source_hash(kind):
     """Hash of the sources the vocabulary-pass kernel is compiled from."""
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "quantized_output_head_b200", "csrc")
-    for f in DECODE_SOURCES:
+    for f in KERNEL_SOURCES[kind]:
         h.update(open(os.path.join(cs, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(cfg, T):
+def recorded_traffic(kind, cfg, T):
     """dram bytes per vocabulary-pass launch from the committed ncu summary, if
     it was taken on the current kernel sources; else None."""
-    p = os.path.join(ROOT, "profiles", f"decode_kernel_cfg{cfg}_T{T}.md")
+    p = os.path.join(ROOT, "profiles", f"{PROFILE_STEM[kind]}_cfg{cfg}_T{T}.md")
     if not os.path.exists(p):
         return None
     txt = open(p).read()
     m = re.search(r"traffic_bytes_per_launch:\s*(\d+)", txt)
     s = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
-    if not m or not s or s.group(1) != source_hash():
+    if not m or not s or s.group(1) != source_hash(kind):
         return None
     return int(m.group(1))
 
@@ -307,7 +324,8 @@ def main():
 
     # Dominant kernel (the vocabulary pass): CUDA events around it, recorded on
     # the call's stream by the library, over a second timed loop.
-    n_launch = math.ceil(T / 8)
+    kind = head.forward_kernel(T)
+    n_launch = math.ceil(T / 8) if kind == "decode" else 1
     from cuda.bindings import runtime as cudart
     _, kb = cudart.cudaEventCreate()
     _, ka = cudart.cudaEventCreate()
@@ -323,13 +341,25 @@ def main():
     cudart.cudaEventDestroy(kb)
     cudart.cudaEventDestroy(ka)
     kernel_ms = tot / k_steps / n_launch
-    hbm, bf16, peak_src = peaks()
-    Kz = -(-shape.r_c // 64) * 64 + -(-shape.r_r // 32) * 32
-    nt = min(T, 8)
-    kbytes = vocab_pass_bytes_per_launch(sh, nt, op, Kz)
-    achieved = kbytes / (kernel_ms / 1e3) / 1e9
-    traffic = recorded_traffic(cfg, T)
+    hbm, bf16, bf16_sust, peak_src = peaks()
+    if kind == "decode":
+        Kz = -(-shape.r_c // 64) * 64 + -(-shape.r_r // 32) * 32
+        kbytes = vocab_pass_bytes_per_launch(sh, min(T, 8), op, Kz)
+        kflops = None
+        bound = "hbm"
+    else:
+        kbytes, kflops = tc_pass_bytes_flops(sh, T, op)
+        # The roofline that binds: HBM streaming of the packed head, or the
+        # tensor cores (fp16 MMA runs at the bf16 rate; sustained peak, the
+        # kernel is timed inside back-to-back calls).
+        bound = "tensor" if kflops / (bf16_sust * 1e12) > kbytes / (hbm * 1e9) else "hbm"
+    if bound == "hbm":
+        achieved, peak, unit = kbytes / (kernel_ms / 1e3) / 1e9, hbm, "GB/s"
+    else:
+        achieved, peak, unit = kflops / (kernel_ms / 1e3) / 1e12, bf16_sust, "TFLOP/s"
+    traffic = recorded_traffic(kind, cfg, T)
     status = head.status(ws)
+    launches_per_step = (1 + n_launch) if kind == "decode" else 3
 
     out = None
     if rank == 0:
@@ -357,18 +387,22 @@ def main():
         out = dict(
             metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
             ms_per_step=ms_per_step, us_per_call=ms_per_step * 1e3, higher_is_better=True, scaling="weak",
-            vs_baseline=None, dtype="bf16 MMA on exact int4/int5/int8 codes, fp32 accumulate",
+            vs_baseline=None, dtype="f16",
+            dtype_detail=("f16 MMA (mma.sync) on exact int4/int5/int8 codes, fp32 accumulate, scales in fp32"
+                          if kind == "decode" else
+                          "f16 MMA (tcgen05) on fp16(scale*code) weights and fp16 [h|z], fp32 accumulate in TMEM"),
             data="synthetic (seeded, shapes of the pages' heads)",
             config=dict(workload=wl.name, V=shape.V, d=shape.d, r_c=shape.r_c, r_r=shape.r_r, g=shape.g,
                         g_B=shape.g_B, T=T, outputs=[k for k, v in op.items() if v],
                         parallelism=f"replicas x{world}", l2="inputs larger than L2 (packed head 382 MB)"),
-            roofline=dict(bound="hbm", achieved=achieved, peak=hbm, unit="GB/s", frac=achieved / hbm,
-                          traffic=traffic, kernel="archead::decode_kernel", kernel_us=kernel_ms * 1e3,
-                          algorithmic_bytes_per_launch=kbytes, peak_source=peak_src),
+            roofline=dict(bound=bound, achieved=achieved, peak=peak, unit=unit, frac=achieved / peak,
+                          traffic=traffic, kernel=f"archead::{PROFILE_STEM[kind]}", kernel_us=kernel_ms * 1e3,
+                          algorithmic_bytes_per_launch=kbytes, algorithmic_flops_per_launch=kflops,
+                          peak_source=peak_src + (" (sustained bf16)" if bound == "tensor" else "")),
             call=dict(algorithmic_bytes=ab, algorithmic_flops=af, gbs=ab / (ms_per_step / 1e3) / 1e9,
                       hbm_frac=ab / (ms_per_step / 1e3) / 1e9 / hbm),
             cpu_baseline=cpu, e2e=e2e, clocks=clk.summary(),
-            gpu_launches=args.steps * (1 + n_launch), device_status=status,
+            gpu_launches=args.steps * launches_per_step, device_status=status,
         )
     if world > 1:
         dist.barrier()

@@ -117,9 +117,22 @@ ARCHEAD_API int archead_pack_load(const archead_desc* desc, const archead_host_c
 ARCHEAD_API int archead_pack_image(const archead_desc* desc, const archead_host_components* comps,
                                    void* host_image, size_t image_bytes);
 
+/* Which kernel a forward call with T tokens runs its vocabulary pass on:
+ *   ARCHEAD_KERNEL_DECODE        the streaming decode kernel (up to 8 tokens
+ *                                per launch, mma.sync fragments in registers);
+ *   ARCHEAD_KERNEL_TENSOR_CORE   the tcgen05 kernel (T >= 16 and g_B a
+ *                                multiple of 64): weights dequantised into
+ *                                tensor memory, 128 rows x up to 128 tokens
+ *                                per unit.
+ * Both compute Eq. 7 of §3.2; -1 if handle is null or T <= 0.  (A library
+ * query with no counterpart in the paper.) */
+enum { ARCHEAD_KERNEL_DECODE = 0, ARCHEAD_KERNEL_TENSOR_CORE = 1 };
+ARCHEAD_API int archead_forward_kernel(const archead_handle* handle, int32_t T);
+
 /* Workspace bytes one forward call with T tokens needs (256-byte aligned
  * scratch, caller-owned; reused across calls on one stream).  Holds the
- * low-rank prologue output z, per-block log-sum-exp partials, a completion
+ * low-rank prologue output z (decode kernel) or the fp16 activation operand
+ * [h | z] (tensor-core kernel), per-block log-sum-exp partials, a completion
  * counter and the status word.  Zero-fill a workspace once before its first
  * use (the status word is sticky); afterwards the calls keep it consistent.
  * Calls that share a workspace must be ordered (same stream).  0 if handle is
@@ -187,7 +200,8 @@ ARCHEAD_API int archead_workspace_status(void* workspace, int clear, archead_str
  * later forward call on this handle records `before` on its stream just before
  * the first vocabulary-pass launch and `after` just after the last one, so
  * cudaEventElapsedTime(before, after) is the device time of the vocabulary
- * pass alone (the low-rank prologue excluded).  NULL, NULL switches it off. */
+ * pass alone (the low-rank prologue or activation kernel and the final
+ * per-token fold excluded).  NULL, NULL switches it off. */
 ARCHEAD_API int archead_set_profile_events(archead_handle* handle, void* before, void* after);
 
 /* Free a handle (host memory only; the arena stays with the caller). */

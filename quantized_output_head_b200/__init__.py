@@ -33,6 +33,7 @@ EXPORTED = (
     "archead_logits", "archead_logits_lse_argmax", "archead_host_workspace_bytes", "archead_lse_argmax_host",
     "archead_workspace_status", "archead_set_profile_events", "archead_free", "archead_last_cuda_error",
     "archead_status_string", "archead_static_workspace_capacity", "archead_logits_lse_argmax_static",
+    "archead_forward_kernel",
 )
 
 
@@ -61,6 +62,7 @@ _sig = {
     "archead_set_profile_events": (ctypes.c_int, [_vp, _vp, _vp]),
     "archead_static_workspace_capacity": (_sz, []),
     "archead_logits_lse_argmax_static": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "archead_forward_kernel": (ctypes.c_int, [_vp, _i32]),
     "archead_free": (None, [_vp]),
     "archead_last_cuda_error": (ctypes.c_int, []),
     "archead_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -153,7 +155,7 @@ class PackedHead:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h is not None and h.value:
+        if h is not None and h.value and _lib is not None:   # _lib is gone at interpreter exit
             _lib.archead_free(h)
             self.handle = None
 
@@ -230,6 +232,13 @@ class PackedHead:
                                             ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
                "archead_lse_argmax_host")
         return lse, am, ce
+
+    def forward_kernel(self, T: int) -> str:
+        """'decode' or 'tensor_core': the kernel a call with T tokens runs on."""
+        k = _lib.archead_forward_kernel(self.handle, int(T))
+        if k < 0:
+            raise ArcheadError(ARCHEAD_EINVAL, "archead_forward_kernel")
+        return "tensor_core" if k == 1 else "decode"
 
     def set_profile_events(self, before, after) -> None:
         """Record `before` / `after` (cudaEvent_t handles as ints, or objects with a

@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(256) act_prep_kernel(const ActParams p) {
   if (blockIdx.y == gridDim.y - 1) {
     // h segment: X[t, j] = h[t, j]·2^(c_t - alpha), c_t = kScaleExp - E_t + mseg.
     if (threadIdx.x < 16 && t0 + static_cast<int>(threadIdx.x) < p.T)
-      p.cexp[t0 + threadIdx.x] = kScaleExp - s_E[threadIdx.x] + p.mseg;
+      p.cinv[t0 + threadIdx.x] = ldexpf(1.f, s_E[threadIdx.x] - kScaleExp - p.mseg);
     const int nb16 = p.d / 16;
     for (int item = threadIdx.x; item < 16 * nb16; item += blockDim.x) {
       const int tl = item / nb16, b = item - tl * nb16, t = t0 + tl;

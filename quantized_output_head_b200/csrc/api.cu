@@ -32,7 +32,7 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
   const Layout& L = h->L;
   const int Kc = tc_kc(L);
   uint32_t* status = reinterpret_cast<uint32_t*>(wb + w.status);
-  int32_t* cexp = reinterpret_cast<int32_t*>(wb + w.cexp);
+  float* cinv = reinterpret_cast<float*>(wb + w.cinv);
   uint16_t* xop = reinterpret_cast<uint16_t*>(wb + w.xop);
   float4* partials = reinterpret_cast<float4*>(wb + w.tpartials);
   float* tgt = reinterpret_cast<float*>(wb + w.tgt);
@@ -46,7 +46,7 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
   ap.targets = targets;
   ap.status = status;
   ap.xop = xop;
-  ap.cexp = cexp;
+  ap.cinv = cinv;
   ap.T = T;
   ap.d = L.d;
   ap.rcp = L.rcp;
@@ -64,7 +64,7 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
   TcParams tp{};
   tp.mtiles = h->arena;
   tp.targets = targets;
-  tp.cexp = cexp;
+  tp.cinv = cinv;
   tp.logits = logits;
   tp.partials = partials;
   tp.tgt = tgt;
@@ -238,6 +238,11 @@ int set_cuda_error(cudaError_t e) {
 }  // namespace archead
 
 using namespace archead;
+
+extern "C" ARCHEAD_API int archead_forward_kernel(const archead_handle* handle, int32_t T) {
+  if (handle == nullptr || T <= 0 || T > kMaxTokens) return -1;
+  return use_tc(*handle, T) ? ARCHEAD_KERNEL_TENSOR_CORE : ARCHEAD_KERNEL_DECODE;
+}
 
 extern "C" ARCHEAD_API size_t archead_workspace_bytes(const archead_handle* handle, int32_t T) {
   if (handle == nullptr || T <= 0 || T > kMaxTokens) return 0;

@@ -39,7 +39,7 @@ inline int tc_n_mt128(const Layout& L) { return (L.n_mtiles + 7) / 8; }
 struct WsLayout {
   size_t counter, status;
   size_t escale, zhi, zlo, partials;   // decode path
-  size_t cexp, xop, tpartials;         // tensor-core path
+  size_t cinv, xop, tpartials;         // tensor-core path
   size_t tgt, total;
   // host-buffer form only
   size_t h_hidden, h_targets, h_lse, h_argmax, h_ce, host_total;
@@ -53,7 +53,7 @@ inline WsLayout ws_layout(const archead_handle& h, int T) {
   w.status = 4;
   o = 256;
   if (use_tc(h, T)) {
-    w.cexp = o;      o += round_up(t * 4, 256);
+    w.cinv = o;      o += round_up(t * 4, 256);
     w.xop = o;       o += round_up(t * tc_kc(h.L) * 2, 256);
     w.tpartials = o; o += round_up(t * tc_n_mt128(h.L) * 16, 256);
   } else {

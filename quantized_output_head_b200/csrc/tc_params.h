@@ -16,16 +16,16 @@ constexpr int kTcBM = 128;            // vocabulary rows per unit (8 m-tile bloc
 constexpr int kTcBK = 64;             // K columns per k-step (one 128-byte row of fp16)
 constexpr int kTcMaxBN = 128;         // tokens per unit
 constexpr int kTcStages = 6;          // k-steps in flight between the producers and the MMA
-constexpr int kTcRing = 8;            // packed k-steps prefetched per dequantising warp
+constexpr int kTcRing = 5;            // ring slots per dequantising warp (kTcRing - 1 k-steps prefetched)
 constexpr int kTcSlotBytes = 1152;    // one packed k-step of one m-tile block (codes + scales)
-constexpr int kTcDeqWarps = 8;        // one per m-tile block of a unit
-constexpr int kTcWarps = 14;          // 8 dequantising, 1 TMA, 1 MMA, 4 epilogue
+constexpr int kTcDeqWarps = 16;       // two per m-tile block of a unit (even / odd k-steps)
+constexpr int kTcWarps = 22;          // 16 dequantising, 1 TMA, 1 MMA, 4 epilogue
 constexpr int kTcMinTokens = 16;      // calls with fewer tokens take the decode kernel
 
 struct TcParams {
   const uint8_t* mtiles;      // arena: m-tile blocks
   const int32_t* targets;     // [T] or null
-  const int32_t* cexp;        // [T] c_t
+  const float* cinv;          // [T] 2^-c_t
   float* logits;              // [T, V] or null
   float4* partials;           // [T, n_mt128]: (max, sum, argmax bits, unused) per 128-row tile
   float* tgt;                 // [T] target logits
@@ -47,7 +47,7 @@ struct ActParams {
   const int32_t* targets;     // [T] or null
   uint32_t* status;
   uint16_t* xop;              // [T, Kc] fp16 activation operand
-  int32_t* cexp;              // [T]
+  float* cinv;                // [T] 2^-c_t
   int32_t T, d, rcp, Kz, Kc, g_B, V;
   int32_t alpha, beta, gamma, mseg;
 };

@@ -6,19 +6,20 @@
 // SM walks its units; per unit the K axis is the concatenation
 //   [ residual: d columns | core: r_c' columns | correction: r_r' columns ]
 // in k-steps of 64 columns.  Roles:
-//   warps 0-7   dequantise: warp w owns m-tile block j = 2(w%4) + w/4 of the
-//               unit (TMEM lanes 16j..16j+15, inside the warp's lane quarter).
-//               It streams its block's packed bytes through a private
-//               cp.async ring, turns each k-step into signed fp16 times the
-//               scale (one rounding: s * 2^alpha * q), and stores the 16 x 64
-//               tile into the stage's TMEM columns (tcgen05.st 16x256b).
-//   warp 8      TMA: the BN x 64 tile of the activation operand X (fp16,
+//   warps 0-15  dequantise: warp w owns m-tile block j = 2(w%4) + (w/4)%2 of
+//               the unit (TMEM lanes 16j..16j+15, inside the warp's lane
+//               quarter) on the k-steps of parity w/8.  It streams its
+//               block's packed bytes through a private cp.async ring, turns
+//               each k-step into signed fp16 times the scale (one rounding:
+//               s * 2^alpha * q), and stores the 16 x 64 tile into the
+//               stage's TMEM columns (tcgen05.st 16x256b).
+//   warp 16     TMA: the BN x 64 tile of the activation operand X (fp16,
 //               128-byte swizzle) into the stage's shared-memory buffer.
-//   warp 9      MMA: one thread issues tcgen05.mma kind::f16 (M=128, N=BN,
+//   warp 17     MMA: one thread issues tcgen05.mma kind::f16 (M=128, N=BN,
 //               K=16 x 4) with A from TMEM and B from shared memory into one
 //               of two fp32 TMEM accumulators, commits each stage back to the
 //               producers and each finished unit to the epilogue.
-//   warps 10-13 epilogue: tcgen05.ld of the accumulator (warp lane quarter =
+//   warps 18-21 epilogue: tcgen05.ld of the accumulator (warp lane quarter =
 //               32 rows), times 2^-c_t per token, optional logits, target
 //               logit, and per-token (max, sum exp, first argmax) over the
 //               128 rows, written as one partial per (token, 128-row tile).
@@ -42,12 +43,12 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 128;            // TMEM columns per accumulator
 constexpr uint32_t kAcol0 = 2 * kAccStride;     // first column of the A stages
 static_assert(kAcol0 + kTcStages * 32 <= kTmemCols, "TMEM plan");
-static_assert(kTcRing == 8, "ring index mask");
 
 struct TcSmem {
   uint8_t* bst;        // [kTcStages][bstage_bytes], 1024-byte aligned
   uint8_t* rings;      // [kTcDeqWarps][kTcRing][kTcSlotBytes]
   float4* epi;         // [4][kTcMaxBN] per-warp (max, sum, idx) of the current unit
+  float* etile;        // [4][32 x 33] per-warp transpose tiles of the epilogue
   uint64_t* full;      // [kTcStages] dequant warps + TMA -> MMA
   uint64_t* empty;     // [kTcStages] MMA -> dequant warps + TMA
   uint64_t* accf;      // [2] MMA -> epilogue
@@ -61,6 +62,7 @@ __device__ __forceinline__ TcSmem tc_smem(uint8_t* base, const TcParams& p) {
   s.bst = base;
   s.rings = base + p.ring_off;
   s.epi = reinterpret_cast<float4*>(base + p.epi_off);
+  s.etile = reinterpret_cast<float*>(base + p.epi_off + 4 * kTcMaxBN * 16);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + p.bar_off);
   s.full = bars;
   s.empty = bars + kTcStages;
@@ -195,69 +197,98 @@ __device__ __forceinline__ void dequant_corr(const TcParams& p, const uint8_t* s
   }
 }
 
+// Block pointer of m-tile block j in this CTA's unit ordinal ui, or null when
+// the unit is past the end or the block past the vocabulary.
+__device__ __forceinline__ const uint8_t* unit_block(const TcParams& p, int ui, int n_my, int j) {
+  if (ui >= n_my) return nullptr;
+  const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
+  const int mt16 = (u / p.n_nt) * 8 + j;
+  return mt16 < p.n_mtiles ? p.mtiles + static_cast<size_t>(mt16) * p.mblk_bytes : nullptr;
+}
+
+// Cursor over the global k-steps it = par, par + 2, ... of this CTA's units.
+struct StepCursor {
+  int ui, ks;
+  const uint8_t* blk;
+};
+__device__ __forceinline__ void cursor_normalize(StepCursor& c, const TcParams& p, int n_my, int j) {
+  while (c.ks >= p.n_ks) {
+    c.ks -= p.n_ks;
+    ++c.ui;
+    c.blk = unit_block(p, c.ui, n_my, j);
+  }
+}
+__device__ __forceinline__ void cursor_advance(StepCursor& c, const TcParams& p, int n_my, int j) {
+  c.ks += 2;
+  cursor_normalize(c, p, n_my, j);
+}
+
+// Warp w dequantises m-tile block j = 2(w%4) + (w/4)%2 of every unit (TMEM
+// lanes 16j..16j+15 lie in the warp's lane quarter w%4) on the global k-steps
+// of parity w/8; a stage index has a fixed parity (kTcStages is even), so each
+// stage is filled by the same eight warps.
 __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int w, int lane) {
-  const int j = 2 * (w & 3) + (w >> 2);
+  static_assert(kTcStages % 2 == 0, "stage parity");
+  const int j = 2 * (w & 3) + ((w >> 2) & 1);
+  const int par = w >> 3;
   const uint32_t ring_s = smem_addr(sm.rings) + static_cast<uint32_t>(w) * kTcRing * kTcSlotBytes;
   const uint8_t* ring = sm.rings + static_cast<size_t>(w) * kTcRing * kTcSlotBytes;
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
-  // Prefetch cursor: unit ordinal pi, k-step pks.
-  int pi = 0, pks = 0;
-  auto issue_next = [&](uint32_t slot) {
-    if (pi < n_my) {
-      const int u = static_cast<int>(blockIdx.x) + pi * static_cast<int>(gridDim.x);
-      const int mt16 = (u / p.n_nt) * 8 + j;
-      if (mt16 < p.n_mtiles)
-        issue_step(p, ring_s + slot * kTcSlotBytes, p.mtiles + static_cast<size_t>(mt16) * p.mblk_bytes, pks, lane);
-      if (++pks == p.n_ks) {
-        pks = 0;
-        ++pi;
-      }
-    }
+  const long total = static_cast<long>(n_my) * p.n_ks;   // global k-steps of this CTA
+
+  // Prefetch kTcRing - 1 of this warp's steps ahead.
+  StepCursor pc{0, par, unit_block(p, 0, n_my, j)};
+  long pit = par;
+  cursor_normalize(pc, p, n_my, j);
+  uint32_t pslot = 0;
+  auto issue_next = [&]() {
+    if (pit < total && pc.blk != nullptr) issue_step(p, ring_s + pslot * kTcSlotBytes, pc.blk, pc.ks, lane);
     cp_async_commit();
+    if (pit < total) {
+      pit += 2;
+      cursor_advance(pc, p, n_my, j);
+    }
+    if (++pslot == kTcRing) pslot = 0;
   };
 #pragma unroll 1
-  for (uint32_t k = 0; k < kTcRing; ++k) issue_next(k);
+  for (int k = 0; k < kTcRing - 1; ++k) issue_next();
 
   const uint32_t tmem_row = tmem_base + (static_cast<uint32_t>(16 * j) << 16) + kAcol0;
-  int s = 0;
+  StepCursor c{0, par, unit_block(p, 0, n_my, j)};
+  cursor_normalize(c, p, n_my, j);
+  int s = par;
   uint32_t ph = 0;
-  uint32_t it = 0;
-  for (int ui = 0; ui < n_my; ++ui) {
-    const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
-    const bool valid = (u / p.n_nt) * 8 + j < p.n_mtiles;
-    for (int ks = 0; ks < p.n_ks; ++ks, ++it) {
-      if (!tc_wait_warp(sm, &sm.empty[s], ph ^ 1u, p.status)) {
-        cp_async_wait_all();
-        return;
-      }
-      tc_fence_after();
-      const uint32_t rs = it & (kTcRing - 1);
-      const uint8_t* slot = ring + rs * kTcSlotBytes;
-      cp_async_wait<kTcRing - 1>();
-      __syncwarp();
-      uint32_t r[16];
-      if (!valid) {
+  uint32_t slot_i = 0;
+  for (long it = par; it < total; it += 2) {
+    issue_next();   // into the slot the previous step freed
+    if (!tc_wait_warp(sm, &sm.empty[s], ph ^ 1u, p.status)) break;
+    tc_fence_after();
+    const uint8_t* slot = ring + slot_i * kTcSlotBytes;
+    cp_async_wait<kTcRing - 1>();
+    __syncwarp();
+    uint32_t r[16];
+    if (c.blk == nullptr) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) r[i] = 0u;
-      } else if (ks < p.ks_core) {
-        dequant_residual(p, slot, ks, lane, r);
-      } else if (ks < p.ks_corr) {
-        dequant_core(p, slot, lane, r);
-      } else {
-        dequant_corr(p, slot, 2 * (ks - p.ks_corr) + 1 < p.n_A, lane, r);
-      }
-      __syncwarp();   // every lane is done reading the slot
-      issue_next(rs);
-      tmem_st_16x256b_x4(tmem_row + static_cast<uint32_t>(s) * 32u, r);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&sm.full[s]));
-      if (++s == kTcStages) {
-        s = 0;
-        ph ^= 1u;
-      }
+      for (int i = 0; i < 16; ++i) r[i] = 0u;
+    } else if (c.ks < p.ks_core) {
+      dequant_residual(p, slot, c.ks, lane, r);
+    } else if (c.ks < p.ks_corr) {
+      dequant_core(p, slot, lane, r);
+    } else {
+      dequant_corr(p, slot, 2 * (c.ks - p.ks_corr) + 1 < p.n_A, lane, r);
+    }
+    tmem_st_16x256b_x4(tmem_row + static_cast<uint32_t>(s) * 32u, r);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();   // every lane is done reading the slot and storing to TMEM
+    if (lane == 0) mbar_arrive(smem_addr(&sm.full[s]));
+    if (++slot_i == kTcRing) slot_i = 0;
+    cursor_advance(c, p, n_my, j);
+    s += 2;
+    if (s >= kTcStages) {
+      s -= kTcStages;
+      ph ^= 1u;
     }
   }
   cp_async_wait_all();
@@ -321,9 +352,17 @@ __device__ void mma_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base
 }
 
 // ----------------------------------------------------------- epilogue warps
+// Warp q owns accumulator rows 32q..32q+31 (its TMEM lane quarter).  Per chunk
+// of 32 token columns it loads its 32 x 32 block, transposes it through a
+// private padded tile in shared memory, and lane c then folds token column c
+// over the 32 rows on its own: max and first argmax, then sum of exp, the
+// target logit if it falls in these rows, and the logits row segment if asked.
+// The four warps' states of a token are merged into one partial per
+// (token, 128-row tile).
 __device__ void epilogue_warps(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int ew, int lane) {
-  grid_dependency_wait();   // c_t, and the previous call's readers of the outputs
+  grid_dependency_wait();   // 2^-c_t, and the previous call's readers of the outputs
   const int q = (kTcDeqWarps + 2 + ew) & 3;   // TMEM lane quarter of this warp
+  float* tile = sm.etile + q * (32 * 33);
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
   bool ok = true;
@@ -334,37 +373,52 @@ __device__ void epilogue_warps(const TcParams& p, const TcSmem& sm, uint32_t tme
     if (ok) ok = tc_wait_warp(sm, &sm.accf[a], (static_cast<uint32_t>(ui) >> 1) & 1u, p.status);
     if (ok) {
       tc_fence_after();
-      const int v = mt * kTcBM + 32 * q + lane;
-      const bool v_ok = v < p.V;
+      const int v0 = mt * kTcBM + 32 * q;
+      const int nrow = min(32, p.V - v0);          // rows of this warp inside the vocabulary
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * kAccStride;
       const int ncol = min(p.BN, p.T - tb);
-      for (int c0 = 0; c0 < ncol; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c0), r);
+      for (int c0 = 0; c0 < ncol; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c0), r);
         tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int col = c0 + jj;
-          if (col >= ncol) break;
+        for (int jj = 0; jj < 32; ++jj) tile[jj * 33 + lane] = __uint_as_float(r[jj]);
+        __syncwarp();
+        const int col = c0 + lane;
+        if (col < ncol && nrow > 0) {
           const int t = tb + col;
-          const float inv = ldexpf(1.f, -__ldg(p.cexp + t));
-          const float y = v_ok ? __uint_as_float(r[jj]) * inv : -INFINITY;
-          if (v_ok) {
-            if (p.logits != nullptr) p.logits[static_cast<size_t>(t) * p.V + v] = y;
-            if (p.targets != nullptr && __ldg(p.targets + t) == v) p.tgt[t] = y;
-          }
-          float m = y;
+          const float inv = __ldg(p.cinv + t);
+          float y[32];
+          float m = -INFINITY;
+          int idx = 0x7fffffff;
 #pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-          float e = v_ok ? __expf(y - m) : 0.f;
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-          const uint32_t ball = __ballot_sync(0xffffffffu, v_ok && y == m);
-          if (lane == 0) {
-            const int idx = ball != 0u ? mt * kTcBM + 32 * q + __ffs(ball) - 1 : 0x7fffffff;
-            sm.epi[q * kTcMaxBN + col] = make_float4(m, e, __int_as_float(idx), 0.f);
+          for (int k = 0; k < 32; ++k) {
+            y[k] = tile[lane * 33 + k] * inv;
+            if (k < nrow && y[k] > m) {
+              m = y[k];
+              idx = v0 + k;
+            }
           }
+          float e = 0.f;
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (k < nrow) e += __expf(y[k] - m);
+          if (p.targets != nullptr) {
+            const int tg = __ldg(p.targets + t) - v0;
+            if (tg >= 0 && tg < nrow) p.tgt[t] = tile[lane * 33 + tg] * inv;
+          }
+          if (p.logits != nullptr) {
+            float* dst = p.logits + static_cast<size_t>(t) * p.V + v0;
+            if (nrow == 32 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 4) *reinterpret_cast<float4*>(dst + k) = make_float4(y[k], y[k + 1], y[k + 2], y[k + 3]);
+            } else {
+              for (int k = 0; k < nrow; ++k) dst[k] = tile[lane * 33 + k] * inv;
+            }
+          }
+          sm.epi[q * kTcMaxBN + col] = make_float4(m, e, __int_as_float(idx), 0.f);
         }
+        __syncwarp();
       }
       tc_fence_before();
     }
@@ -377,6 +431,7 @@ __device__ void epilogue_warps(const TcParams& p, const TcSmem& sm, uint32_t tme
       LseState st = lse_init();
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
+        if (mt * kTcBM + 32 * w >= p.V) continue;   // rows past the vocabulary: no state
         const float4 e = sm.epi[w * kTcMaxBN + col];
         st = lse_merge(st, LseState{e.x, e.y, __float_as_int(e.z)});
       }
@@ -396,7 +451,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(smem_addr(&sm.full[s]), kTcDeqWarps + 1);
+      mbar_init(smem_addr(&sm.full[s]), kTcDeqWarps / 2 + 1);   // the eight warps of the stage's parity + TMA
       mbar_init(smem_addr(&sm.empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -458,7 +513,7 @@ void tc_smem_plan(TcParams& p) {
   p.bstage_bytes = static_cast<uint32_t>(p.BN) * 128u;   // multiple of 2048 (BN % 16 == 0)
   p.ring_off = kTcStages * p.bstage_bytes;
   p.epi_off = p.ring_off + kTcDeqWarps * kTcRing * kTcSlotBytes;
-  p.bar_off = p.epi_off + 4 * kTcMaxBN * 16;
+  p.bar_off = p.epi_off + 4 * kTcMaxBN * 16 + 4 * 32 * 33 * 4;
 }
 
 size_t tc_smem_bytes(const TcParams& p) { return static_cast<size_t>(p.bar_off) + 256 + 1024; }
