@@ -86,6 +86,7 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
   tp.ks_core = L.n_res;
   tp.ks_corr = L.n_res + L.n_L;
   tp.n_ks = Kc / kTcBK;
+  tp.n_st = (tp.n_ks + kTcStepsPerStage - 1) / kTcStepsPerStage;
   tp.off_res = L.off_res;
   tp.off_Lnib = L.off_Lnib;
   tp.off_Lhi = L.off_Lhi;

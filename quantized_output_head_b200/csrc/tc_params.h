@@ -14,10 +14,12 @@ namespace archead {
 
 constexpr int kTcBM = 128;            // vocabulary rows per unit (8 m-tile blocks of 16)
 constexpr int kTcBK = 64;             // K columns per k-step (one 128-byte row of fp16)
+constexpr int kTcStepsPerStage = 2;   // k-steps per pipeline stage
 constexpr int kTcMaxBN = 128;         // tokens per unit
-constexpr int kTcStages = 6;          // k-steps in flight between the producers and the MMA
-constexpr int kTcRing = 5;            // ring slots per dequantising warp (kTcRing - 1 k-steps prefetched)
-constexpr int kTcSlotBytes = 1152;    // one packed k-step of one m-tile block (codes + scales)
+constexpr int kTcMaxStages = 8;       // stages in flight between the producers and the MMA (even)
+constexpr int kTcRingSmall = 3;       // ring slots (stages of packed bytes) per dequantising warp, BN <= 64
+constexpr int kTcRingLarge = 2;       // the same for BN > 64
+constexpr int kTcSlotBytes = 1056;    // one packed k-step of one m-tile block (codes + scales)
 constexpr int kTcDeqWarps = 16;       // two per m-tile block of a unit (even / odd k-steps)
 constexpr int kTcWarps = 22;          // 16 dequantising, 1 TMA, 1 MMA, 4 epilogue
 constexpr int kTcMinTokens = 16;      // calls with fewer tokens take the decode kernel
@@ -33,8 +35,11 @@ struct TcParams {
   int32_t T, V, BN, n_nt, n_mt128, n_units;
   int32_t n_res, n_L, n_A, n_mtiles, g_log2;   // chunks per segment; log2 of the residual group
   int32_t n_ks, ks_core, ks_corr;              // k-steps: total, first core, first correction
+  int32_t n_st;                                // stages per unit: ceil(n_ks / 2)
   uint32_t off_res, off_Lnib, off_Lhi, off_A, off_sres, off_sL, off_sA, mblk_bytes;
   float sc_res, sc_L, sc_A;                    // 2^alpha, 2^beta, 2^gamma
+  int32_t stages, ring;                        // stage buffers (even, <= kTcMaxStages); ring slots per warp
+  uint32_t acc_stride, acol0;                  // TMEM columns: accumulator stride, first A stage
   uint32_t bstage_bytes, ring_off, epi_off, bar_off;   // shared-memory plan
 };
 

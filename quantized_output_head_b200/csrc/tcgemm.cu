@@ -29,6 +29,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "device.cuh"
@@ -40,17 +41,15 @@ namespace archead {
 namespace {
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccStride = 128;            // TMEM columns per accumulator
-constexpr uint32_t kAcol0 = 2 * kAccStride;     // first column of the A stages
-static_assert(kAcol0 + kTcStages * 32 <= kTmemCols, "TMEM plan");
+static_assert(kTcMaxStages % 2 == 0, "stage parity");
 
 struct TcSmem {
-  uint8_t* bst;        // [kTcStages][bstage_bytes], 1024-byte aligned
-  uint8_t* rings;      // [kTcDeqWarps][kTcRing][kTcSlotBytes]
+  uint8_t* bst;        // [stages][bstage_bytes], 1024-byte aligned
+  uint8_t* rings;      // [kTcDeqWarps][ring][2 x kTcSlotBytes]
   float4* epi;         // [4][kTcMaxBN] per-warp (max, sum, idx) of the current unit
   float* etile;        // [4][32 x 33] per-warp transpose tiles of the epilogue
-  uint64_t* full;      // [kTcStages] dequant warps + TMA -> MMA
-  uint64_t* empty;     // [kTcStages] MMA -> dequant warps + TMA
+  uint64_t* full;      // [kTcMaxStages] dequant warps + TMA -> MMA
+  uint64_t* empty;     // [kTcMaxStages] MMA -> dequant warps + TMA
   uint64_t* accf;      // [2] MMA -> epilogue
   uint64_t* acce;      // [2] epilogue -> MMA
   uint32_t* tmem;      // TMEM base address
@@ -65,10 +64,10 @@ __device__ __forceinline__ TcSmem tc_smem(uint8_t* base, const TcParams& p) {
   s.etile = reinterpret_cast<float*>(base + p.epi_off + 4 * kTcMaxBN * 16);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + p.bar_off);
   s.full = bars;
-  s.empty = bars + kTcStages;
-  s.accf = bars + 2 * kTcStages;
-  s.acce = bars + 2 * kTcStages + 2;
-  s.tmem = reinterpret_cast<uint32_t*>(bars + 2 * kTcStages + 4);
+  s.empty = bars + kTcMaxStages;
+  s.accf = bars + 2 * kTcMaxStages;
+  s.acce = bars + 2 * kTcMaxStages + 2;
+  s.tmem = reinterpret_cast<uint32_t*>(bars + 2 * kTcMaxStages + 4);
   s.abort_flag = reinterpret_cast<int*>(s.tmem + 1);
   return s;
 }
@@ -100,27 +99,30 @@ __device__ __forceinline__ bool tc_wait_warp(const TcSmem& s, uint64_t* bar, uin
 }
 
 // ------------------------------------------------------- dequantising warps
-// Packed bytes of one k-step of one m-tile block -> ring slot:
-//   residual  [0,512) codes, [1024, ...) group scales of the 64 columns
-//   core      [0,512) low nibbles, [512,640) fifth bits, [1024,1056) s_L
+// Packed bytes of one k-step of one m-tile block -> ring slot (kTcSlotBytes):
+//   residual   [0,512) codes, [512, 512 + 32 * groups) group scales
+//   core       [0,512) low nibbles, [512,640) fifth bits, [640,672) s_L
 //   correction [0,1024) two 32-column chunks, [1024,1056) s_A
+constexpr int kSlotResScales = 512, kSlotCoreHi = 512, kSlotCoreScales = 640, kSlotCorrScales = 1024;
+
 __device__ __forceinline__ void issue_step(const TcParams& p, uint32_t dst, const uint8_t* blk, int ks, int lane) {
   if (ks < p.ks_core) {
     cp_async16(dst + lane * 16, blk + p.off_res + ks * kResChunkBytes + lane * 16);
     const int gsh = p.g_log2;
     const int g0 = (ks * kTcBK) >> gsh;
     const int nbytes = (gsh >= 6 ? 1 : (kTcBK >> gsh)) * kSresGroupBytes;
-    if (lane * 16 < nbytes) cp_async16(dst + 1024 + lane * 16, blk + p.off_sres + g0 * kSresGroupBytes + lane * 16);
+    if (lane * 16 < nbytes)
+      cp_async16(dst + kSlotResScales + lane * 16, blk + p.off_sres + g0 * kSresGroupBytes + lane * 16);
   } else if (ks < p.ks_corr) {
     const int c = ks - p.ks_core;
     cp_async16(dst + lane * 16, blk + p.off_Lnib + c * kLNibChunkBytes + lane * 16);
-    if (lane < 8) cp_async16(dst + 512 + lane * 16, blk + p.off_Lhi + c * kLHiChunkBytes + lane * 16);
-    if (lane < 2) cp_async16(dst + 1024 + lane * 16, blk + p.off_sL + lane * 16);
+    if (lane < 8) cp_async16(dst + kSlotCoreHi + lane * 16, blk + p.off_Lhi + c * kLHiChunkBytes + lane * 16);
+    if (lane < 2) cp_async16(dst + kSlotCoreScales + lane * 16, blk + p.off_sL + lane * 16);
   } else {
     const int a = 2 * (ks - p.ks_corr);
     cp_async16(dst + lane * 16, blk + p.off_A + a * kAChunkBytes + lane * 16);
     if (a + 1 < p.n_A) cp_async16(dst + 512 + lane * 16, blk + p.off_A + (a + 1) * kAChunkBytes + lane * 16);
-    if (lane < 2) cp_async16(dst + 1024 + lane * 16, blk + p.off_sA + lane * 16);
+    if (lane < 2) cp_async16(dst + kSlotCorrScales + lane * 16, blk + p.off_sA + lane * 16);
   }
 }
 
@@ -150,7 +152,7 @@ __device__ __forceinline__ void dequant_residual(const TcParams& p, const uint8_
   for (int st = 0; st < 4; ++st) {
     // local group of this k16 step (groups are >= 16 columns, powers of two)
     const int lg = ((ks * kTcBK + 16 * st) >> gsh) - ((ks * kTcBK) >> gsh);
-    if (st == 0 || gsh < 6) scale_pair(slot + 1024 + lg * kSresGroupBytes + gr * 4, p.sc_res, s0, s1);
+    if (st == 0 || gsh < 6) scale_pair(slot + kSlotResScales + lg * kSresGroupBytes + gr * 4, p.sc_res, s0, s1);
     uint32_t a[4];
     unpack_int4_signed(w[st], a);
     place(a, s0, s1, r + 4 * st);
@@ -160,9 +162,9 @@ __device__ __forceinline__ void dequant_residual(const TcParams& p, const uint8_
 __device__ __forceinline__ void dequant_core(const TcParams& p, const uint8_t* slot, int lane, uint32_t (&r)[16]) {
   const int gr = lane >> 2;
   const uint4 n = *reinterpret_cast<const uint4*>(slot + lane * 16);
-  const uint32_t hb = *reinterpret_cast<const uint32_t*>(slot + 512 + lane * 4);
+  const uint32_t hb = *reinterpret_cast<const uint32_t*>(slot + kSlotCoreHi + lane * 4);
   uint32_t s0, s1;
-  scale_pair(slot + 1024 + gr * 4, p.sc_L, s0, s1);
+  scale_pair(slot + kSlotCoreScales + gr * 4, p.sc_L, s0, s1);
   uint32_t a[4];
   unpack_int5_signed<0>(n.x, hb, a);
   place(a, s0, s1, r + 0);
@@ -178,7 +180,7 @@ __device__ __forceinline__ void dequant_corr(const TcParams& p, const uint8_t* s
                                              uint32_t (&r)[16]) {
   const int gr = lane >> 2;
   uint32_t s0, s1;
-  scale_pair(slot + 1024 + gr * 4, p.sc_A, s0, s1);
+  scale_pair(slot + kSlotCorrScales + gr * 4, p.sc_A, s0, s1);
   const uint4 c0 = *reinterpret_cast<const uint4*>(slot + lane * 16);
   uint32_t a[4];
   unpack_int8_signed(c0.x, c0.y, a);
@@ -206,88 +208,107 @@ __device__ __forceinline__ const uint8_t* unit_block(const TcParams& p, int ui, 
   return mt16 < p.n_mtiles ? p.mtiles + static_cast<size_t>(mt16) * p.mblk_bytes : nullptr;
 }
 
-// Cursor over the global k-steps it = par, par + 2, ... of this CTA's units.
-struct StepCursor {
-  int ui, ks;
+// Cursor over the global stages g = par, par + 2, ... of this CTA's units
+// (stage st of a unit holds k-steps 2st and 2st + 1).
+struct StageCursor {
+  int ui, st;
   const uint8_t* blk;
 };
-__device__ __forceinline__ void cursor_normalize(StepCursor& c, const TcParams& p, int n_my, int j) {
-  while (c.ks >= p.n_ks) {
-    c.ks -= p.n_ks;
+__device__ __forceinline__ void cursor_normalize(StageCursor& c, const TcParams& p, int n_my, int j) {
+  while (c.st >= p.n_st) {
+    c.st -= p.n_st;
     ++c.ui;
     c.blk = unit_block(p, c.ui, n_my, j);
   }
 }
-__device__ __forceinline__ void cursor_advance(StepCursor& c, const TcParams& p, int n_my, int j) {
-  c.ks += 2;
+__device__ __forceinline__ void cursor_advance(StageCursor& c, const TcParams& p, int n_my, int j) {
+  c.st += 2;
   cursor_normalize(c, p, n_my, j);
 }
 
+__device__ __forceinline__ void dequant_step(const TcParams& p, const uint8_t* slot, int ks, int lane,
+                                             uint32_t (&r)[16]) {
+  if (ks < p.ks_core) dequant_residual(p, slot, ks, lane, r);
+  else if (ks < p.ks_corr) dequant_core(p, slot, lane, r);
+  else dequant_corr(p, slot, 2 * (ks - p.ks_corr) + 1 < p.n_A, lane, r);
+}
+
 // Warp w dequantises m-tile block j = 2(w%4) + (w/4)%2 of every unit (TMEM
-// lanes 16j..16j+15 lie in the warp's lane quarter w%4) on the global k-steps
-// of parity w/8; a stage index has a fixed parity (kTcStages is even), so each
-// stage is filled by the same eight warps.
+// lanes 16j..16j+15 lie in the warp's lane quarter w%4) on the global stages
+// of parity w/8; a stage buffer has a fixed parity (the buffer count is even),
+// so each buffer is filled by the same eight warps.  R: ring slots, each the
+// packed bytes of one stage (two k-steps).
+template <int R>
 __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int w, int lane) {
-  static_assert(kTcStages % 2 == 0, "stage parity");
+  constexpr uint32_t kPair = 2 * kTcSlotBytes;
   const int j = 2 * (w & 3) + ((w >> 2) & 1);
   const int par = w >> 3;
-  const uint32_t ring_s = smem_addr(sm.rings) + static_cast<uint32_t>(w) * kTcRing * kTcSlotBytes;
-  const uint8_t* ring = sm.rings + static_cast<size_t>(w) * kTcRing * kTcSlotBytes;
+  const uint32_t ring_s = smem_addr(sm.rings) + static_cast<uint32_t>(w) * R * kPair;
+  const uint8_t* ring = sm.rings + static_cast<size_t>(w) * R * kPair;
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
-  const long total = static_cast<long>(n_my) * p.n_ks;   // global k-steps of this CTA
+  const long total = static_cast<long>(n_my) * p.n_st;   // global stages of this CTA
 
-  // Prefetch kTcRing - 1 of this warp's steps ahead.
-  StepCursor pc{0, par, unit_block(p, 0, n_my, j)};
-  long pit = par;
+  // Prefetch R - 1 of this warp's stages ahead.
+  StageCursor pc{0, par, unit_block(p, 0, n_my, j)};
   cursor_normalize(pc, p, n_my, j);
+  long pg = par;
   uint32_t pslot = 0;
   auto issue_next = [&]() {
-    if (pit < total && pc.blk != nullptr) issue_step(p, ring_s + pslot * kTcSlotBytes, pc.blk, pc.ks, lane);
+    if (pg < total && pc.blk != nullptr) {
+      const uint32_t dst = ring_s + pslot * kPair;
+      const int ks0 = 2 * pc.st;
+      issue_step(p, dst, pc.blk, ks0, lane);
+      if (ks0 + 1 < p.n_ks) issue_step(p, dst + kTcSlotBytes, pc.blk, ks0 + 1, lane);
+    }
     cp_async_commit();
-    if (pit < total) {
-      pit += 2;
+    if (pg < total) {
+      pg += 2;
       cursor_advance(pc, p, n_my, j);
     }
-    if (++pslot == kTcRing) pslot = 0;
+    if (++pslot == R) pslot = 0;
   };
 #pragma unroll 1
-  for (int k = 0; k < kTcRing - 1; ++k) issue_next();
+  for (int k = 0; k < R - 1; ++k) issue_next();
 
-  const uint32_t tmem_row = tmem_base + (static_cast<uint32_t>(16 * j) << 16) + kAcol0;
-  StepCursor c{0, par, unit_block(p, 0, n_my, j)};
+  const uint32_t tmem_row = tmem_base + (static_cast<uint32_t>(16 * j) << 16) + p.acol0;
+  StageCursor c{0, par, unit_block(p, 0, n_my, j)};
   cursor_normalize(c, p, n_my, j);
   int s = par;
   uint32_t ph = 0;
   uint32_t slot_i = 0;
-  for (long it = par; it < total; it += 2) {
-    issue_next();   // into the slot the previous step freed
+  for (long g = par; g < total; g += 2) {
+    issue_next();   // into the slot the previous stage freed
     if (!tc_wait_warp(sm, &sm.empty[s], ph ^ 1u, p.status)) break;
     tc_fence_after();
-    const uint8_t* slot = ring + slot_i * kTcSlotBytes;
-    cp_async_wait<kTcRing - 1>();
+    const uint8_t* slot = ring + slot_i * kPair;
+    cp_async_wait<R - 1>();
     __syncwarp();
-    uint32_t r[16];
+    const int ks0 = 2 * c.st;
+    const bool two = ks0 + 1 < p.n_ks;
+    uint32_t r0[16], r1[16];
     if (c.blk == nullptr) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) r[i] = 0u;
-    } else if (c.ks < p.ks_core) {
-      dequant_residual(p, slot, c.ks, lane, r);
-    } else if (c.ks < p.ks_corr) {
-      dequant_core(p, slot, lane, r);
+      for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
+    } else if (two && ks0 + 1 < p.ks_core) {
+      dequant_residual(p, slot, ks0, lane, r0);   // the common case: both k-steps residual
+      dequant_residual(p, slot + kTcSlotBytes, ks0 + 1, lane, r1);
     } else {
-      dequant_corr(p, slot, 2 * (c.ks - p.ks_corr) + 1 < p.n_A, lane, r);
+      dequant_step(p, slot, ks0, lane, r0);
+      if (two) dequant_step(p, slot + kTcSlotBytes, ks0 + 1, lane, r1);
     }
-    tmem_st_16x256b_x4(tmem_row + static_cast<uint32_t>(s) * 32u, r);
+    const uint32_t ta = tmem_row + static_cast<uint32_t>(s) * 64u;
+    tmem_st_16x256b_x4(ta, r0);
+    if (two) tmem_st_16x256b_x4(ta + 32u, r1);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();   // every lane is done reading the slot and storing to TMEM
     if (lane == 0) mbar_arrive(smem_addr(&sm.full[s]));
-    if (++slot_i == kTcRing) slot_i = 0;
+    if (++slot_i == R) slot_i = 0;
     cursor_advance(c, p, n_my, j);
     s += 2;
-    if (s >= kTcStages) {
-      s -= kTcStages;
+    if (s >= p.stages) {
+      s -= p.stages;
       ph ^= 1u;
     }
   }
@@ -295,9 +316,10 @@ __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_
 }
 
 // ---------------------------------------------------------------- TMA warp
+// Stage buffer: two BN x 64 tiles of X (one per k-step), 128-byte swizzle.
 __device__ void tma_warp(const TcParams& p, const TcSmem& sm, const CUtensorMap* xmap, int lane) {
   if (lane != 0) return;
-  grid_dependency_wait();   // X and c_t come from the activation kernel
+  grid_dependency_wait();   // X and 2^-c_t come from the activation kernel
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
   const uint32_t bst = smem_addr(sm.bst);
@@ -306,12 +328,16 @@ __device__ void tma_warp(const TcParams& p, const TcSmem& sm, const CUtensorMap*
   for (int ui = 0; ui < n_my; ++ui) {
     const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
     const int y = (u % p.n_nt) * p.BN;
-    for (int ks = 0; ks < p.n_ks; ++ks) {
+    for (int st = 0; st < p.n_st; ++st) {
       if (!tc_wait(sm, &sm.empty[s], ph ^ 1u, p.status)) return;
+      const int ks0 = 2 * st;
+      const bool two = ks0 + 1 < p.n_ks;
       const uint32_t bar = smem_addr(&sm.full[s]);
-      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(p.BN) * 128u);
-      tma_load_2d(bst + static_cast<uint32_t>(s) * p.bstage_bytes, xmap, ks * kTcBK, y, bar);
-      if (++s == kTcStages) {
+      const uint32_t dst = bst + static_cast<uint32_t>(s) * 2u * p.bstage_bytes;
+      mbar_arrive_expect_tx(bar, (two ? 2u : 1u) * static_cast<uint32_t>(p.BN) * 128u);
+      tma_load_2d(dst, xmap, ks0 * kTcBK, y, bar);
+      if (two) tma_load_2d(dst + p.bstage_bytes, xmap, (ks0 + 1) * kTcBK, y, bar);
+      if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
       }
@@ -332,17 +358,21 @@ __device__ void mma_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base
     const uint32_t a = static_cast<uint32_t>(ui) & 1u;
     if (!tc_wait(sm, &sm.acce[a], ((static_cast<uint32_t>(ui) >> 1) & 1u) ^ 1u, p.status)) return;
     tc_fence_after();
-    const uint32_t d_tmem = tmem_base + a * kAccStride;
-    for (int ks = 0; ks < p.n_ks; ++ks) {
+    const uint32_t d_tmem = tmem_base + a * p.acc_stride;
+    for (int st = 0; st < p.n_st; ++st) {
       if (!tc_wait(sm, &sm.full[s], ph, p.status)) return;
       tc_fence_after();
-      const uint64_t bdesc = smem_desc_k128(bst + static_cast<uint32_t>(s) * p.bstage_bytes);
-      const uint32_t a_tmem = tmem_base + kAcol0 + static_cast<uint32_t>(s) * 32u;
+      const int nk = 2 * st + 1 < p.n_ks ? 2 : 1;
+      const uint32_t b0 = bst + static_cast<uint32_t>(s) * 2u * p.bstage_bytes;
+      const uint32_t a0 = tmem_base + p.acol0 + static_cast<uint32_t>(s) * 64u;
+      for (int h = 0; h < nk; ++h) {
+        const uint64_t bdesc = smem_desc_k128(b0 + static_cast<uint32_t>(h) * p.bstage_bytes);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        tc_mma_ts(d_tmem, a_tmem + 8u * i, bdesc + 2u * i, idesc, (ks | i) != 0 ? 1u : 0u);
+        for (int i = 0; i < 4; ++i)
+          tc_mma_ts(d_tmem, a0 + 32u * h + 8u * i, bdesc + 2u * i, idesc, (st | h | i) != 0 ? 1u : 0u);
+      }
       tc_commit(smem_addr(&sm.empty[s]));
-      if (++s == kTcStages) {
+      if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
       }
@@ -375,7 +405,7 @@ __device__ void epilogue_warps(const TcParams& p, const TcSmem& sm, uint32_t tme
       tc_fence_after();
       const int v0 = mt * kTcBM + 32 * q;
       const int nrow = min(32, p.V - v0);          // rows of this warp inside the vocabulary
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * kAccStride;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * p.acc_stride;
       const int ncol = min(p.BN, p.T - tb);
       for (int c0 = 0; c0 < ncol; c0 += 32) {
         uint32_t r[32];
@@ -443,6 +473,7 @@ __device__ void epilogue_warps(const TcParams& p, const TcSmem& sm, uint32_t tme
 
 }  // namespace
 
+template <int R>
 __global__ void __launch_bounds__(kTcWarps * 32, 1)
     tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap xmap) {
   extern __shared__ uint8_t smem_raw[];
@@ -450,7 +481,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1)
   const TcSmem sm = tc_smem(base, p);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < kTcMaxStages; ++s) {
       mbar_init(smem_addr(&sm.full[s]), kTcDeqWarps / 2 + 1);   // the eight warps of the stage's parity + TMA
       mbar_init(smem_addr(&sm.empty[s]), 1);
     }
@@ -470,7 +501,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1)
   tc_fence_after();
   const uint32_t tmem_base = *sm.tmem;
 
-  if (warp < kTcDeqWarps) dequant_warp(p, sm, tmem_base, warp, lane);
+  if (warp < kTcDeqWarps) dequant_warp<R>(p, sm, tmem_base, warp, lane);
   else if (warp == kTcDeqWarps) tma_warp(p, sm, &xmap, lane);
   else if (warp == kTcDeqWarps + 1) mma_warp(p, sm, tmem_base, lane);
   else epilogue_warps(p, sm, tmem_base, warp - kTcDeqWarps - 2, lane);
@@ -509,25 +540,47 @@ __global__ void __launch_bounds__(256) tc_merge_kernel(const float4* partials, i
 }
 
 // ------------------------------------------------------------------- host
+// TMEM: two accumulators of acc_stride columns, then one 64-column A tile (two
+// k-steps) per stage buffer; the buffers use what the accumulators leave of the
+// 512 columns.  Shared memory: two X tiles per stage buffer, the dequantising
+// warps' rings, the epilogue tiles and the barriers.
 void tc_smem_plan(TcParams& p) {
-  p.bstage_bytes = static_cast<uint32_t>(p.BN) * 128u;   // multiple of 2048 (BN % 16 == 0)
-  p.ring_off = kTcStages * p.bstage_bytes;
-  p.epi_off = p.ring_off + kTcDeqWarps * kTcRing * kTcSlotBytes;
+  p.acc_stride = static_cast<uint32_t>((p.BN + 31) / 32 * 32);
+  p.acol0 = 2 * p.acc_stride;
+  p.stages = static_cast<int32_t>(std::min<uint32_t>(kTcMaxStages, (kTmemCols - p.acol0) / 64)) & ~1;
+  p.ring = p.BN <= 64 ? kTcRingSmall : kTcRingLarge;
+  p.bstage_bytes = static_cast<uint32_t>(p.BN) * 128u;   // one X tile; multiple of 2048 (BN % 16 == 0)
+  p.ring_off = static_cast<uint32_t>(p.stages) * 2u * p.bstage_bytes;
+  p.epi_off = p.ring_off + kTcDeqWarps * p.ring * 2 * kTcSlotBytes;
   p.bar_off = p.epi_off + 4 * kTcMaxBN * 16 + 4 * 32 * 33 * 4;
 }
 
 size_t tc_smem_bytes(const TcParams& p) { return static_cast<size_t>(p.bar_off) + 256 + 1024; }
 
 size_t tc_smem_max() {
-  TcParams p{};
-  p.BN = kTcMaxBN;
-  tc_smem_plan(p);
-  return tc_smem_bytes(p);
+  size_t m = 0;
+  for (int bn = 16; bn <= kTcMaxBN; bn += 16) {
+    TcParams p{};
+    p.BN = bn;
+    tc_smem_plan(p);
+    m = std::max(m, tc_smem_bytes(p));
+  }
+  return m;
 }
 
+namespace {
+const void* tc_kernel_for(int ring) {
+  return ring == kTcRingSmall ? reinterpret_cast<const void*>(&tc_kernel<kTcRingSmall>)
+                              : reinterpret_cast<const void*>(&tc_kernel<kTcRingLarge>);
+}
+}  // namespace
+
 cudaError_t tc_set_attributes() {
-  return cudaFuncSetAttribute(reinterpret_cast<const void*>(&tc_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(tc_smem_max()));
+  const int smem = static_cast<int>(tc_smem_max());
+  cudaError_t e = cudaFuncSetAttribute(tc_kernel_for(kTcRingSmall), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tc_kernel_for(kTcRingLarge), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
 }
 
 namespace {
@@ -570,7 +623,7 @@ cudaError_t launch_tc(const TcParams& p, const CUtensorMap& map, int grid, cudaS
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   void* args[] = {const_cast<TcParams*>(&p), const_cast<CUtensorMap*>(&map)};
-  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&tc_kernel), args);
+  return cudaLaunchKernelExC(&cfg, tc_kernel_for(p.ring), args);
 }
 
 cudaError_t launch_tc_merge(const float4* partials, int n_mt128, int T, const int32_t* targets, const float* tgt,
