@@ -190,7 +190,7 @@ def test_small_shapes(qoh, V, d, r_c, r_r, g, g_B, T):
     assert np.array_equal(am.cpu().numpy(), am2.cpu().numpy())
 
 
-# Calls of >= 16 tokens take the tensor-core kernel when g_B is a multiple of 64.
+# Calls of >= 9 tokens take the tensor-core kernel when g_B is a multiple of 64.
 SMALL_TC = [
     # V,    d,   r_c, r_r, g,   g_B, T
     (1000, 320, 32, 8, 64, 64, 16),       # ragged vocabulary, one 32-column correction chunk
@@ -198,7 +198,8 @@ SMALL_TC = [
     (1500, 512, 64, 0, 32, 64, 130),      # no correction, g = 32, two token tiles
     (4099, 512, 128, 64, 256, 128, 40),   # g = 256, last 128-row tile nearly empty
     (300, 128, 64, 32, 128, 128, 200),    # three 128-row tiles, the last partial
-    (1003, 320, 100, 40, 16, 10, 20),     # g_B = 10: 16+ tokens through the decode kernel
+    (777, 192, 64, 64, 64, 64, 9),        # fewest tokens of the tensor-core path, odd k-step count
+    (1003, 320, 100, 40, 16, 10, 20),     # g_B = 10: 9+ tokens through the decode kernel
 ]
 
 
