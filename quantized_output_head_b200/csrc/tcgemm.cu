@@ -316,9 +316,9 @@ __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_
 }
 
 // ---------------------------------------------------------------- TMA warp
-// Stage buffer: two BN x 64 tiles of X (one per k-step), 128-byte swizzle.
+// Stage buffer: two BN x 64 tiles of X (one per k-step), 128-byte swizzle.  The
+// whole warp walks the stages; one elected lane issues.
 __device__ void tma_warp(const TcParams& p, const TcSmem& sm, const CUtensorMap* xmap, int lane) {
-  if (lane != 0) return;
   grid_dependency_wait();   // X and 2^-c_t come from the activation kernel
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
@@ -329,14 +329,17 @@ __device__ void tma_warp(const TcParams& p, const TcSmem& sm, const CUtensorMap*
     const int u = static_cast<int>(blockIdx.x) + ui * static_cast<int>(gridDim.x);
     const int y = (u % p.n_nt) * p.BN;
     for (int st = 0; st < p.n_st; ++st) {
-      if (!tc_wait(sm, &sm.empty[s], ph ^ 1u, p.status)) return;
+      if (!tc_wait_warp(sm, &sm.empty[s], ph ^ 1u, p.status)) return;
       const int ks0 = 2 * st;
       const bool two = ks0 + 1 < p.n_ks;
-      const uint32_t bar = smem_addr(&sm.full[s]);
-      const uint32_t dst = bst + static_cast<uint32_t>(s) * 2u * p.bstage_bytes;
-      mbar_arrive_expect_tx(bar, (two ? 2u : 1u) * static_cast<uint32_t>(p.BN) * 128u);
-      tma_load_2d(dst, xmap, ks0 * kTcBK, y, bar);
-      if (two) tma_load_2d(dst + p.bstage_bytes, xmap, (ks0 + 1) * kTcBK, y, bar);
+      if (elect_one()) {
+        const uint32_t bar = smem_addr(&sm.full[s]);
+        const uint32_t dst = bst + static_cast<uint32_t>(s) * 2u * p.bstage_bytes;
+        mbar_arrive_expect_tx(bar, (two ? 2u : 1u) * static_cast<uint32_t>(p.BN) * 128u);
+        tma_load_2d(dst, xmap, ks0 * kTcBK, y, bar);
+        if (two) tma_load_2d(dst + p.bstage_bytes, xmap, (ks0 + 1) * kTcBK, y, bar);
+      }
+      __syncwarp();
       if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
@@ -346,8 +349,9 @@ __device__ void tma_warp(const TcParams& p, const TcSmem& sm, const CUtensorMap*
 }
 
 // ---------------------------------------------------------------- MMA warp
+// The whole warp walks the stages (warp-uniform descriptors); one elected lane
+// issues the MMAs and the commits that track them.
 __device__ void mma_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int lane) {
-  if (lane != 0) return;
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
   const uint32_t idesc = tc_idesc_f16(kTcBM, p.BN);
@@ -356,28 +360,32 @@ __device__ void mma_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base
   uint32_t ph = 0;
   for (int ui = 0; ui < n_my; ++ui) {
     const uint32_t a = static_cast<uint32_t>(ui) & 1u;
-    if (!tc_wait(sm, &sm.acce[a], ((static_cast<uint32_t>(ui) >> 1) & 1u) ^ 1u, p.status)) return;
+    if (!tc_wait_warp(sm, &sm.acce[a], ((static_cast<uint32_t>(ui) >> 1) & 1u) ^ 1u, p.status)) return;
     tc_fence_after();
     const uint32_t d_tmem = tmem_base + a * p.acc_stride;
     for (int st = 0; st < p.n_st; ++st) {
-      if (!tc_wait(sm, &sm.full[s], ph, p.status)) return;
+      if (!tc_wait_warp(sm, &sm.full[s], ph, p.status)) return;
       tc_fence_after();
       const int nk = 2 * st + 1 < p.n_ks ? 2 : 1;
       const uint32_t b0 = bst + static_cast<uint32_t>(s) * 2u * p.bstage_bytes;
       const uint32_t a0 = tmem_base + p.acol0 + static_cast<uint32_t>(s) * 64u;
-      for (int h = 0; h < nk; ++h) {
-        const uint64_t bdesc = smem_desc_k128(b0 + static_cast<uint32_t>(h) * p.bstage_bytes);
+      if (elect_one()) {
+        for (int h = 0; h < nk; ++h) {
+          const uint64_t bdesc = smem_desc_k128(b0 + static_cast<uint32_t>(h) * p.bstage_bytes);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          tc_mma_ts(d_tmem, a0 + 32u * h + 8u * i, bdesc + 2u * i, idesc, (st | h | i) != 0 ? 1u : 0u);
+          for (int i = 0; i < 4; ++i)
+            tc_mma_ts(d_tmem, a0 + 32u * h + 8u * i, bdesc + 2u * i, idesc, (st | h | i) != 0 ? 1u : 0u);
+        }
+        tc_commit(smem_addr(&sm.empty[s]));
       }
-      tc_commit(smem_addr(&sm.empty[s]));
+      __syncwarp();
       if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
       }
     }
-    tc_commit(smem_addr(&sm.accf[a]));
+    if (elect_one()) tc_commit(smem_addr(&sm.accf[a]));
+    __syncwarp();
   }
 }
 
