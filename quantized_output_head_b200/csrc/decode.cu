@@ -25,10 +25,11 @@
 // private shared-memory ring with cp.async (16 B per lane, L2 only) and waits
 // only on its own copies: no producer warp and no block-wide synchronisation.
 // After an m-tile the warp stores its 16 x nt partial logits in its own region
-// of a slot and arrives on reduced[r].  Warp 0, the epilogue, sums each slot's
-// regions in warp order (deterministic), pushes the logits into a running
-// log-sum-exp / argmax state, writes logits when asked, and frees the slot
-// (redfree[r]).  At the end every block writes one
+// of a slot and arrives on reduced[r].  Warps 0-1, the epilogue, each take half
+// of a slot's elements (two adjacent per lane), sum the warps' regions in warp
+// order (deterministic),
+// push the logits into running log-sum-exp / argmax states, write logits when
+// asked, and free the slot (redfree[r]).  At the end every block writes one
 // partial per token; the last block to finish (atomic ticket, no spinning)
 // merges them into LSE, argmax and CE.  Every mbarrier wait is bounded
 // (kWaitLimitNs); on expiry the block raises ARCHEAD_STATUS_WAIT_TIMEOUT and
@@ -42,14 +43,14 @@ namespace archead {
 
 namespace {
 
-constexpr int kEpiSlots = 4;     // kGroupTile x 16 logits / 32 lanes
 constexpr int kGroupTile = 8;    // m-tiles x tokens per partial-logit group (mg * nt)
 
 struct SmemView {
   uint8_t* rings;                // per compute warp: kRing slices
   float* part;                   // [slots][nw_work][mg][nt][16 rows] per-warp partial logits
-  uint64_t* reduced;             // [slots] compute warps -> epilogue warp
-  uint64_t* redfree;             // [slots] epilogue warp -> compute warps
+  uint64_t* reduced;             // [slots] compute warps -> epilogue warps
+  uint64_t* redfree;             // [slots] epilogue warps -> compute warps
+  float4* tokstate;              // [kEpiWarps][kDecodeTokens] per-warp token states of the block
   int* flags;                    // [0] abort
 };
 
@@ -59,7 +60,8 @@ __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams&
   v.part = reinterpret_cast<float*>(smem + p.ring_bytes);
   v.reduced = reinterpret_cast<uint64_t*>(v.part + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16);
   v.redfree = v.reduced + p.slots;
-  v.flags = reinterpret_cast<int*>(v.redfree + p.slots);
+  v.tokstate = reinterpret_cast<float4*>(v.redfree + p.slots);
+  v.flags = reinterpret_cast<int*>(v.tokstate + kEpiWarps * kDecodeTokens);
   return v;
 }
 
@@ -594,69 +596,80 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
   cp_async_wait_all();
 }
 
-// ------------------------------------------------------------ epilogue warp
-__device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int lane) {
+// ----------------------------------------------------------- epilogue warps
+// kEpiWarps warps share each group tile: lane l of epilogue warp ew holds the
+// two adjacent elements e, e + 1 with e = 2 (32 ew + l) of every group (same
+// token, rows r and r + 1), so a lane keeps one running state and reads each
+// warp's region with one 8-byte load.
+static_assert(kGroupTile * 16 == 64 * kEpiWarps, "two elements per epilogue lane");
+__device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int ew, int lane) {
   grid_dependency_wait();   // the workspace is shared with the previous launch
-  // Lane l, slot k holds element e = l + 32k of every group tile (fixed token).
-  LseState st[kEpiSlots];
-  int target[kEpiSlots];
-#pragma unroll
-  for (int k = 0; k < kEpiSlots; ++k) {
-    st[k] = lse_init();
-    const int e = lane + 32 * k;
-    target[k] = p.targets != nullptr ? p.targets[p.t0 + (e >> 4) % p.nt] : -1;
-  }
+  const int e = 2 * (32 * ew + lane);
+  LseState st = lse_init();
+  const int target = p.targets != nullptr ? p.targets[p.t0 + (e >> 4) % p.nt] : -1;
+  const int m = e / (16 * p.nt);            // m-tile of the group, token t, rows r, r + 1
+  const int t = (e >> 4) - m * p.nt, row = e & 15;
   const int ngroups = (n_my + p.mg - 1) >> p.mg_log2;
   for (int grp = 0; grp < ngroups; ++grp) {
     const int r = grp & (p.slots - 1);
     const bool ok = warp_wait(sv, &sv.reduced[r], (grp >> p.slots_log2) & 1, p.status, lane);
-    const float* part = sv.part + r * p.nw_work * (kGroupTile * 16);
+    const float* part = sv.part + r * p.nw_work * (kGroupTile * 16) + e;
     const int i0 = grp << p.mg_log2;
-#pragma unroll
-    for (int k = 0; k < kEpiSlots; ++k) {
-      // element e = (m * nt + t) * 16 + row of this group's tile
-      const int e = lane + 32 * k;
-      const int m = e / (16 * p.nt);
-      if (ok && m < p.mg && i0 + m < n_my) {
-        // warp-order sum with four independent chains
-        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-        int w = 0;
-        for (; w + 4 <= p.nw_work; w += 4) {
-          y0 += part[(w + 0) * (kGroupTile * 16) + e];
-          y1 += part[(w + 1) * (kGroupTile * 16) + e];
-          y2 += part[(w + 2) * (kGroupTile * 16) + e];
-          y3 += part[(w + 3) * (kGroupTile * 16) + e];
-        }
-        for (; w < p.nw_work; ++w) y0 += part[w * (kGroupTile * 16) + e];
-        const float y = (y0 + y1) + (y2 + y3);
-        const int row = e & 15, t = (e >> 4) - m * p.nt;
-        const int v = mtile_of(i0 + m) * kMT + row;
-        if (v < p.V) {
-          lse_push(st[k], y, v);
-          if (p.logits != nullptr) p.logits[static_cast<size_t>(p.t0 + t) * p.V + v] = y;
-          if (v == target[k]) p.tgt[p.t0 + t] = y;
-        }
+    if (ok && m < p.mg && i0 + m < n_my) {
+      // warp-order sums, two independent chains per element
+      float2 ya = make_float2(0.f, 0.f), yb = make_float2(0.f, 0.f);
+      int w = 0;
+      for (; w + 2 <= p.nw_work; w += 2) {
+        const float2 qa = *reinterpret_cast<const float2*>(part + (w + 0) * (kGroupTile * 16));
+        const float2 qb = *reinterpret_cast<const float2*>(part + (w + 1) * (kGroupTile * 16));
+        ya.x += qa.x;
+        ya.y += qa.y;
+        yb.x += qb.x;
+        yb.y += qb.y;
+      }
+      if (w < p.nw_work) {
+        const float2 qa = *reinterpret_cast<const float2*>(part + w * (kGroupTile * 16));
+        ya.x += qa.x;
+        ya.y += qa.y;
+      }
+      const float y0 = ya.x + yb.x, y1 = ya.y + yb.y;
+      const int v = mtile_of(i0 + m) * kMT + row;
+      if (v < p.V) {
+        lse_push(st, y0, v);
+        if (p.logits != nullptr) p.logits[static_cast<size_t>(p.t0 + t) * p.V + v] = y0;
+        if (v == target) p.tgt[p.t0 + t] = y0;
+      }
+      if (v + 1 < p.V) {
+        lse_push(st, y1, v + 1);
+        if (p.logits != nullptr) p.logits[static_cast<size_t>(p.t0 + t) * p.V + v + 1] = y1;
+        if (v + 1 == target) p.tgt[p.t0 + t] = y1;
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&sv.redfree[r]));
   }
-  // Block partial per token: the 16 lanes of half-warp h in slot k hold
-  // element rows of token ((32k + 16h) / 16) mod nt; merge per half-warp,
-  // then gather the half-warps of each token through shared memory order.
+  // Per token: merge each octet of lanes (16 rows of one token); octet
+  // q = 4 ew + (lane >> 3) carries token q mod nt.  Each warp leaves one state
+  // per token in shared memory; warp 0 merges them in warp order.
 #pragma unroll
-  for (int k = 0; k < kEpiSlots; ++k) {
-#pragma unroll
-    for (int m = 8; m >= 1; m >>= 1) st[k] = lse_merge(st[k], lse_shfl_xor(st[k], m));
-  }
-  for (int t = 0; t < p.nt; ++t) {
-    // half-warp q = 2k + (lane >> 4) carries token q mod nt
+  for (int o = 4; o >= 1; o >>= 1) st = lse_merge(st, lse_shfl_xor(st, o));
+  for (int tt = 0; tt < p.nt; ++tt) {
     LseState a = lse_init();
 #pragma unroll
-    for (int k = 0; k < kEpiSlots; ++k) {
-      const LseState lo = lse_shfl_idx(st[k], 0), hi = lse_shfl_idx(st[k], 16);
-      if ((2 * k) % p.nt == t) a = lse_merge(a, lo);
-      if ((2 * k + 1) % p.nt == t) a = lse_merge(a, hi);
+    for (int oc = 0; oc < 4; ++oc) {
+      const LseState b = lse_shfl_idx(st, 8 * oc);
+      if ((4 * ew + oc) % p.nt == tt) a = lse_merge(a, b);
+    }
+    if (lane == 0) sv.tokstate[ew * kDecodeTokens + tt] = make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
+  }
+  named_bar_sync(1, kEpiWarps * 32);
+  if (ew != 0) return;
+  for (int t = 0; t < p.nt; ++t) {
+    LseState a = lse_init();
+#pragma unroll
+    for (int w = 0; w < kEpiWarps; ++w) {
+      const float4 q = sv.tokstate[w * kDecodeTokens + t];
+      a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
     }
     if (lane == 0)
       p.partials[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] =
@@ -706,18 +719,18 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
   if (threadIdx.x == 0) {
     for (int r = 0; r < p.slots; ++r) {
       mbar_init(smem_addr(&sv.reduced[r]), p.nw_work);
-      mbar_init(smem_addr(&sv.redfree[r]), 1);
+      mbar_init(smem_addr(&sv.redfree[r]), kEpiWarps);
     }
     sv.flags[0] = 0;
     mbar_fence_init();
   }
   __syncthreads();
 
-  if (warp == 0) {
-    epilogue_warp(p, sv, n_my, lane);
+  if (warp < kEpiWarps) {
+    epilogue_warp(p, sv, n_my, warp, lane);
     return;
   }
-  const int cw = warp - 1;
+  const int cw = warp - kEpiWarps;
   if (cw < p.nw_res) {
     residual_warp<G>(p, sv, n_my, cw, cw, lane);
   } else if (cw < p.nw_res + p.nw_L) {
@@ -742,7 +755,7 @@ void decode_smem_plan(DecodeParams& p, int g_steps) {
 
 size_t decode_smem_bytes(const DecodeParams& p) {
   return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16 * 4 +
-         static_cast<size_t>(2) * p.slots * 8 + 16;
+         static_cast<size_t>(2) * p.slots * 8 + kEpiWarps * kDecodeTokens * 16 + 16;
 }
 
 namespace {
@@ -769,7 +782,7 @@ cudaError_t decode_set_attributes(int g_steps, size_t smem) {
 cudaError_t launch_decode(int g_steps, const DecodeParams& p, int grid, size_t smem, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3((1 + p.nw_work) * 32);
+  cfg.blockDim = dim3((kEpiWarps + p.nw_work) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

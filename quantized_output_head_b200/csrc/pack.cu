@@ -138,7 +138,7 @@ bool plan_decode(archead_handle* h, int smem_optin) {
   const int nw_L = (L.n_L + kCL - 1) / kCL;
   const int nw_A = (L.n_A + kCA - 1) / kCA;
   const int nw_work = nw_res + nw_L + nw_A;
-  if (1 + nw_work > kMaxDecodeWarps) return false;
+  if (kEpiWarps + nw_work > kMaxDecodeWarps) return false;
   // The rings and slots of the widest launch (8 tokens) must fit.
   DecodeParams dp{};
   dp.nw_res = nw_res;

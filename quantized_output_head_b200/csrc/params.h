@@ -11,6 +11,7 @@ constexpr int kCRes = 4;
 constexpr int kCL = 2;
 constexpr int kCA = 2;
 constexpr int kMaxDecodeWarps = 24;      // launch bound of the decode kernel
+constexpr int kEpiWarps = 2;             // decode epilogue warps (share each group of partial logits)
 constexpr int kDecodeTokens = 8;         // N of one m16n8k16 fragment
 constexpr int kRing = 4;                 // m-tiles in flight per compute warp
 // h is scaled per token by 2^(kScaleExp - E_t), E_t the binary exponent of
