@@ -415,6 +415,36 @@ __device__ __forceinline__ void issue_core(uint32_t dst, const uint8_t* g_nib, c
   if (sl_lane) cp_async16(dst + kCL * (kLNibChunkBytes + kLHiChunkBytes), g_sl);
 }
 
+// One core chunk (4 k16 steps, fp16 pair hi + lo of z) of one m-tile slot into acc.
+__device__ __forceinline__ void core_chunk(const uint8_t* slot, int c, int lane, const uint32_t (&zf)[kCL][4][2][2],
+                                           float (&acc)[4]) {
+  const uint4 nib = *reinterpret_cast<const uint4*>(slot + c * kLNibChunkBytes + lane * 16);
+  const uint32_t hb = *reinterpret_cast<const uint32_t*>(slot + kCL * kLNibChunkBytes + c * kLHiChunkBytes + lane * 4);
+  uint32_t a[4];
+  unpack_int5_biased<0>(nib.x, hb, a);
+  mma_f16_16816(acc, a, zf[c][0][0][0], zf[c][0][0][1]);
+  mma_f16_16816(acc, a, zf[c][0][1][0], zf[c][0][1][1]);
+  unpack_int5_biased<1>(nib.y, hb, a);
+  mma_f16_16816(acc, a, zf[c][1][0][0], zf[c][1][0][1]);
+  mma_f16_16816(acc, a, zf[c][1][1][0], zf[c][1][1][1]);
+  unpack_int5_biased<2>(nib.z, hb, a);
+  mma_f16_16816(acc, a, zf[c][2][0][0], zf[c][2][0][1]);
+  mma_f16_16816(acc, a, zf[c][2][1][0], zf[c][2][1][1]);
+  unpack_int5_biased<3>(nib.w, hb, a);
+  mma_f16_16816(acc, a, zf[c][3][0][0], zf[c][3][0][1]);
+  mma_f16_16816(acc, a, zf[c][3][1][0], zf[c][3][1][1]);
+}
+
+// Row scale, constant part and token scale of a finished core tile.
+__device__ __forceinline__ void core_finish(const uint8_t* slot, int gr, float2 cbc, float2 unscale, float (&acc)[4]) {
+  const float2 sc = half2_bits_to_float2(
+      *reinterpret_cast<const uint32_t*>(slot + kCL * (kLNibChunkBytes + kLHiChunkBytes) + gr * 4));
+  acc[0] = (acc[0] - cbc.x) * (sc.x * unscale.x);
+  acc[1] = (acc[1] - cbc.y) * (sc.x * unscale.y);
+  acc[2] = (acc[2] - cbc.x) * (sc.y * unscale.x);
+  acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
+}
+
 __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wl, int cw, int lane) {
   const int gr = lane >> 2;
   const int chunk0 = wl * kCL;
@@ -460,7 +490,41 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
   const float2 unscale = column_pair(zs, lane);
 
   float* tile = nullptr;
-  for (int i = 0; i < n_my; ++i) {
+  int i = 0;
+  if (nch == kCL) {
+    // Pairs of m-tiles: two independent MMA chains interleave.
+    for (; i + 1 < n_my; i += 2) {
+      const uint32_t k = static_cast<uint32_t>(i) & (kRing - 1);   // even: k, k + 1 < kRing
+      const uint8_t* slot = ring + k * sbytes;
+      cp_async_wait<kRing - 2>();
+      __syncwarp();
+      float acc_a[4] = {0.f, 0.f, 0.f, 0.f};
+      float acc_b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < kCL; ++c) {
+        core_chunk(slot, c, lane, zf, acc_a);
+        core_chunk(slot + sbytes, c, lane, zf, acc_b);
+      }
+      core_finish(slot, gr, cbc, unscale, acc_a);
+      core_finish(slot + sbytes, gr, cbc, unscale, acc_b);
+      __syncwarp();   // every lane is done reading both slots
+      if (i + kRing < n_my) issue_core(ring_s + k * sbytes, g_nib, g_hi, g_sl, nch, hi_lane, sl_lane);
+      cp_async_commit();
+      if (i + 1 + kRing < n_my)
+        issue_core(ring_s + (k + 1) * sbytes, g_nib + stride, g_hi + stride, g_sl + stride, nch, hi_lane, sl_lane);
+      cp_async_commit();
+      g_nib += 2 * stride;
+      g_hi += 2 * stride;
+      g_sl += 2 * stride;
+      if ((i & (p.mg - 1)) == 0) tile = group_begin(sv, p, i, cw, lane);
+      store_partial(tile, p, i, lane, acc_a);
+      group_end(sv, p, i, n_my, lane);
+      if (((i + 1) & (p.mg - 1)) == 0) tile = group_begin(sv, p, i + 1, cw, lane);
+      store_partial(tile, p, i + 1, lane, acc_b);
+      group_end(sv, p, i + 1, n_my, lane);
+    }
+  }
+  for (; i < n_my; ++i) {
     if ((i & (p.mg - 1)) == 0) tile = group_begin(sv, p, i, cw, lane);
     const uint32_t k = static_cast<uint32_t>(i) & (kRing - 1);
     const uint8_t* slot = ring + k * sbytes;
@@ -468,32 +532,9 @@ __device__ void core_warp(const DecodeParams& p, const SmemView& sv, int n_my, i
     __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < kCL; ++c) {
-      if (c < nch) {
-        const uint4 nib = *reinterpret_cast<const uint4*>(slot + c * kLNibChunkBytes + lane * 16);
-        const uint32_t hb =
-            *reinterpret_cast<const uint32_t*>(slot + kCL * kLNibChunkBytes + c * kLHiChunkBytes + lane * 4);
-        uint32_t a[4];
-        unpack_int5_biased<0>(nib.x, hb, a);
-        mma_f16_16816(acc, a, zf[c][0][0][0], zf[c][0][0][1]);
-        mma_f16_16816(acc, a, zf[c][0][1][0], zf[c][0][1][1]);
-        unpack_int5_biased<1>(nib.y, hb, a);
-        mma_f16_16816(acc, a, zf[c][1][0][0], zf[c][1][0][1]);
-        mma_f16_16816(acc, a, zf[c][1][1][0], zf[c][1][1][1]);
-        unpack_int5_biased<2>(nib.z, hb, a);
-        mma_f16_16816(acc, a, zf[c][2][0][0], zf[c][2][0][1]);
-        mma_f16_16816(acc, a, zf[c][2][1][0], zf[c][2][1][1]);
-        unpack_int5_biased<3>(nib.w, hb, a);
-        mma_f16_16816(acc, a, zf[c][3][0][0], zf[c][3][0][1]);
-        mma_f16_16816(acc, a, zf[c][3][1][0], zf[c][3][1][1]);
-      }
-    }
-    const float2 sc = half2_bits_to_float2(
-        *reinterpret_cast<const uint32_t*>(slot + kCL * (kLNibChunkBytes + kLHiChunkBytes) + gr * 4));
-    acc[0] = (acc[0] - cbc.x) * (sc.x * unscale.x);
-    acc[1] = (acc[1] - cbc.y) * (sc.x * unscale.y);
-    acc[2] = (acc[2] - cbc.x) * (sc.y * unscale.x);
-    acc[3] = (acc[3] - cbc.y) * (sc.y * unscale.y);
+    for (int c = 0; c < kCL; ++c)
+      if (c < nch) core_chunk(slot, c, lane, zf, acc);
+    core_finish(slot, gr, cbc, unscale, acc);
     __syncwarp();
     if (i + kRing < n_my) issue_core(ring_s + k * sbytes, g_nib, g_hi, g_sl, nch, hi_lane, sl_lane);
     g_nib += stride;

@@ -169,7 +169,7 @@ SMALL = [
     (1000, 320, 32, 8, 64, 64, 3),       # ragged vocabulary tail (not a multiple of 16)
     (1003, 320, 100, 40, 16, 10, 9),     # ragged ranks, g = 16, g_B not a power of two, two launches
     (16, 64, 0, 0, 64, 1, 1),            # residual only, one m-tile
-    (47, 128, 64, 32, 128, 128, 17),     # three launches of <= 8 tokens
+    (47, 128, 64, 32, 128, 128, 17),     # one 128-row tile, mostly past the vocabulary (tensor-core path)
     (4099, 512, 64, 64, 256, 32, 8),     # group of 256 spans a whole residual warp
     (2048, 1024, 512, 64, 512, 128, 5),  # group larger than a warp's columns
 ]
@@ -190,16 +190,17 @@ def test_small_shapes(qoh, V, d, r_c, r_r, g, g_B, T):
     assert np.array_equal(am.cpu().numpy(), am2.cpu().numpy())
 
 
-# Calls of >= 9 tokens take the tensor-core kernel when g_B is a multiple of 64.
+# Calls of >= 13 tokens take the tensor-core kernel when g_B is a multiple of 64.
 SMALL_TC = [
     # V,    d,   r_c, r_r, g,   g_B, T
-    (1000, 320, 32, 8, 64, 64, 16),       # ragged vocabulary, one 32-column correction chunk
+    (1000, 320, 32, 8, 64, 64, 17),       # ragged vocabulary, one 32-column correction chunk
     (2000, 256, 0, 0, 16, 64, 33),        # residual only, g = 16, ragged token tile
     (1500, 512, 64, 0, 32, 64, 130),      # no correction, g = 32, two token tiles
     (4099, 512, 128, 64, 256, 128, 40),   # g = 256, last 128-row tile nearly empty
     (300, 128, 64, 32, 128, 128, 200),    # three 128-row tiles, the last partial
-    (777, 192, 64, 64, 64, 64, 9),        # fewest tokens of the tensor-core path, odd k-step count
-    (1003, 320, 100, 40, 16, 10, 20),     # g_B = 10: 9+ tokens through the decode kernel
+    (777, 192, 64, 64, 64, 64, 13),       # fewest tokens of the tensor-core path, odd k-step count
+    (777, 192, 64, 64, 64, 64, 12),       # most tokens of the decode kernel (two launches)
+    (1003, 320, 100, 40, 16, 10, 20),     # g_B = 10: 13+ tokens through the decode kernel
 ]
 
 
