@@ -51,6 +51,7 @@ struct SmemView {
   uint64_t* reduced;             // [slots] compute warps -> epilogue warps
   uint64_t* redfree;             // [slots] epilogue warps -> compute warps
   float4* tokstate;              // [kEpiWarps][kDecodeTokens] per-warp token states of the block
+  float* hmax;                   // [kMaxDecodeWarps][kDecodeTokens] max|h_t| over each residual warp's columns
   int* flags;                    // [0] abort
 };
 
@@ -61,7 +62,8 @@ __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams&
   v.reduced = reinterpret_cast<uint64_t*>(v.part + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16);
   v.redfree = v.reduced + p.slots;
   v.tokstate = reinterpret_cast<float4*>(v.redfree + p.slots);
-  v.flags = reinterpret_cast<int*>(v.tokstate + kEpiWarps * kDecodeTokens);
+  v.hmax = reinterpret_cast<float*>(v.tokstate + kEpiWarps * kDecodeTokens);
+  v.flags = reinterpret_cast<int*>(v.hmax + kMaxDecodeWarps * kDecodeTokens);
   return v;
 }
 
@@ -297,31 +299,53 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
   }
   g_codes += kRing * stride;
   g_scales += kRing * stride;
-  grid_dependency_wait();
+  // The residual warps read every column of h between them, so they find E_t
+  // (max|h_t| < 2^E_t, the same value the prologue computes) without waiting
+  // for the prologue: a max over each warp's columns, then over the warps.
   const bool tok = gr < p.nt;
-  float hs = 0.f;
-  if (tok) hs = ldexpf(1.f, kScaleExp - p.escale[p.t0 + gr]);
-  // fp16 h fragments of this warp's columns, and the constant-part sum of each
-  // local group for token gr.
-  uint32_t hf[kCRes][4][2];
-  float cg[kNG];
-#pragma unroll
-  for (int g = 0; g < kNG; ++g) cg[g] = 0.f;
   const uint16_t* hrow = p.hidden + static_cast<size_t>(p.t0 + (tok ? gr : 0)) * p.d;
+  uint32_t hf[kCRes][4][2];   // bf16 pairs of this warp's columns, then fp16 fragments
+  float mx = 0.f;
 #pragma unroll
   for (int c = 0; c < kCRes; ++c) {
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      uint32_t b[2] = {0u, 0u};
-      if (tok && c < rs.nchunks) {
-        const uint16_t* r = hrow + (rs.chunk0 + c) * kResChunkK + s * 16 + 2 * (lane & 3);
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const uint32_t bits = *reinterpret_cast<const uint32_t*>(r + 8 * j);
-          const float lo = __uint_as_float(bits << 16) * hs;
-          const float hi = __uint_as_float(bits & 0xFFFF0000u) * hs;
-          b[j] = pack_half2(lo, hi);
-        }
+      for (int j = 0; j < 2; ++j) {
+        uint32_t bits = 0u;
+        if (tok && c < rs.nchunks)
+          bits = *reinterpret_cast<const uint32_t*>(hrow + (rs.chunk0 + c) * kResChunkK + s * 16 + 2 * (lane & 3) + 8 * j);
+        hf[c][s][j] = bits;
+        mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(bits << 16)), fabsf(__uint_as_float(bits & 0xFFFF0000u))));
+      }
+    }
+  }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  if ((lane & 3) == 0) sv.hmax[wres * kDecodeTokens + gr] = mx;
+  named_bar_sync(2, p.nw_res * 32);
+  float hs = 0.f;
+  if (tok) {
+    float m = 0.f;
+    for (int w = 0; w < p.nw_res; ++w) m = fmaxf(m, sv.hmax[w * kDecodeTokens + gr]);
+    int E = 0;
+    frexpf(m, &E);
+    hs = ldexpf(1.f, kScaleExp - E);
+  }
+  // fp16 h fragments of this warp's columns, and the constant-part sum of each
+  // local group for token gr.
+  float cg[kNG];
+#pragma unroll
+  for (int g = 0; g < kNG; ++g) cg[g] = 0.f;
+#pragma unroll
+  for (int c = 0; c < kCRes; ++c) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      uint32_t b[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t bits = hf[c][s][j];
+        b[j] = pack_half2(__uint_as_float(bits << 16) * hs, __uint_as_float(bits & 0xFFFF0000u) * hs);
       }
       hf[c][s][0] = b[0];
       hf[c][s][1] = b[1];
@@ -644,7 +668,6 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
 // warp's region with one 8-byte load.
 static_assert(kGroupTile * 16 == 64 * kEpiWarps, "two elements per epilogue lane");
 __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int ew, int lane) {
-  grid_dependency_wait();   // the workspace is shared with the previous launch
   const int e = 2 * (32 * ew + lane);
   LseState st = lse_init();
   const int target = p.targets != nullptr ? p.targets[p.t0 + (e >> 4) % p.nt] : -1;
@@ -705,6 +728,9 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
   }
   named_bar_sync(1, kEpiWarps * 32);
   if (ew != 0) return;
+  // The prologue resets the completion ticket, and the previous launch on this
+  // workspace must be done with it: wait for the preceding grid here.
+  grid_dependency_wait();
   for (int t = 0; t < p.nt; ++t) {
     LseState a = lse_init();
 #pragma unroll
@@ -796,7 +822,8 @@ void decode_smem_plan(DecodeParams& p, int g_steps) {
 
 size_t decode_smem_bytes(const DecodeParams& p) {
   return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16 * 4 +
-         static_cast<size_t>(2) * p.slots * 8 + kEpiWarps * kDecodeTokens * 16 + 16;
+         static_cast<size_t>(2) * p.slots * 8 + kEpiWarps * kDecodeTokens * 16 + kMaxDecodeWarps * kDecodeTokens * 4 +
+         16;
 }
 
 namespace {
