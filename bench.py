@@ -73,6 +73,24 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def max_over_ranks(ms, device):
+    """The slowest rank's device time (ms): an all-reduce MAX over the process
+    group, or ms itself when there is one process."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_step, steps, ms):
+    """Whole-job tokens/s: every rank serves its own batch each step (replicas,
+    weak scaling); ms is the slowest rank's time for all steps."""
+    return world * tokens_per_step * steps / (ms / 1e3)
+
+
 def workload(cfg, T):
     wl = gen.WORKLOADS[cfg]
     T = wl.T if T is None else T
@@ -314,13 +332,9 @@ def main():
         ev1.record()
         torch.cuda.synchronize()
         barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_per_step = ms / args.steps
-    value = world * T * args.steps / (ms / 1e3)
+    value = job_throughput(world, T, args.steps, ms)
 
     # Dominant kernel (the vocabulary pass): CUDA events around it, recorded on
     # the call's stream by the library, over a second timed loop.

@@ -140,4 +140,5 @@ def test_forward_rejects_null_handle(qoh):
     assert L.archead_logits_lse_argmax(None, 4096, 1, None, 4096, 4096, None, 4096, 1 << 20, None) == \
         qoh.ARCHEAD_EINVAL
     assert L.archead_workspace_bytes(None, 4) == 0
+    assert L.archead_forward_kernel(None, 4) == -1
     assert L.archead_status_string(qoh.ARCHEAD_EUNSUP) == b"unsupported shape or device"

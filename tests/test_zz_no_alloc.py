@@ -20,13 +20,15 @@ from parity import check_argmax, check_lse_ce
 pytestmark = pytest.mark.gpu
 
 
-def test_static_entry_matches_workspace_entry_twice():
+@pytest.mark.parametrize("T", [5, 24])   # the decode kernel, then the tensor-core kernel
+def test_static_entry_matches_workspace_entry_twice(T):
     import quantized_output_head_b200 as qoh
     lib = qoh._lib
     shape = (1000, 256, 32, 8, 64, 64)
     comps = gen.random_components(gen.HeadShape(*shape), seed=2024)
-    h_bits, targets = gen.random_hidden(256, 5, seed=2025, V=shape[0])
+    h_bits, targets = gen.random_hidden(256, T, seed=2025, V=shape[0])
     head = qoh.PackedHead(*shape, comps)
+    assert head.forward_kernel(T) == ("decode" if T <= 8 else "tensor_core")
     hd = torch.from_numpy(h_bits.view(np.int16)).cuda()
     td = torch.from_numpy(targets).cuda()
     ref_lse, ref_am, ref_ce = head.lse_argmax(hd, td)
@@ -34,10 +36,10 @@ def test_static_entry_matches_workspace_entry_twice():
     tol = oracle.tolerance(h_bits, rowmax)
     stream = torch.cuda.current_stream().cuda_stream
     for _ in range(2):
-        lse = torch.full((5,), float("nan"), device="cuda")
-        am = torch.full((5,), -1, dtype=torch.int32, device="cuda")
-        ce = torch.full((5,), float("nan"), device="cuda")
-        rc = lib.archead_logits_lse_argmax_static(head.handle, hd.data_ptr(), 5, td.data_ptr(), lse.data_ptr(),
+        lse = torch.full((T,), float("nan"), device="cuda")
+        am = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+        ce = torch.full((T,), float("nan"), device="cuda")
+        rc = lib.archead_logits_lse_argmax_static(head.handle, hd.data_ptr(), T, td.data_ptr(), lse.data_ptr(),
                                                    am.data_ptr(), ce.data_ptr(), stream)
         assert rc == qoh.ARCHEAD_OK, lib.archead_status_string(rc)
         torch.cuda.synchronize()
