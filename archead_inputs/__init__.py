@@ -67,6 +67,15 @@ WORKLOADS: Dict[int, Workload] = {
 }
 SWEEP_T = (2, 8, 32, 64)   # config 3 uses the first T rows of its 64-row draw
 
+# The pages' storage-matched comparison heads at the Qwen3-8B shape, as shapes of
+# the same packed format: a plain group-INT4 head (no low-rank branches) whose
+# 16-column groups bring its bytes to ARCHead's, and the core + residual head
+# without the metric correction.
+BASELINE_SHAPES: Dict[str, HeadShape] = {
+    "naive-int4": HeadShape(151936, 4096, 0, 0, 16, 128),
+    "core-int4": HeadShape(151936, 4096, 512, 0, 128, 128),
+}
+
 # Scale magnitudes of the seeded components (standard deviations of the
 # half-normal draws).  Each branch then contributes a comparable share of every
 # head entry, so dropping any branch is visible.

@@ -21,6 +21,7 @@ bounded sample of vocabulary rows, scaled to the full head.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -58,6 +59,9 @@ def parse_args():
     ap.add_argument("--config", type=int, default=2, choices=sorted(OPS))
     ap.add_argument("--T", type=int, default=None, help="override the token count of the config")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", default="archead", choices=["archead", "naive-int4", "core-int4"],
+                    help="head format: ARCHead, or one of the pages' storage-matched comparison heads "
+                         "(Qwen-shaped configs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -91,15 +95,25 @@ def job_throughput(world, tokens_per_step, steps, ms):
     return world * tokens_per_step * steps / (ms / 1e3)
 
 
-def workload(cfg, T):
+def workload(cfg, T, variant="archead"):
+    """The config's workload; a --variant swaps in one of the storage-matched
+    comparison heads of the same (Qwen3-8B) shape."""
     wl = gen.WORKLOADS[cfg]
     T = wl.T if T is None else T
+    if variant != "archead":
+        base = gen.BASELINE_SHAPES[variant]
+        if (wl.shape.V, wl.shape.d) != (base.V, base.d):
+            raise SystemExit(f"--variant {variant} applies to the Qwen3-8B-shaped configs (2, 3, 5)")
+        wl = dataclasses.replace(wl, name=f"{wl.name} [{variant}]", shape=base)
     return wl, T
 
 
 def row_bytes(shape):
+    """Packed bytes per vocabulary row: INT5 core factor and its fp16 row scale,
+    INT4 residual and its fp16 group scales, INT8 correction factor and its
+    fp16 row scale (a rank-0 branch has no row scale to read)."""
     V, d, r_c, r_r, g, g_B = shape
-    return 5 * r_c / 8 + 2 + d / 2 + 2 * d / g + r_r + 2
+    return 5 * r_c / 8 + (2 if r_c else 0) + d / 2 + 2 * d / g + r_r + (2 if r_r else 0)
 
 
 def algorithmic(shape, T, op):
@@ -272,7 +286,7 @@ def cpu_baseline(cfg, wl, T, comps, h_bits):
 def main():
     args = parse_args()
     cfg = args.config
-    wl, T = workload(cfg, args.T)
+    wl, T = workload(cfg, args.T, args.variant)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

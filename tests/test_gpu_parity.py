@@ -141,6 +141,21 @@ def test_qwen_status_clean(qwen):
     assert head.status(head.workspace(1)) == 0
 
 
+@pytest.mark.parametrize("variant", sorted(gen.BASELINE_SHAPES))
+def test_qwen_storage_matched_baselines(qoh, variant):
+    """The pages' comparison heads (plain group-INT4; core + residual) on both kernels, every logit."""
+    shape = gen.BASELINE_SHAPES[variant]
+    comps = gen.draw_components(shape, 2)
+    head = qoh.PackedHead(*shape.as_tuple(), comps)
+    h_bits, _ = gen.draw_activations(shape.d, 20, shape.V, 3)
+    y, tol = _oracle(comps, shape.as_tuple(), h_bits)
+    for T in (1, 20):
+        assert head.forward_kernel(T) == ("decode" if T == 1 else "tensor_core")
+        lg, am = head.logits(_dev_hidden(h_bits[:T]))
+        check_logits(lg.cpu().numpy(), y[:T], tol[:T])
+        check_argmax(am.cpu().numpy(), y[:T], tol[:T])
+
+
 # ------------------------------------------------------------- config 4
 @pytest.fixture(scope="module")
 def gemma(qoh):
