@@ -190,6 +190,36 @@ ARCHEAD_API int archead_logits_lse_argmax_static(const archead_handle* handle, c
                                                  int32_t T, const int32_t* targets, float* lse,
                                                  int32_t* argmax, float* ce, archead_stream_t stream);
 
+/* Vocabulary shards (one process per GPU, each holding a contiguous range of
+ * vocabulary rows; R, B and their scales replicated).  The rows of Eq. 7 of
+ * §3.2 are independent, so a shard computes its logits alone and only the
+ * per-token softmax statistics cross GPUs.  (A library extension for
+ * vocabulary-parallel serving; the paper runs on one GPU.)
+ *
+ * archead_set_vocab_shard: this head holds global rows
+ *   [row_offset, row_offset + V) of a vocabulary of vocab_total rows.  After it,
+ *   argmax ids are global, target ids are global ids in [0, vocab_total) (others
+ *   raise ARCHEAD_STATUS_BAD_TARGET; a target in another shard is not an error),
+ *   and the forward entry points report over this shard's rows (CE is NaN when
+ *   the target is elsewhere).  EINVAL unless 0 <= row_offset and
+ *   row_offset + V <= vocab_total.
+ * archead_shard_partials: per token t, partials[4t .. 4t+3] = (log-sum-exp over
+ *   this shard's rows, the largest logit, the global row of its first
+ *   occurrence as int32 bits, the target logit or NaN when the target row is
+ *   in another shard or targets is NULL).  partials is device memory, 16-byte
+ *   aligned; same workspace and stream rules as archead_logits_lse_argmax.
+ * archead_merge_shards: partials of n_shards shards stacked [n_shards][T][4]
+ *   in increasing row order (an all-gather in rank order when ranks hold
+ *   increasing row ranges) -> LSE over all rows, first argmax, CE = LSE - the
+ *   target logit (NaN if no shard held the target).  Any output may be NULL,
+ *   not all three.  Device pointers; no workspace. */
+ARCHEAD_API int archead_set_vocab_shard(archead_handle* handle, int32_t row_offset, int32_t vocab_total);
+ARCHEAD_API int archead_shard_partials(const archead_handle* handle, const uint16_t* hidden, int32_t T,
+                                       const int32_t* targets, float* partials, void* workspace,
+                                       size_t workspace_bytes, archead_stream_t stream);
+ARCHEAD_API int archead_merge_shards(const float* partials, int32_t n_shards, int32_t T, float* lse,
+                                     int32_t* argmax, float* ce, archead_stream_t stream);
+
 /* Read (and with clear != 0, reset) the device status word of a workspace:
  * a bitwise OR of ARCHEAD_STATUS_* since the last clear.  Synchronises the
  * stream.  Returns ARCHEAD_ETIMEOUT if ARCHEAD_STATUS_WAIT_TIMEOUT is set. */

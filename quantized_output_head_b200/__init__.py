@@ -33,7 +33,7 @@ EXPORTED = (
     "archead_logits", "archead_logits_lse_argmax", "archead_host_workspace_bytes", "archead_lse_argmax_host",
     "archead_workspace_status", "archead_set_profile_events", "archead_free", "archead_last_cuda_error",
     "archead_status_string", "archead_static_workspace_capacity", "archead_logits_lse_argmax_static",
-    "archead_forward_kernel",
+    "archead_forward_kernel", "archead_set_vocab_shard", "archead_shard_partials", "archead_merge_shards",
 )
 
 
@@ -63,6 +63,9 @@ _sig = {
     "archead_static_workspace_capacity": (_sz, []),
     "archead_logits_lse_argmax_static": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "archead_forward_kernel": (ctypes.c_int, [_vp, _i32]),
+    "archead_set_vocab_shard": (ctypes.c_int, [_vp, _i32, _i32]),
+    "archead_shard_partials": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "archead_merge_shards": (ctypes.c_int, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "archead_free": (None, [_vp]),
     "archead_last_cuda_error": (ctypes.c_int, []),
     "archead_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -233,6 +236,28 @@ class PackedHead:
                "archead_lse_argmax_host")
         return lse, am, ce
 
+    # --------------------------------------------------- vocabulary shards
+    def set_vocab_shard(self, row_offset: int, vocab_total: int) -> None:
+        """This head holds global rows [row_offset, row_offset + V) of a
+        vocabulary of vocab_total rows: argmax and target ids become global."""
+        _check(_lib.archead_set_vocab_shard(self.handle, int(row_offset), int(vocab_total)),
+               "archead_set_vocab_shard")
+        self.row_offset, self.vocab_total = int(row_offset), int(vocab_total)
+
+    def shard_partials(self, hidden: torch.Tensor, targets: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Per-token softmax statistics of this shard: [T, 4] fp32 rows
+        (lse over the shard's rows, max logit, global argmax as int32 bits,
+        target logit or NaN)."""
+        _check_hidden(hidden, self.d)
+        T = int(hidden.shape[0])
+        if targets is not None:
+            targets = targets.to(device=self.device, dtype=torch.int32).contiguous()
+        out = torch.empty((T, 4), dtype=torch.float32, device=self.device)
+        ws = self.workspace(T)
+        _check(_lib.archead_shard_partials(self.handle, hidden.data_ptr(), T, _ptr(targets), out.data_ptr(),
+                                           ws.data_ptr(), ws.numel(), _stream_ptr(None)), "archead_shard_partials")
+        return out
+
     def forward_kernel(self, T: int) -> str:
         """'decode' or 'tensor_core': the kernel a call with T tokens runs on."""
         k = _lib.archead_forward_kernel(self.handle, int(T))
@@ -256,6 +281,54 @@ class PackedHead:
         if rc not in (ARCHEAD_OK, ARCHEAD_ETIMEOUT):
             _check(rc, "archead_workspace_status")
         return int(v.value)
+
+
+# ------------------------------------------------------- vocabulary shards
+def shard_rows(V: int, world: int, rank: int, tile: int = 128) -> Tuple[int, int]:
+    """Rows [v0, v1) of rank `rank` among `world` vocabulary shards: whole
+    128-row tiles split as evenly as possible, in rank order."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank must be in [0, world)")
+    tiles = -(-V // tile)
+    t0 = rank * tiles // world
+    t1 = (rank + 1) * tiles // world
+    return min(V, t0 * tile), min(V, t1 * tile)
+
+
+# Components indexed by vocabulary row (the rest, R, B and their scales, are
+# shared by every shard).
+_ROW_COMPONENTS = ("L", "s_L", "q", "s_res", "A", "s_A")
+
+
+def shard_components(comps: Dict[str, np.ndarray], v0: int, v1: int) -> Dict[str, np.ndarray]:
+    """The canonical components of rows [v0, v1) of a head."""
+    return {k: (np.ascontiguousarray(v[v0:v1]) if k in _ROW_COMPONENTS else v) for k, v in comps.items()}
+
+
+def gather_partials(parts: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather every rank's [T, 4] shard partials into [world, T, 4], in rank
+    order (the one cross-GPU exchange of a vocabulary-sharded head)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    bufs = [torch.empty_like(parts) for _ in range(world)]
+    dist.all_gather(bufs, parts.contiguous(), group=group)
+    return torch.stack(bufs)
+
+
+def merge_shards(parts: torch.Tensor):
+    """Fold [n_shards, T, 4] partials (increasing row order) into
+    (lse [T], argmax [T] int32, ce [T]); all on the partials' CUDA device."""
+    if parts.dim() != 3 or parts.shape[2] != 4 or parts.dtype != torch.float32 or not parts.is_cuda:
+        raise ValueError("parts must be a [n_shards, T, 4] float32 CUDA tensor")
+    parts = parts.contiguous()
+    n, T = int(parts.shape[0]), int(parts.shape[1])
+    lse = torch.empty(T, dtype=torch.float32, device=parts.device)
+    am = torch.empty(T, dtype=torch.int32, device=parts.device)
+    ce = torch.empty(T, dtype=torch.float32, device=parts.device)
+    with torch.cuda.device(parts.device):
+        _check(_lib.archead_merge_shards(parts.data_ptr(), n, T, lse.data_ptr(), am.data_ptr(), ce.data_ptr(),
+                                         _stream_ptr(None)), "archead_merge_shards")
+    return lse, am, ce
 
 
 def _check_hidden(hidden: torch.Tensor, d: int) -> None:

@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(256) act_prep_kernel(const ActParams p) {
   if (p.targets != nullptr && blockIdx.x == 0 && blockIdx.y == 0) {
     for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
       const int v = p.targets[t];
-      if (v < 0 || v >= p.V) atomicOr(p.status, static_cast<uint32_t>(ARCHEAD_STATUS_BAD_TARGET));
+      if (v < 0 || v >= p.v_total) atomicOr(p.status, static_cast<uint32_t>(ARCHEAD_STATUS_BAD_TARGET));
     }
   }
   // E_t of the tile's tokens: |bf16| orders like its bit pattern without the sign.

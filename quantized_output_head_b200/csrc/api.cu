@@ -28,7 +28,8 @@ int check_device(const archead_handle* h) {
 // Tensor-core path: activation operand, the tensor-core kernel, and the
 // per-token fold of its partials.
 int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const int32_t* targets, float* logits,
-               int32_t* argmax, float* lse, float* ce, uint8_t* wb, const WsLayout& w, cudaStream_t stream) {
+               int32_t* argmax, float* lse, float* ce, float4* shard_out, uint8_t* wb, const WsLayout& w,
+               cudaStream_t stream) {
   const Layout& L = h->L;
   const int Kc = tc_kc(L);
   uint32_t* status = reinterpret_cast<uint32_t*>(wb + w.status);
@@ -54,6 +55,7 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
   ap.Kc = Kc;
   ap.g_B = L.g_B;
   ap.V = L.V;
+  ap.v_total = h->v_total;
   ap.alpha = h->tc_alpha;
   ap.beta = h->tc_beta;
   ap.gamma = h->tc_gamma;
@@ -71,6 +73,7 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
   tp.status = status;
   tp.T = T;
   tp.V = L.V;
+  tp.row0 = h->row0;
   tp.n_nt = (T + kTcMaxBN - 1) / kTcMaxBN;
   const int per = (T + tp.n_nt - 1) / tp.n_nt;
   tp.BN = (per + 15) / 16 * 16;
@@ -113,18 +116,19 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
     e = cudaEventRecord(h->ev_after, stream);
     if (e != cudaSuccess) return set_cuda_error(e);
   }
-  if (argmax != nullptr || lse != nullptr || ce != nullptr) {
-    e = launch_tc_merge(partials, tp.n_mt128, T, targets, tgt, L.V, lse, argmax, ce, stream);
+  if (argmax != nullptr || lse != nullptr || ce != nullptr || shard_out != nullptr) {
+    e = launch_tc_merge(partials, tp.n_mt128, T, targets, tgt, L.V, h->row0, lse, argmax, ce, shard_out, stream);
     if (e != cudaSuccess) return set_cuda_error(e);
   }
   return ARCHEAD_OK;
 }
 
 int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const int32_t* targets, float* logits,
-            int32_t* argmax, float* lse, float* ce, void* ws, size_t ws_bytes, cudaStream_t stream) {
+            int32_t* argmax, float* lse, float* ce, void* ws, size_t ws_bytes, cudaStream_t stream,
+            float4* shard_out = nullptr) {
   if (h == nullptr || hidden == nullptr || ws == nullptr) return ARCHEAD_EINVAL;
   if (T <= 0 || T > kMaxTokens) return ARCHEAD_EINVAL;
-  if (logits == nullptr && argmax == nullptr && lse == nullptr) return ARCHEAD_EINVAL;
+  if (logits == nullptr && argmax == nullptr && lse == nullptr && shard_out == nullptr) return ARCHEAD_EINVAL;
   if (ce != nullptr && targets == nullptr) return ARCHEAD_EINVAL;
   if (!aligned(hidden, 16) || !aligned(ws, 256)) return ARCHEAD_EALIGN;
   if (!aligned(logits, 4) || !aligned(argmax, 4) || !aligned(lse, 4) || !aligned(ce, 4) || !aligned(targets, 4))
@@ -135,7 +139,7 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   if (dc != ARCHEAD_OK) return dc;
 
   uint8_t* wb = static_cast<uint8_t*>(ws);
-  if (use_tc(*h, T)) return forward_tc(h, hidden, T, targets, logits, argmax, lse, ce, wb, w, stream);
+  if (use_tc(*h, T)) return forward_tc(h, hidden, T, targets, logits, argmax, lse, ce, shard_out, wb, w, stream);
   const Layout& L = h->L;
   uint32_t* counter = reinterpret_cast<uint32_t*>(wb + w.counter);
   uint32_t* status = reinterpret_cast<uint32_t*>(wb + w.status);
@@ -163,6 +167,7 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   pp.Kz = L.Kz;
   pp.g_B = L.g_B;
   pp.V = L.V;
+  pp.v_total = h->v_total;
   cudaError_t e = launch_prologue(pp, stream);
   if (e != cudaSuccess) return set_cuda_error(e);
 
@@ -183,6 +188,8 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   dp.status = status;
   dp.T = T;
   dp.V = L.V;
+  dp.row0 = h->row0;
+  dp.shard_out = shard_out;
   dp.d = L.d;
   dp.Kz = L.Kz;
   dp.rcp = L.rcp;
@@ -304,6 +311,33 @@ extern "C" ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle,
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return set_cuda_error(e);
   return ARCHEAD_OK;
+}
+
+extern "C" ARCHEAD_API int archead_set_vocab_shard(archead_handle* handle, int32_t row_offset, int32_t vocab_total) {
+  if (handle == nullptr || row_offset < 0 || vocab_total <= 0) return ARCHEAD_EINVAL;
+  if (static_cast<int64_t>(row_offset) + handle->L.V > vocab_total) return ARCHEAD_EINVAL;
+  handle->row0 = row_offset;
+  handle->v_total = vocab_total;
+  return ARCHEAD_OK;
+}
+
+extern "C" ARCHEAD_API int archead_shard_partials(const archead_handle* handle, const uint16_t* hidden, int32_t T,
+                                                  const int32_t* targets, float* partials, void* workspace,
+                                                  size_t workspace_bytes, archead_stream_t stream) {
+  if (partials == nullptr) return ARCHEAD_EINVAL;
+  if (!aligned(partials, 16)) return ARCHEAD_EALIGN;
+  return forward(handle, hidden, T, targets, nullptr, nullptr, nullptr, nullptr, workspace, workspace_bytes,
+                 reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<float4*>(partials));
+}
+
+extern "C" ARCHEAD_API int archead_merge_shards(const float* partials, int32_t n_shards, int32_t T, float* lse,
+                                                int32_t* argmax, float* ce, archead_stream_t stream) {
+  if (partials == nullptr || n_shards <= 0 || T <= 0 || T > kMaxTokens) return ARCHEAD_EINVAL;
+  if (lse == nullptr && argmax == nullptr && ce == nullptr) return ARCHEAD_EINVAL;
+  if (!aligned(partials, 16) || !aligned(lse, 4) || !aligned(argmax, 4) || !aligned(ce, 4)) return ARCHEAD_EALIGN;
+  const cudaError_t e = launch_shard_merge(reinterpret_cast<const float4*>(partials), n_shards, T, lse, argmax, ce,
+                                           reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
 }
 
 extern "C" ARCHEAD_API int archead_workspace_status(void* workspace, int clear, archead_stream_t stream,

@@ -670,7 +670,8 @@ static_assert(kGroupTile * 16 == 64 * kEpiWarps, "two elements per epilogue lane
 __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int ew, int lane) {
   const int e = 2 * (32 * ew + lane);
   LseState st = lse_init();
-  const int target = p.targets != nullptr ? p.targets[p.t0 + (e >> 4) % p.nt] : -1;
+  // target as a local row (a target in another vocabulary shard never matches)
+  const int target = p.targets != nullptr ? p.targets[p.t0 + (e >> 4) % p.nt] - p.row0 : -1;
   const int m = e / (16 * p.nt);            // m-tile of the group, token t, rows r, r + 1
   const int t = (e >> 4) - m * p.nt, row = e & 15;
   const int ngroups = (n_my + p.mg - 1) >> p.mg_log2;
@@ -763,12 +764,14 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     if (lane == 0) {
       const int tg = p.t0 + t;
       const float lse = a.m + logf(a.s);
+      const int gidx = a.idx + p.row0;
+      // target logit when the target row is one of this head's rows
+      const int tl = p.targets != nullptr ? p.targets[tg] - p.row0 : -1;
+      const float tgt = (tl >= 0 && tl < p.V) ? __ldcg(p.tgt + tg) : __int_as_float(0x7fc00000);
       if (p.lse != nullptr) p.lse[tg] = lse;
-      if (p.argmax != nullptr) p.argmax[tg] = a.idx;
-      if (p.ce != nullptr) {
-        const int target_id = p.targets[tg];
-        p.ce[tg] = (target_id >= 0 && target_id < p.V) ? lse - __ldcg(p.tgt + tg) : __int_as_float(0x7fc00000);
-      }
+      if (p.argmax != nullptr) p.argmax[tg] = gidx;
+      if (p.ce != nullptr) p.ce[tg] = lse - tgt;
+      if (p.shard_out != nullptr) p.shard_out[tg] = make_float4(lse, a.m, __int_as_float(gidx), tgt);
     }
   }
   if (lane == 0) *p.counter = 0u;

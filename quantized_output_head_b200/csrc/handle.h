@@ -21,6 +21,8 @@ struct archead_handle {
   // the shape can take it.
   bool tc_ok;
   int tc_alpha, tc_beta, tc_gamma, tc_mseg;
+  int row0;                 // vocabulary shard: global id of row 0, and the global vocabulary size
+  int v_total;
   cudaEvent_t ev_before;    // optional profiling events (not owned)
   cudaEvent_t ev_after;
 };
@@ -89,7 +91,10 @@ cudaError_t tc_set_attributes();
 cudaError_t tc_encode_xmap(CUtensorMap* map, const uint16_t* xop, int T, int Kc, int BN);
 cudaError_t launch_tc(const TcParams& p, const CUtensorMap& map, int grid, cudaStream_t stream);
 cudaError_t launch_tc_merge(const float4* partials, int n_mt128, int T, const int32_t* targets, const float* tgt,
-                            int V, float* lse, int32_t* argmax, float* ce, cudaStream_t stream);
+                            int V, int row0, float* lse, int32_t* argmax, float* ce, float4* shard_out,
+                            cudaStream_t stream);
+cudaError_t launch_shard_merge(const float4* parts, int n, int T, float* lse, int32_t* argmax, float* ce,
+                               cudaStream_t stream);
 
 // Thread-local record of the last CUDA error (api.cu).
 int set_cuda_error(cudaError_t e);

@@ -317,6 +317,8 @@ extern "C" ARCHEAD_API int archead_pack_load(const archead_desc* desc, const arc
     return ARCHEAD_EUNSUP;
   }
   h->e_B = row_norm_exponent(L, *comps);
+  h->row0 = 0;
+  h->v_total = L.V;
   plan_tc(h, *comps, optin);
   e = decode_set_attributes(L.g_steps, static_cast<size_t>(optin));
   if (e == cudaSuccess && h->tc_ok) e = tc_set_attributes();

@@ -35,6 +35,8 @@ struct DecodeParams {
   uint32_t* status;            // ARCHEAD_STATUS_* bits
   int32_t T, t0, nt;           // this launch covers tokens [t0, t0 + nt), nt <= 8
   int32_t V, d, Kz, rcp, e_B;
+  int32_t row0;                // global id of local row 0 (vocabulary shard); targets and argmax are global
+  float4* shard_out;           // [T] (lse, max, argmax bits, target logit or NaN) of this shard, or null
   int32_t n_res, n_L, n_A, n_mtiles, g_steps_log2;
   uint32_t off_res, off_Lnib, off_Lhi, off_A, off_sres, off_sL, off_sA, mblk_bytes;
   int32_t nw_res, nw_L, nw_A, nw_work;   // compute warps by role
@@ -58,6 +60,7 @@ struct PrologueParams {
   uint32_t* counter;
   uint32_t* status;
   int32_t T, d, rcp, rrp, Kz, g_B, V, e_B;
+  int32_t v_total;             // target ids are checked against [0, v_total)
 };
 
 }  // namespace archead

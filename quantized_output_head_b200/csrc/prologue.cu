@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(256) prologue_kernel(const PrologueParams p) {
   if (p.targets != nullptr) {
     for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < p.T; t += gridDim.x * blockDim.x) {
       const int v = p.targets[t];
-      if (v < 0 || v >= p.V) atomicOr(p.status, static_cast<uint32_t>(ARCHEAD_STATUS_BAD_TARGET));
+      if (v < 0 || v >= p.v_total) atomicOr(p.status, static_cast<uint32_t>(ARCHEAD_STATUS_BAD_TARGET));
     }
   }
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);

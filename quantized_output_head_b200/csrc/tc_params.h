@@ -33,6 +33,7 @@ struct TcParams {
   float* tgt;                 // [T] target logits
   uint32_t* status;
   int32_t T, V, BN, n_nt, n_mt128, n_units;
+  int32_t row0;                                // global id of local row 0 (vocabulary shard)
   int32_t n_res, n_L, n_A, n_mtiles, g_log2;   // chunks per segment; log2 of the residual group
   int32_t n_ks, ks_core, ks_corr;              // k-steps: total, first core, first correction
   int32_t n_st;                                // stages per unit: ceil(n_ks / 2)
@@ -54,6 +55,7 @@ struct ActParams {
   uint16_t* xop;              // [T, Kc] fp16 activation operand
   float* cinv;                // [T] 2^-c_t
   int32_t T, d, rcp, Kz, Kc, g_B, V;
+  int32_t v_total;                             // target ids are checked against [0, v_total)
   int32_t alpha, beta, gamma, mseg;
 };
 

@@ -442,7 +442,7 @@ __device__ void epilogue_warps(const TcParams& p, const TcSmem& sm, uint32_t tme
           for (int k = 0; k < 32; ++k)
             if (k < nrow) e += __expf(y[k] - m);
           if (p.targets != nullptr) {
-            const int tg = __ldg(p.targets + t) - v0;
+            const int tg = __ldg(p.targets + t) - p.row0 - v0;   // row within this warp's 32
             if (tg >= 0 && tg < nrow) p.tgt[t] = tile[lane * 33 + tg] * inv;
           }
           if (p.logits != nullptr) {
@@ -524,8 +524,8 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1)
 
 // Per-token fold of the partials: LSE, first argmax, cross-entropy.
 __global__ void __launch_bounds__(256) tc_merge_kernel(const float4* partials, int n_mt128, int T,
-                                                       const int32_t* targets, const float* tgt, int V, float* lse,
-                                                       int32_t* argmax, float* ce) {
+                                                       const int32_t* targets, const float* tgt, int V, int row0,
+                                                       float* lse, int32_t* argmax, float* ce, float4* shard_out) {
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   grid_dependency_wait();
   if (t >= T) return;
@@ -538,12 +538,14 @@ __global__ void __launch_bounds__(256) tc_merge_kernel(const float4* partials, i
   for (int o = 16; o >= 1; o >>= 1) a = lse_merge(a, lse_shfl_xor(a, o));
   if (lane == 0) {
     const float l = a.m + logf(a.s);
+    const int gidx = a.idx + row0;
+    // target logit when the target row is one of this head's rows
+    const int tl = targets != nullptr ? targets[t] - row0 : -1;
+    const float tv = (tl >= 0 && tl < V) ? tgt[t] : __int_as_float(0x7fc00000);
     if (lse != nullptr) lse[t] = l;
-    if (argmax != nullptr) argmax[t] = a.idx;
-    if (ce != nullptr) {
-      const int tg = targets[t];
-      ce[t] = (tg >= 0 && tg < V) ? l - tgt[t] : __int_as_float(0x7fc00000);
-    }
+    if (argmax != nullptr) argmax[t] = gidx;
+    if (ce != nullptr) ce[t] = l - tv;
+    if (shard_out != nullptr) shard_out[t] = make_float4(l, a.m, __int_as_float(gidx), tv);
   }
 }
 
@@ -635,8 +637,43 @@ cudaError_t launch_tc(const TcParams& p, const CUtensorMap& map, int grid, cudaS
 }
 
 cudaError_t launch_tc_merge(const float4* partials, int n_mt128, int T, const int32_t* targets, const float* tgt,
-                            int V, float* lse, int32_t* argmax, float* ce, cudaStream_t stream) {
-  tc_merge_kernel<<<(T + 7) / 8, 256, 0, stream>>>(partials, n_mt128, T, targets, tgt, V, lse, argmax, ce);
+                            int V, int row0, float* lse, int32_t* argmax, float* ce, float4* shard_out,
+                            cudaStream_t stream) {
+  tc_merge_kernel<<<(T + 7) / 8, 256, 0, stream>>>(partials, n_mt128, T, targets, tgt, V, row0, lse, argmax, ce,
+                                                   shard_out);
+  return cudaGetLastError();
+}
+
+// Per token, fold the states of n vocabulary shards (stacked in increasing row
+// order): LSE over all rows, the first maximum, and the target logit of the one
+// shard that holds the target.
+__global__ void __launch_bounds__(256) shard_merge_kernel(const float4* parts, int n, int T, float* lse,
+                                                          int32_t* argmax, float* ce) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  float M = -INFINITY;
+  for (int r = 0; r < n; ++r) M = fmaxf(M, parts[static_cast<size_t>(r) * T + t].x);
+  float s = 0.f, best = -INFINITY, tv = __int_as_float(0x7fc00000);
+  int idx = 0x7fffffff;
+  for (int r = 0; r < n; ++r) {
+    const float4 q = parts[static_cast<size_t>(r) * T + t];
+    s += expf(q.x - M);
+    const int qi = __float_as_int(q.z);
+    if (q.y > best || (q.y == best && qi < idx)) {
+      best = q.y;
+      idx = qi;
+    }
+    if (q.w == q.w) tv = q.w;   // not NaN: this shard holds the target row
+  }
+  const float l = M + logf(s);
+  if (lse != nullptr) lse[t] = l;
+  if (argmax != nullptr) argmax[t] = idx;
+  if (ce != nullptr) ce[t] = l - tv;
+}
+
+cudaError_t launch_shard_merge(const float4* parts, int n, int T, float* lse, int32_t* argmax, float* ce,
+                               cudaStream_t stream) {
+  shard_merge_kernel<<<(T + 255) / 256, 256, 0, stream>>>(parts, n, T, lse, argmax, ce);
   return cudaGetLastError();
 }
 

@@ -224,6 +224,39 @@ def test_small_shapes_many_tokens(qoh, V, d, r_c, r_r, g, g_B, T):
     test_small_shapes(qoh, V, d, r_c, r_r, g, g_B, T)
 
 
+@pytest.mark.parametrize("T", [5, 24])   # the decode kernel, then the tensor-core kernel
+def test_vocab_shards_merge_to_the_whole_head(qoh, T):
+    """Three vocabulary shards of one head, merged, against the unsharded head and the oracle."""
+    shape = (1000, 256, 32, 8, 64, 64)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=321)
+    h_bits, targets = gen.random_hidden(256, T, seed=322, V=shape[0])
+    hd, tg = _dev_hidden(h_bits), torch.from_numpy(targets)
+    y, tol = _oracle(comps, shape, h_bits)
+    whole = qoh.PackedHead(*shape, comps)
+    lse_w, am_w, ce_w = whole.lse_argmax(hd, tg)
+    parts = []
+    for r in range(3):
+        v0, v1 = qoh.shard_rows(shape[0], 3, r)
+        head = qoh.PackedHead(v1 - v0, *shape[1:], qoh.shard_components(comps, v0, v1))
+        head.set_vocab_shard(v0, shape[0])
+        p = head.shard_partials(hd, tg)
+        parts.append(p)
+        # the shard's own statistics: global argmax inside its rows, target logit only when it holds the target
+        pc = p.cpu().numpy()
+        am = pc[:, 2].view(np.int32)
+        assert np.all((am >= v0) & (am < v1))
+        inside = (targets >= v0) & (targets < v1)
+        assert np.all(np.isnan(pc[~inside, 3]))
+        np.testing.assert_allclose(pc[inside, 3], y[np.arange(T)[inside], targets[inside]],
+                                   atol=float(tol.max()), rtol=0)
+        np.testing.assert_allclose(pc[:, 1], y[:, v0:v1].max(axis=1), atol=float(tol.max()), rtol=0)
+    lse, am, ce = qoh.merge_shards(torch.stack(parts))
+    check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, targets)
+    check_argmax(am.cpu().numpy(), y, tol)
+    np.testing.assert_allclose(lse.cpu().numpy(), lse_w.cpu().numpy(), atol=float(tol.max()), rtol=0)
+    np.testing.assert_allclose(ce.cpu().numpy(), ce_w.cpu().numpy(), atol=2 * float(tol.max()), rtol=0)
+
+
 def test_zero_residual_and_correction_is_core_product(qoh):
     shape = (512, 256, 64, 32, 64, 64)
     comps = gen.random_components(gen.HeadShape(*shape), seed=99)
