@@ -59,6 +59,9 @@ def parse_args():
     ap.add_argument("--config", type=int, default=2, choices=sorted(OPS))
     ap.add_argument("--T", type=int, default=None, help="override the token count of the config")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--shard-vocab", action="store_true",
+                    help="vocabulary-sharded head: each rank holds a contiguous range of rows; one batch per step, "
+                         "per-token partials all-gathered and merged (strong scaling); LSE / argmax / CE out")
     ap.add_argument("--variant", default="archead", choices=["archead", "naive-int4", "core-int4"],
                     help="head format: ARCHead, or one of the pages' storage-matched comparison heads "
                          "(Qwen-shaped configs only)")
@@ -308,10 +311,20 @@ def main():
 
     shape = wl.shape
     sh = (shape.V, shape.d, shape.r_c, shape.r_r, shape.g, shape.g_B)
-    op = OPS[cfg]
+    op = dict(OPS[cfg])
     comps = gen.draw_components(shape, wl.head_seed_cfg)
     h_bits, targets = gen.draw_activations(shape.d, T, shape.V, cfg)
-    head = qoh.PackedHead(*sh, comps)
+    sharded = args.shard_vocab
+    if sharded:
+        # This rank's rows; logits stay on their shard, the merged outputs are LSE / argmax (/ CE).
+        v0, v1 = qoh.shard_rows(shape.V, world, rank)
+        sh_head = (v1 - v0,) + sh[1:]
+        head = qoh.PackedHead(*sh_head, qoh.shard_components(comps, v0, v1))
+        head.set_vocab_shard(v0, shape.V)
+        op.update(logits=False, lse=True)
+    else:
+        sh_head = sh
+        head = qoh.PackedHead(*sh, comps)
     dev = head.device
     hd = torch.from_numpy(h_bits.view(np.int16)).to(dev)
     td = torch.from_numpy(targets).to(dev)
@@ -322,6 +335,10 @@ def main():
     ws = head.workspace(T)
 
     def step():
+        if sharded:
+            parts = head.shard_partials(hd, td if op["ce"] else None)
+            allp = qoh.gather_partials(parts) if world > 1 else parts.unsqueeze(0)
+            return qoh.merge_shards(allp)
         if op["logits"]:
             head.logits_into(hd, logits, am, ws)
         else:
@@ -348,7 +365,8 @@ def main():
         barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_per_step = ms / args.steps
-    value = job_throughput(world, T, args.steps, ms)
+    # Replicas: every rank serves its own batch; sharded: all ranks serve one batch.
+    value = job_throughput(1 if sharded else world, T, args.steps, ms)
 
     # Dominant kernel (the vocabulary pass): CUDA events around it, recorded on
     # the call's stream by the library, over a second timed loop.
@@ -372,11 +390,11 @@ def main():
     hbm, bf16, bf16_sust, peak_src = peaks()
     if kind == "decode":
         Kz = -(-shape.r_c // 64) * 64 + -(-shape.r_r // 32) * 32
-        kbytes = vocab_pass_bytes_per_launch(sh, min(T, 8), op, Kz)
+        kbytes = vocab_pass_bytes_per_launch(sh_head, min(T, 8), op, Kz)
         kflops = None
         bound = "hbm"
     else:
-        kbytes, kflops = tc_pass_bytes_flops(sh, T, op)
+        kbytes, kflops = tc_pass_bytes_flops(sh_head, T, op)
         # The roofline that binds: HBM streaming of the packed head, or the
         # tensor cores (fp16 MMA runs at the bf16 rate; sustained peak, the
         # kernel is timed inside back-to-back calls).
@@ -387,7 +405,7 @@ def main():
         achieved, peak, unit = kflops / (kernel_ms / 1e3) / 1e12, bf16_sust, "TFLOP/s"
     traffic = recorded_traffic(kind, cfg, T)
     status = head.status(ws)
-    launches_per_step = (1 + n_launch) if kind == "decode" else 3
+    launches_per_step = ((1 + n_launch) if kind == "decode" else 3) + (1 if sharded else 0)
 
     out = None
     if rank == 0:
@@ -395,7 +413,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_baseline(cfg, wl, T, comps, h_bits)
         e2e = None
-        if not args.no_e2e:
+        if not args.no_e2e and not sharded:
             hh = torch.from_numpy(h_bits.view(np.int16)).pin_memory().numpy().view(np.uint16)
             th = torch.from_numpy(targets).pin_memory().numpy()
             outs = (torch.empty(T, dtype=torch.float32).pin_memory().numpy(),
@@ -414,7 +432,8 @@ def main():
         ab, af = algorithmic(sh, T, op)
         out = dict(
             metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
-            ms_per_step=ms_per_step, us_per_call=ms_per_step * 1e3, higher_is_better=True, scaling="weak",
+            ms_per_step=ms_per_step, us_per_call=ms_per_step * 1e3, higher_is_better=True,
+            scaling="strong" if sharded else "weak",
             vs_baseline=None, dtype="f16",
             dtype_detail=("f16 MMA (mma.sync) on exact int4/int5/int8 codes, fp32 accumulate, scales in fp32"
                           if kind == "decode" else
@@ -422,7 +441,9 @@ def main():
             data="synthetic (seeded, shapes of the pages' heads)",
             config=dict(workload=wl.name, V=shape.V, d=shape.d, r_c=shape.r_c, r_r=shape.r_r, g=shape.g,
                         g_B=shape.g_B, T=T, outputs=[k for k, v in op.items() if v],
-                        parallelism=f"replicas x{world}", l2="inputs larger than L2 (packed head 382 MB)"),
+                        parallelism=(f"vocabulary shards x{world} (rows {v0}-{v1} on rank 0)" if sharded
+                                     else f"replicas x{world}"),
+                        l2="inputs larger than L2 (packed head 382 MB)"),
             roofline=dict(bound=bound, achieved=achieved, peak=peak, unit=unit, frac=achieved / peak,
                           traffic=traffic, kernel=f"archead::{PROFILE_STEM[kind]}", kernel_us=kernel_ms * 1e3,
                           algorithmic_bytes_per_launch=kbytes, algorithmic_flops_per_launch=kflops,
