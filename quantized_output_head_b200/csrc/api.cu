@@ -1,7 +1,13 @@
 // Forward entry points of the C ABI (include/archead.h): argument checks,
-// workspace carving, and the launch sequence
-//   prologue (z_c, z_r)  ->  decode launches of <= 8 tokens each
-// on the caller's stream, with no host synchronisation.
+// workspace carving, and one of two launch sequences on the caller's stream,
+// with no host synchronisation:
+//   T < kTcMinTokens (or g_B not a multiple of 64):
+//     prologue (z_c, z_r, E_t)  ->  decode launches of <= 8 tokens each
+//   otherwise:
+//     activation operand [h | z_c | z_r]  ->  tensor-core pass  ->  per-token fold
+// Vocabulary shards (archead_set_vocab_shard) only shift row ids: the same
+// sequences run, and archead_shard_partials / archead_merge_shards carry the
+// per-token statistics across shards.
 #include <cuda_runtime.h>
 
 #include <cmath>

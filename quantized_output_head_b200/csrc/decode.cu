@@ -18,22 +18,25 @@
 // block + grid, ...): every compute warp owns a fixed slice of every m-tile
 // block, so it streams its own bytes:
 //   residual warps    16 k16 steps of d each; their fp16 h fragments stay in
-//                     registers for the whole launch
+//                     registers for the whole launch; between them they read
+//                     all of h, so they find each token's exponent E_t
+//                     themselves and start without waiting for the prologue
 //   core warps        kCL 64-column chunks of r_c' each
-//   correction warps  kCA 32-column chunks of r_r' each
-// Each compute warp prefetches its slice of the next kRing m-tiles into a
-// private shared-memory ring with cp.async (16 B per lane, L2 only) and waits
-// only on its own copies: no producer warp and no block-wide synchronisation.
-// After an m-tile the warp stores its 16 x nt partial logits in its own region
-// of a slot and arrives on reduced[r].  Warps 0-1, the epilogue, each take half
-// of a slot's elements (two adjacent per lane), sum the warps' regions in warp
-// order (deterministic),
-// push the logits into running log-sum-exp / argmax states, write logits when
-// asked, and free the slot (redfree[r]).  At the end every block writes one
-// partial per token; the last block to finish (atomic ticket, no spinning)
-// merges them into LSE, argmax and CE.  Every mbarrier wait is bounded
-// (kWaitLimitNs); on expiry the block raises ARCHEAD_STATUS_WAIT_TIMEOUT and
-// skips the remaining work.
+//   correction warps  kCA 32-column chunks of r_r' each (these and the core
+//                     warps wait for the prologue's z)
+// Residual and core warps take m-tiles in interleaved pairs (two independent
+// MMA chains).  Each compute warp prefetches its slice of the next kRing
+// m-tiles into a private shared-memory ring with cp.async (16 B per lane, L2
+// only) and waits only on its own copies: no producer warp and no block-wide
+// synchronisation.  After an m-tile the warp stores its 16 x nt partial logits
+// in its own region of a slot and arrives on reduced[r].  Warps 0-1, the
+// epilogue, each take half of a slot's elements (two adjacent per lane), sum
+// the warps' regions in warp order (deterministic), push the logits into
+// running log-sum-exp / argmax states, write logits when asked, and free the
+// slot (redfree[r]).  At the end every block writes one partial per token; the
+// last block to finish (atomic ticket, no spinning) merges them into LSE,
+// argmax and CE.  Every mbarrier wait is bounded (kWaitLimitNs); on expiry the
+// block raises ARCHEAD_STATUS_WAIT_TIMEOUT and skips the remaining work.
 #include <cuda_runtime.h>
 
 #include "device.cuh"
