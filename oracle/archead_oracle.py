@@ -228,6 +228,70 @@ def tolerance(h_bits: np.ndarray, rowmax: np.ndarray, rel: float = 2e-3) -> np.n
     return rel * hn[:, None] * rowmax[None, :]
 
 
+# ----------------------------------------------------------------- sampling
+# Not part of the paper: temperature sampling from the head's logits by the
+# Gumbel-max construction (argmax_v of y_v / tau + G_v with G_v independent
+# standard Gumbel draws samples v with probability softmax(y / tau)_v), the
+# definition behind the library's sampling entry point.  The draws come from
+# Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+# as 1, 2, 3", SC 2011), written here from that definition: ten rounds of two
+# 64 x 64 -> 128-bit multiplies with the published multipliers, the key bumped
+# by the published Weyl constants between rounds.
+_PHILOX_M0, _PHILOX_M1 = np.uint64(0xD2E7470EE14C6C93), np.uint64(0xCA5A826395121157)
+_PHILOX_W0, _PHILOX_W1 = np.uint64(0x9E3779B97F4A7C15), np.uint64(0xBB67AE8584CAA73B)
+_M32 = np.uint64(0xFFFFFFFF)
+
+
+def _mulhilo64(a: np.ndarray, b: np.uint64):
+    """High and low 64-bit words of a * b (uint64, elementwise), from 32-bit limbs."""
+    a = np.asarray(a, dtype=np.uint64)
+    a0, a1 = a & _M32, a >> np.uint64(32)
+    b0, b1 = np.uint64(int(b) & 0xFFFFFFFF), np.uint64(int(b) >> 32)
+    p00, p01, p10, p11 = a0 * b0, a0 * b1, a1 * b0, a1 * b1
+    mid = (p00 >> np.uint64(32)) + (p01 & _M32) + (p10 & _M32)
+    lo = (p00 & _M32) | ((mid & _M32) << np.uint64(32))
+    hi = p11 + (p01 >> np.uint64(32)) + (p10 >> np.uint64(32)) + (mid >> np.uint64(32))
+    return hi, lo
+
+
+def philox4x64(ctr0, ctr1, ctr2, ctr3, key0, key1, rounds: int = 10):
+    """Philox4x64-R on uint64 arrays (broadcast): returns the four output words."""
+    c = [np.asarray(x, dtype=np.uint64) for x in (ctr0, ctr1, ctr2, ctr3)]
+    k0, k1 = np.asarray(key0, dtype=np.uint64), np.asarray(key1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        for _ in range(rounds):
+            hi0, lo0 = _mulhilo64(c[0], _PHILOX_M0)
+            hi1, lo1 = _mulhilo64(c[2], _PHILOX_M1)
+            c = [hi1 ^ c[1] ^ k0, lo1, hi0 ^ c[3] ^ k1, lo0]
+            k0, k1 = k0 + _PHILOX_W0, k1 + _PHILOX_W1
+    return c
+
+
+def gumbel_noise(seed: int, token_ids: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """G[t, v] for global token ids and global vocabulary rows: word (v mod 4)
+    of Philox4x64-10 at counter (token, v div 4, 0, 0), key (seed, 0); its top 23
+    bits k give u = (k + 1/2) / 2^23 in (0, 1), and G = -log(-log(u))."""
+    t = np.asarray(token_ids, dtype=np.uint64)[:, None]
+    v = np.asarray(rows, dtype=np.uint64)[None, :]
+    w = philox4x64(t, v >> np.uint64(2), 0, 0, np.uint64(seed), 0)
+    sel = (v & np.uint64(3)).astype(np.int64)
+    word = np.choose(np.broadcast_to(sel, np.broadcast_shapes(t.shape, v.shape)),
+                     [np.broadcast_to(x, np.broadcast_shapes(t.shape, v.shape)) for x in w])
+    u = ((word >> np.uint64(41)).astype(np.float64) + 0.5) / 2.0 ** 23
+    return -np.log(-np.log(u))
+
+
+def sample_gumbel(y: np.ndarray, temperature: float, seed: int, offset: int, row0: int = 0):
+    """Sampled row per token (first maximum of y / tau + G) and the perturbed
+    values z = y / tau + G.  Token t uses counter offset + t; rows are global
+    (row0 + local index)."""
+    y = np.asarray(y, dtype=np.float64)
+    T, V = y.shape
+    g = gumbel_noise(seed, offset + np.arange(T, dtype=np.uint64), row0 + np.arange(V, dtype=np.uint64))
+    z = y / temperature + g
+    return row0 + np.argmax(z, axis=1), z
+
+
 # ------------------------------------------------------------- byte count
 def component_bytes(V: int, d: int, r_c: int, r_r: int, g: int, g_B: int) -> Dict[str, int]:
     """numel x element size of every registered packed tensor (Eq. 10); INT5 and

@@ -410,3 +410,43 @@ def test_planted_mapback_mistake_is_caught():
     Et = E @ T_p
     ev = np.sort(np.linalg.eigvalsh(Et.T @ Et))[::-1]
     assert wrong > np.sum(ev[r:]) * (1 + 1e-6)
+
+
+# ------------------------------------------------------------- sampling
+def test_philox4x64_matches_numpys_bit_generator():
+    """The oracle's Philox4x64-10 (written from its definition) against numpy's
+    Philox bit generator, which increments its 256-bit counter before each block."""
+    rng = np.random.default_rng(5)
+    for _ in range(6):
+        c0, c1, c2 = (int(x) for x in rng.integers(1, 2**63, size=3, dtype=np.int64))
+        k = rng.integers(0, 2**63, size=2, dtype=np.int64).astype(np.uint64) * np.uint64(2) + np.uint64(1)
+        bg = np.random.Philox(counter=np.array([c0 - 1, c1, c2, 0], dtype=np.uint64), key=k)
+        ref = bg.random_raw(4)
+        got = oracle.philox4x64(c0, c1, c2, 0, k[0], k[1])
+        assert [int(x) for x in got] == [int(x) for x in ref]
+
+
+def test_gumbel_max_draws_follow_softmax():
+    """40000 seeded draws over six logits: chi-square against softmax(y / tau)."""
+    y = np.array([0.3, -1.2, 2.0, 0.5, 0.0, 1.1])
+    tau, T = 0.8, 40000
+    idx, _ = oracle.sample_gumbel(np.tile(y, (T, 1)), tau, seed=1234567, offset=10)
+    p = np.exp(y / tau - (y / tau).max())
+    p /= p.sum()
+    counts = np.bincount(idx, minlength=y.size)
+    chi2 = float((((counts - T * p) ** 2) / (T * p)).sum())
+    assert chi2 < 20.5   # 99.9 % point of chi-square with 5 degrees of freedom
+
+
+def test_gumbel_sampling_invariants():
+    rng = np.random.default_rng(9)
+    y = rng.normal(size=(50, 300)) * 3
+    a, _ = oracle.sample_gumbel(y, 0.7, seed=42, offset=1000)
+    b, _ = oracle.sample_gumbel(y + 7.25, 0.7, seed=42, offset=1000)       # softmax is shift invariant
+    assert np.array_equal(a, b)
+    c, _ = oracle.sample_gumbel(y, 1e-4, seed=42, offset=1000)              # tau -> 0: the argmax
+    assert np.array_equal(c, np.argmax(y, axis=1))
+    d, _ = oracle.sample_gumbel(y[:, 100:], 0.7, seed=42, offset=1000, row0=100)   # global rows
+    assert np.all((d >= 100) & (d < 300))
+    g = oracle.gumbel_noise(42, np.arange(3, dtype=np.uint64), np.arange(8, dtype=np.uint64))
+    assert np.all(np.isfinite(g))
