@@ -190,6 +190,21 @@ ARCHEAD_API int archead_logits_lse_argmax_static(const archead_handle* handle, c
                                                  int32_t T, const int32_t* targets, float* lse,
                                                  int32_t* argmax, float* ce, archead_stream_t stream);
 
+/* Temperature sampling fused into the vocabulary pass (a consumer of the
+ * logits of Eq. 7 with no counterpart in the paper): for each token t,
+ *   sampled[t] = first argmax over rows v of  y[t,v] / temperature + G[t,v],
+ * G[t,v] = -log(-log(u)), u = (k + 1/2) / 2^23 with k the top 23 bits of word
+ * (v mod 4) of Philox4x64-10 (Salmon et al., SC 2011) at counter
+ * (offset + t, v / 4, 0, 0) and key (seed, 0); v is the global row (see the
+ * vocabulary shards below).  This draws v with probability
+ * softmax(y[t] / temperature)_v (Gumbel-max).  lse and argmax (of the
+ * untempered logits) may be NULL.  Runs on the decode kernel for every T;
+ * same workspace and stream rules as archead_logits_lse_argmax.  EINVAL unless
+ * 0 < temperature < inf. */
+ARCHEAD_API int archead_sample(const archead_handle* handle, const uint16_t* hidden, int32_t T, float temperature,
+                               uint64_t seed, uint64_t offset, int32_t* sampled, float* lse, int32_t* argmax,
+                               void* workspace, size_t workspace_bytes, archead_stream_t stream);
+
 /* Vocabulary shards (one process per GPU, each holding a contiguous range of
  * vocabulary rows; R, B and their scales replicated).  The rows of Eq. 7 of
  * §3.2 are independent, so a shard computes its logits alone and only the
@@ -201,8 +216,8 @@ ARCHEAD_API int archead_logits_lse_argmax_static(const archead_handle* handle, c
  *   argmax ids are global, target ids are global ids in [0, vocab_total) (others
  *   raise ARCHEAD_STATUS_BAD_TARGET; a target in another shard is not an error),
  *   and the forward entry points report over this shard's rows (CE is NaN when
- *   the target is elsewhere).  EINVAL unless 0 <= row_offset and
- *   row_offset + V <= vocab_total.
+ *   the target is elsewhere).  EINVAL unless 0 <= row_offset, row_offset is a
+ *   multiple of 16 and row_offset + V <= vocab_total.
  * archead_shard_partials: per token t, partials[4t .. 4t+3] = (log-sum-exp over
  *   this shard's rows, the largest logit, the global row of its first
  *   occurrence as int32 bits, the target logit or NaN when the target row is

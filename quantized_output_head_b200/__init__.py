@@ -34,6 +34,7 @@ EXPORTED = (
     "archead_workspace_status", "archead_set_profile_events", "archead_free", "archead_last_cuda_error",
     "archead_status_string", "archead_static_workspace_capacity", "archead_logits_lse_argmax_static",
     "archead_forward_kernel", "archead_set_vocab_shard", "archead_shard_partials", "archead_merge_shards",
+    "archead_sample",
 )
 
 
@@ -64,6 +65,8 @@ _sig = {
     "archead_logits_lse_argmax_static": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "archead_forward_kernel": (ctypes.c_int, [_vp, _i32]),
     "archead_set_vocab_shard": (ctypes.c_int, [_vp, _i32, _i32]),
+    "archead_sample": (ctypes.c_int, [_vp, _vp, _i32, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, _vp, _vp,
+                                      _vp, _vp, _sz, _vp]),
     "archead_shard_partials": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "archead_merge_shards": (ctypes.c_int, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "archead_free": (None, [_vp]),
@@ -235,6 +238,21 @@ class PackedHead:
                                             ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
                "archead_lse_argmax_host")
         return lse, am, ce
+
+    def sample(self, hidden: torch.Tensor, temperature: float, seed: int, offset: int = 0):
+        """Gumbel-max temperature sampling fused into the vocabulary pass: returns
+        (sampled [T] int32, lse [T], argmax [T]) of this head's rows; token t
+        draws its noise at Philox counter offset + t under key seed."""
+        _check_hidden(hidden, self.d)
+        T = int(hidden.shape[0])
+        out = torch.empty(T, dtype=torch.int32, device=self.device)
+        lse = torch.empty(T, dtype=torch.float32, device=self.device)
+        am = torch.empty(T, dtype=torch.int32, device=self.device)
+        ws = self.workspace(T)
+        _check(_lib.archead_sample(self.handle, hidden.data_ptr(), T, float(temperature), int(seed), int(offset),
+                                   out.data_ptr(), lse.data_ptr(), am.data_ptr(), ws.data_ptr(), ws.numel(),
+                                   _stream_ptr(None)), "archead_sample")
+        return out, lse, am
 
     # --------------------------------------------------- vocabulary shards
     def set_vocab_shard(self, row_offset: int, vocab_total: int) -> None:

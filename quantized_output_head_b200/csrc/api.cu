@@ -129,12 +129,20 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
   return ARCHEAD_OK;
 }
 
+// Sampling request of one call (decode kernel only).
+struct SampleArgs {
+  int32_t* sampled;
+  float inv_temp;
+  uint64_t seed, offset;
+};
+
 int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const int32_t* targets, float* logits,
             int32_t* argmax, float* lse, float* ce, void* ws, size_t ws_bytes, cudaStream_t stream,
-            float4* shard_out = nullptr) {
+            float4* shard_out = nullptr, const SampleArgs* sample = nullptr) {
   if (h == nullptr || hidden == nullptr || ws == nullptr) return ARCHEAD_EINVAL;
   if (T <= 0 || T > kMaxTokens) return ARCHEAD_EINVAL;
-  if (logits == nullptr && argmax == nullptr && lse == nullptr && shard_out == nullptr) return ARCHEAD_EINVAL;
+  if (logits == nullptr && argmax == nullptr && lse == nullptr && shard_out == nullptr && sample == nullptr)
+    return ARCHEAD_EINVAL;
   if (ce != nullptr && targets == nullptr) return ARCHEAD_EINVAL;
   if (!aligned(hidden, 16) || !aligned(ws, 256)) return ARCHEAD_EALIGN;
   if (!aligned(logits, 4) || !aligned(argmax, 4) || !aligned(lse, 4) || !aligned(ce, 4) || !aligned(targets, 4))
@@ -145,7 +153,8 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   if (dc != ARCHEAD_OK) return dc;
 
   uint8_t* wb = static_cast<uint8_t*>(ws);
-  if (use_tc(*h, T)) return forward_tc(h, hidden, T, targets, logits, argmax, lse, ce, shard_out, wb, w, stream);
+  if (sample == nullptr && use_tc(*h, T))
+    return forward_tc(h, hidden, T, targets, logits, argmax, lse, ce, shard_out, wb, w, stream);
   const Layout& L = h->L;
   uint32_t* counter = reinterpret_cast<uint32_t*>(wb + w.counter);
   uint32_t* status = reinterpret_cast<uint32_t*>(wb + w.status);
@@ -196,6 +205,13 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   dp.V = L.V;
   dp.row0 = h->row0;
   dp.shard_out = shard_out;
+  if (sample != nullptr) {
+    dp.sampled = sample->sampled;
+    dp.spart = reinterpret_cast<float2*>(wb + w.spart);
+    dp.inv_temp = sample->inv_temp;
+    dp.seed = sample->seed;
+    dp.ctr0 = sample->offset;
+  }
   dp.d = L.d;
   dp.Kz = L.Kz;
   dp.rcp = L.rcp;
@@ -319,8 +335,20 @@ extern "C" ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle,
   return ARCHEAD_OK;
 }
 
+extern "C" ARCHEAD_API int archead_sample(const archead_handle* handle, const uint16_t* hidden, int32_t T,
+                                          float temperature, uint64_t seed, uint64_t offset, int32_t* sampled,
+                                          float* lse, int32_t* argmax, void* workspace, size_t workspace_bytes,
+                                          archead_stream_t stream) {
+  if (sampled == nullptr || !(temperature > 0.f) || !(temperature < INFINITY)) return ARCHEAD_EINVAL;
+  if (!aligned(sampled, 4)) return ARCHEAD_EALIGN;
+  const SampleArgs sa{sampled, 1.f / temperature, seed, offset};
+  return forward(handle, hidden, T, nullptr, nullptr, argmax, lse, nullptr, workspace, workspace_bytes,
+                 reinterpret_cast<cudaStream_t>(stream), nullptr, &sa);
+}
+
 extern "C" ARCHEAD_API int archead_set_vocab_shard(archead_handle* handle, int32_t row_offset, int32_t vocab_total) {
   if (handle == nullptr || row_offset < 0 || vocab_total <= 0) return ARCHEAD_EINVAL;
+  if (row_offset % 16 != 0) return ARCHEAD_EINVAL;   // shards start on m-tile (16-row) boundaries
   if (static_cast<int64_t>(row_offset) + handle->L.V > vocab_total) return ARCHEAD_EINVAL;
   handle->row0 = row_offset;
   handle->v_total = vocab_total;

@@ -54,6 +54,7 @@ struct SmemView {
   uint64_t* reduced;             // [slots] compute warps -> epilogue warps
   uint64_t* redfree;             // [slots] epilogue warps -> compute warps
   float4* tokstate;              // [kEpiWarps][kDecodeTokens] per-warp token states of the block
+  float2* pickstate;             // [kEpiWarps][kDecodeTokens] per-warp sampling states of the block
   float* hmax;                   // [kMaxDecodeWarps][kDecodeTokens] max|h_t| over each residual warp's columns
   int* flags;                    // [0] abort
 };
@@ -65,7 +66,8 @@ __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams&
   v.reduced = reinterpret_cast<uint64_t*>(v.part + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16);
   v.redfree = v.reduced + p.slots;
   v.tokstate = reinterpret_cast<float4*>(v.redfree + p.slots);
-  v.hmax = reinterpret_cast<float*>(v.tokstate + kEpiWarps * kDecodeTokens);
+  v.pickstate = reinterpret_cast<float2*>(v.tokstate + kEpiWarps * kDecodeTokens);
+  v.hmax = reinterpret_cast<float*>(v.pickstate + kEpiWarps * kDecodeTokens);
   v.flags = reinterpret_cast<int*>(v.hmax + kMaxDecodeWarps * kDecodeTokens);
   return v;
 }
@@ -673,6 +675,7 @@ static_assert(kGroupTile * 16 == 64 * kEpiWarps, "two elements per epilogue lane
 __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int ew, int lane) {
   const int e = 2 * (32 * ew + lane);
   LseState st = lse_init();
+  PickState pk = pick_init();   // sampling: first maximum of y / tau + G
   // target as a local row (a target in another vocabulary shard never matches)
   const int target = p.targets != nullptr ? p.targets[p.t0 + (e >> 4) % p.nt] - p.row0 : -1;
   const int m = e / (16 * p.nt);            // m-tile of the group, token t, rows r, r + 1
@@ -702,6 +705,16 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
       }
       const float y0 = ya.x + yb.x, y1 = ya.y + yb.y;
       const int v = mtile_of(i0 + m) * kMT + row;
+      if (p.sampled != nullptr) {
+        // Rows v, v + 1 (global row even: shards start on 16-row boundaries)
+        // share one Philox block of four words.
+        const uint64_t vg = static_cast<uint64_t>(p.row0 + v);
+        uint64_t w[4];
+        philox4x64_10(p.ctr0 + static_cast<uint64_t>(p.t0 + t), vg >> 2, p.seed, w);
+        const bool upper = (vg & 2u) != 0;
+        if (v < p.V) pick_push(pk, fmaf(y0, p.inv_temp, gumbel_of(upper ? w[2] : w[0])), p.row0 + v);
+        if (v + 1 < p.V) pick_push(pk, fmaf(y1, p.inv_temp, gumbel_of(upper ? w[3] : w[1])), p.row0 + v + 1);
+      }
       if (v < p.V) {
         lse_push(st, y0, v);
         if (p.logits != nullptr) p.logits[static_cast<size_t>(p.t0 + t) * p.V + v] = y0;
@@ -720,15 +733,26 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
   // q = 4 ew + (lane >> 3) carries token q mod nt.  Each warp leaves one state
   // per token in shared memory; warp 0 merges them in warp order.
 #pragma unroll
-  for (int o = 4; o >= 1; o >>= 1) st = lse_merge(st, lse_shfl_xor(st, o));
+  for (int o = 4; o >= 1; o >>= 1) {
+    st = lse_merge(st, lse_shfl_xor(st, o));
+    pk = pick_merge(pk, pick_shfl_xor(pk, o));
+  }
   for (int tt = 0; tt < p.nt; ++tt) {
     LseState a = lse_init();
+    PickState b = pick_init();
 #pragma unroll
     for (int oc = 0; oc < 4; ++oc) {
-      const LseState b = lse_shfl_idx(st, 8 * oc);
-      if ((4 * ew + oc) % p.nt == tt) a = lse_merge(a, b);
+      const LseState q = lse_shfl_idx(st, 8 * oc);
+      const PickState r = pick_shfl_idx(pk, 8 * oc);
+      if ((4 * ew + oc) % p.nt == tt) {
+        a = lse_merge(a, q);
+        b = pick_merge(b, r);
+      }
     }
-    if (lane == 0) sv.tokstate[ew * kDecodeTokens + tt] = make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
+    if (lane == 0) {
+      sv.tokstate[ew * kDecodeTokens + tt] = make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
+      sv.pickstate[ew * kDecodeTokens + tt] = make_float2(b.z, __int_as_float(b.idx));
+    }
   }
   named_bar_sync(1, kEpiWarps * 32);
   if (ew != 0) return;
@@ -737,14 +761,20 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
   grid_dependency_wait();
   for (int t = 0; t < p.nt; ++t) {
     LseState a = lse_init();
+    PickState b = pick_init();
 #pragma unroll
     for (int w = 0; w < kEpiWarps; ++w) {
       const float4 q = sv.tokstate[w * kDecodeTokens + t];
       a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
+      const float2 r = sv.pickstate[w * kDecodeTokens + t];
+      b = pick_merge(b, PickState{r.x, __float_as_int(r.y)});
     }
-    if (lane == 0)
+    if (lane == 0) {
       p.partials[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] =
           make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
+      if (p.sampled != nullptr)
+        p.spart[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] = make_float2(b.z, __int_as_float(b.idx));
+    }
   }
   __threadfence();
   __syncwarp();
@@ -764,6 +794,17 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) a = lse_merge(a, lse_shfl_xor(a, m));
+    if (p.sampled != nullptr) {
+      const float2* sp = p.spart + static_cast<size_t>(p.t0 + t) * gridDim.x;
+      PickState b = pick_init();
+      for (int blk = lane; blk < static_cast<int>(gridDim.x); blk += 32) {
+        const float2 q = __ldcg(sp + blk);
+        b = pick_merge(b, PickState{q.x, __float_as_int(q.y)});
+      }
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) b = pick_merge(b, pick_shfl_xor(b, m));
+      if (lane == 0) p.sampled[p.t0 + t] = b.idx;
+    }
     if (lane == 0) {
       const int tg = p.t0 + t;
       const float lse = a.m + logf(a.s);
@@ -828,8 +869,8 @@ void decode_smem_plan(DecodeParams& p, int g_steps) {
 
 size_t decode_smem_bytes(const DecodeParams& p) {
   return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16 * 4 +
-         static_cast<size_t>(2) * p.slots * 8 + kEpiWarps * kDecodeTokens * 16 + kMaxDecodeWarps * kDecodeTokens * 4 +
-         16;
+         static_cast<size_t>(2) * p.slots * 8 + kEpiWarps * kDecodeTokens * (16 + 8) +
+         kMaxDecodeWarps * kDecodeTokens * 4 + 16;
 }
 
 namespace {

@@ -229,4 +229,60 @@ __device__ __forceinline__ LseState lse_shfl_xor(const LseState& a, int mask) {
   return o;
 }
 
+// --------------------------------------------------------------- sampling
+// Philox4x64-10 (Salmon, Moraes, Dror, Shaw, SC 2011) from its definition:
+// ten rounds of two 64 x 64 -> 128-bit multiplies, the key bumped by the Weyl
+// constants between rounds.  Counter (c0, c1, 0, 0), key (k0, 0).
+__device__ __forceinline__ void philox4x64_10(uint64_t c0, uint64_t c1, uint64_t k0, uint64_t (&out)[4]) {
+  constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+  uint64_t c2 = 0, c3 = 0, k1 = 0;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t hi0 = __umul64hi(M0, c0), lo0 = M0 * c0;
+    const uint64_t hi1 = __umul64hi(M1, c2), lo1 = M1 * c2;
+    c0 = hi1 ^ c1 ^ k0;
+    c1 = lo1;
+    c2 = hi0 ^ c3 ^ k1;
+    c3 = lo0;
+    k0 += W0;
+    k1 += W1;
+  }
+  out[0] = c0;
+  out[1] = c1;
+  out[2] = c2;
+  out[3] = c3;
+}
+
+// Standard Gumbel draw from the top 23 bits k of a word: u = (k + 1/2) / 2^23
+// (exact in fp32, strictly inside (0, 1)), G = -log(-log(u)).
+__device__ __forceinline__ float gumbel_of(uint64_t w) {
+  const float u = (static_cast<float>(static_cast<uint32_t>(w >> 41)) + 0.5f) * (1.0f / 8388608.0f);
+  return -logf(-logf(u));
+}
+
+// Running first maximum (value, row) of the perturbed logits y / tau + G.
+struct PickState {
+  float z;
+  int idx;
+};
+__device__ __forceinline__ PickState pick_init() { return PickState{-INFINITY, 0x7fffffff}; }
+__device__ __forceinline__ void pick_push(PickState& s, float z, int v) {
+  if (z > s.z) {
+    s.z = z;
+    s.idx = v;
+  }
+}
+__device__ __forceinline__ PickState pick_merge(const PickState& a, const PickState& b) {
+  if (a.z > b.z) return a;
+  if (b.z > a.z) return b;
+  return PickState{a.z, min(a.idx, b.idx)};
+}
+__device__ __forceinline__ PickState pick_shfl_xor(const PickState& a, int mask) {
+  return PickState{__shfl_xor_sync(0xffffffffu, a.z, mask), __shfl_xor_sync(0xffffffffu, a.idx, mask)};
+}
+__device__ __forceinline__ PickState pick_shfl_idx(const PickState& a, int src) {
+  return PickState{__shfl_sync(0xffffffffu, a.z, src), __shfl_sync(0xffffffffu, a.idx, src)};
+}
+
 }  // namespace archead

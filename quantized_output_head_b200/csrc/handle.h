@@ -37,12 +37,14 @@ inline bool use_tc(const archead_handle& h, int T) { return h.tc_ok && T >= kTcM
 inline int tc_kc(const Layout& L) { return L.d + L.rcp + static_cast<int>(round_up(L.rrp, 64)); }
 inline int tc_n_mt128(const Layout& L) { return (L.n_mtiles + 7) / 8; }
 
-// Workspace regions of one forward call with T tokens.
+// Workspace regions of one forward call with T tokens.  Both kernels' regions
+// start after the shared header and target logits, so one workspace of the
+// larger size serves whichever kernel a call takes.
 struct WsLayout {
-  size_t counter, status;
-  size_t escale, zhi, zlo, partials;   // decode path
-  size_t cinv, xop, tpartials;         // tensor-core path
-  size_t tgt, total;
+  size_t counter, status, tgt;
+  size_t escale, zhi, zlo, partials, spart;   // decode path
+  size_t cinv, xop, tpartials;                // tensor-core path
+  size_t total;
   // host-buffer form only
   size_t h_hidden, h_targets, h_lse, h_argmax, h_ce, host_total;
 };
@@ -50,22 +52,25 @@ struct WsLayout {
 inline WsLayout ws_layout(const archead_handle& h, int T) {
   WsLayout w{};
   const size_t t = static_cast<size_t>(T);
-  size_t o = 0;
   w.counter = 0;
   w.status = 4;
-  o = 256;
-  if (use_tc(h, T)) {
+  w.tgt = 256;
+  const size_t base = w.tgt + round_up(t * 4, 256);
+  size_t o = base;
+  w.escale = o;   o += round_up(t * 4, 256);
+  w.zhi = o;      o += round_up(t * h.L.Kz * 2, 256);
+  w.zlo = o;      o += round_up(t * h.L.Kz * 2, 256);
+  w.partials = o; o += round_up(t * h.grid * 16, 256);
+  w.spart = o;    o += round_up(t * h.grid * 8, 256);
+  const size_t dec_end = o;
+  o = base;
+  if (h.tc_ok && T >= kTcMinTokens) {
     w.cinv = o;      o += round_up(t * 4, 256);
     w.xop = o;       o += round_up(t * tc_kc(h.L) * 2, 256);
     w.tpartials = o; o += round_up(t * tc_n_mt128(h.L) * 16, 256);
-  } else {
-    w.escale = o;   o += round_up(t * 4, 256);
-    w.zhi = o;      o += round_up(t * h.L.Kz * 2, 256);
-    w.zlo = o;      o += round_up(t * h.L.Kz * 2, 256);
-    w.partials = o; o += round_up(t * h.grid * 16, 256);
   }
-  w.tgt = o;      o += round_up(t * 4, 256);
-  w.total = o;
+  w.total = o > dec_end ? o : dec_end;
+  o = w.total;
   w.h_hidden = o;  o += round_up(t * h.L.d * 2, 256);
   w.h_targets = o; o += round_up(t * 4, 256);
   w.h_lse = o;     o += round_up(t * 4, 256);

@@ -37,6 +37,12 @@ struct DecodeParams {
   int32_t V, d, Kz, rcp, e_B;
   int32_t row0;                // global id of local row 0 (vocabulary shard); targets and argmax are global
   float4* shard_out;           // [T] (lse, max, argmax bits, target logit or NaN) of this shard, or null
+  // Sampling (sampled != null): per token the first maximum of y / tau + G,
+  // G Gumbel draws from Philox4x64-10 keyed by seed at counter (ctr0 + t, row / 4).
+  int32_t* sampled;            // [T] or null
+  float2* spart;               // [T, gridDim.x]: (max of y / tau + G, row bits) per block
+  float inv_temp;
+  uint64_t seed, ctr0;
   int32_t n_res, n_L, n_A, n_mtiles, g_steps_log2;
   uint32_t off_res, off_Lnib, off_Lhi, off_A, off_sres, off_sL, off_sA, mblk_bytes;
   int32_t nw_res, nw_L, nw_A, nw_work;   // compute warps by role

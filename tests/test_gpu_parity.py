@@ -250,11 +250,73 @@ def test_vocab_shards_merge_to_the_whole_head(qoh, T):
         np.testing.assert_allclose(pc[inside, 3], y[np.arange(T)[inside], targets[inside]],
                                    atol=float(tol.max()), rtol=0)
         np.testing.assert_allclose(pc[:, 1], y[:, v0:v1].max(axis=1), atol=float(tol.max()), rtol=0)
+    with pytest.raises(qoh.ArcheadError):
+        head.set_vocab_shard(8, shape[0])               # shards start on 16-row boundaries
     lse, am, ce = qoh.merge_shards(torch.stack(parts))
     check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, targets)
     check_argmax(am.cpu().numpy(), y, tol)
     np.testing.assert_allclose(lse.cpu().numpy(), lse_w.cpu().numpy(), atol=float(tol.max()), rtol=0)
     np.testing.assert_allclose(ce.cpu().numpy(), ce_w.cpu().numpy(), atol=2 * float(tol.max()), rtol=0)
+
+
+def _check_samples(got, y, tol, temperature, seed, offset):
+    """Sampled ids against the oracle's Gumbel-max picks: equal, or the oracle's
+    perturbed values of the two rows within the logit tolerance / temperature
+    (plus the fp32 rounding of the Gumbel draw)."""
+    want, z = oracle.sample_gumbel(y, temperature, seed, offset)
+    for t, (a, b) in enumerate(zip(np.asarray(got), want)):
+        if a == b:
+            continue
+        assert 0 <= a < y.shape[1], f"sample[{t}] = {a} out of range"
+        gap = z[t, b] - z[t, a]
+        assert gap <= max(tol[t, a], tol[t, b]) / temperature + 1e-4, f"sample[{t}]: gpu {a}, oracle {b}, gap {gap:.3g}"
+
+
+@pytest.mark.parametrize("T", [5, 20])   # one and three decode launches
+def test_sampling_matches_oracle(qoh, T):
+    shape = (1000, 256, 32, 8, 64, 64)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=77)
+    h_bits, _ = gen.random_hidden(256, T, seed=78, V=shape[0])
+    head = qoh.PackedHead(*shape, comps)
+    y, tol = _oracle(comps, shape, h_bits)
+    for temperature, seed, offset in ((0.7, 12345, 0), (1.5, 2**40 + 3, 2**33 + 7)):
+        s1, lse, am = head.sample(_dev_hidden(h_bits), temperature, seed, offset)
+        _check_samples(s1.cpu().numpy(), y, tol, temperature, seed, offset)
+        check_lse_ce(lse.cpu().numpy(), None, y, tol)
+        check_argmax(am.cpu().numpy(), y, tol)
+        s2, _, _ = head.sample(_dev_hidden(h_bits), temperature, seed, offset)
+        assert torch.equal(s1, s2)                      # counter-based: reproducible
+    a, _, _ = head.sample(_dev_hidden(h_bits), 1.0, 1, 0)
+    b, _, _ = head.sample(_dev_hidden(h_bits), 1.0, 1, 1000)
+    assert not torch.equal(a, b)                        # another counter range draws other noise
+
+
+def test_sampling_frequencies_follow_softmax(qoh):
+    """One token repeated 16384 times over a 64-row head: chi-square of the GPU's
+    draws against softmax(y / tau) of the oracle's logits."""
+    shape = (64, 64, 16, 8, 16, 16)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=5)
+    h1, _ = gen.random_hidden(64, 1, seed=6, V=64)
+    y, _ = _oracle(comps, shape, h1)
+    tau, n = 0.9, 16384
+    head = qoh.PackedHead(*shape, comps)
+    got, _, _ = head.sample(_dev_hidden(np.repeat(h1, n, axis=0)), tau, seed=99, offset=0)
+    p = np.exp(y[0] / tau - (y[0] / tau).max())
+    p /= p.sum()
+    counts = np.bincount(got.cpu().numpy(), minlength=64)
+    keep = n * p >= 5                                   # chi-square cells with enough expected draws
+    rest = counts[~keep].sum(), n * p[~keep].sum()
+    obs = np.append(counts[keep], rest[0])
+    exp = np.append(n * p[keep], rest[1])
+    chi2 = float(((obs - exp) ** 2 / np.maximum(exp, 1e-12)).sum())
+    assert chi2 < 110.0   # well above the 99.9 % point for <= 64 cells
+
+
+def test_qwen_sampling_T1(qwen):
+    head = qwen["head"]
+    s, lse, am = head.sample(_dev_hidden(qwen["h1"]), 0.8, seed=2024, offset=5)
+    _check_samples(s.cpu().numpy(), qwen["y1"], qwen["tol1"], 0.8, 2024, 5)
+    check_argmax(am.cpu().numpy(), qwen["y1"], qwen["tol1"])
 
 
 def test_zero_residual_and_correction_is_core_product(qoh):
