@@ -62,6 +62,9 @@ def parse_args():
     ap.add_argument("--shard-vocab", action="store_true",
                     help="vocabulary-sharded head: each rank holds a contiguous range of rows; one batch per step, "
                          "per-token partials all-gathered and merged (strong scaling); LSE / argmax / CE out")
+    ap.add_argument("--sample", type=float, default=None, metavar="TEMPERATURE",
+                    help="measure the sampling entry point (Gumbel-max draw per token at this temperature, "
+                         "plus LSE and argmax) instead of the config's outputs")
     ap.add_argument("--variant", default="archead", choices=["archead", "naive-int4", "core-int4"],
                     help="head format: ARCHead, or one of the pages' storage-matched comparison heads "
                          "(Qwen-shaped configs only)")
@@ -315,6 +318,10 @@ def main():
     comps = gen.draw_components(shape, wl.head_seed_cfg)
     h_bits, targets = gen.draw_activations(shape.d, T, shape.V, cfg)
     sharded = args.shard_vocab
+    if args.sample is not None:
+        if sharded:
+            raise SystemExit("--sample and --shard-vocab do not combine")
+        op.update(logits=False, lse=True, argmax=True, ce=False)
     if sharded:
         # This rank's rows; logits stay on their shard, the merged outputs are LSE / argmax (/ CE).
         v0, v1 = qoh.shard_rows(shape.V, world, rank)
@@ -334,7 +341,12 @@ def main():
     ce = torch.empty(T, dtype=torch.float32, device=dev) if op["ce"] else None
     ws = head.workspace(T)
 
+    sample_offset = [0]
+
     def step():
+        if args.sample is not None:
+            sample_offset[0] += T   # a fresh counter range every step
+            return head.sample(hd, args.sample, seed=20261202, offset=sample_offset[0])
         if sharded:
             parts = head.shard_partials(hd, td if op["ce"] else None)
             allp = qoh.gather_partials(parts) if world > 1 else parts.unsqueeze(0)
@@ -370,7 +382,7 @@ def main():
 
     # Dominant kernel (the vocabulary pass): CUDA events around it, recorded on
     # the call's stream by the library, over a second timed loop.
-    kind = head.forward_kernel(T)
+    kind = "decode" if args.sample is not None else head.forward_kernel(T)
     n_launch = math.ceil(T / 8) if kind == "decode" else 1
     from cuda.bindings import runtime as cudart
     _, kb = cudart.cudaEventCreate()
@@ -413,7 +425,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_baseline(cfg, wl, T, comps, h_bits)
         e2e = None
-        if not args.no_e2e and not sharded:
+        if not args.no_e2e and not sharded and args.sample is None:
             hh = torch.from_numpy(h_bits.view(np.int16)).pin_memory().numpy().view(np.uint16)
             th = torch.from_numpy(targets).pin_memory().numpy()
             outs = (torch.empty(T, dtype=torch.float32).pin_memory().numpy(),
@@ -439,8 +451,9 @@ def main():
                           if kind == "decode" else
                           "f16 MMA (tcgen05) on fp16(scale*code) weights and fp16 [h|z], fp32 accumulate in TMEM"),
             data="synthetic (seeded, shapes of the pages' heads)",
-            config=dict(workload=wl.name, V=shape.V, d=shape.d, r_c=shape.r_c, r_r=shape.r_r, g=shape.g,
-                        g_B=shape.g_B, T=T, outputs=[k for k, v in op.items() if v],
+            config=dict(workload=wl.name + (f" [sampling, temperature {args.sample}]" if args.sample is not None else ""),
+                        V=shape.V, d=shape.d, r_c=shape.r_c, r_r=shape.r_r, g=shape.g,
+                        g_B=shape.g_B, T=T, outputs=[k for k, v in op.items() if v] + (["sample"] if args.sample is not None else []),
                         parallelism=(f"vocabulary shards x{world} (rows {v0}-{v1} on rank 0)" if sharded
                                      else f"replicas x{world}"),
                         l2="inputs larger than L2 (packed head 382 MB)"),
