@@ -363,26 +363,34 @@ __device__ void mma_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base
     if (!tc_wait_warp(sm, &sm.acce[a], ((static_cast<uint32_t>(ui) >> 1) & 1u) ^ 1u, p.status)) return;
     tc_fence_after();
     const uint32_t d_tmem = tmem_base + a * p.acc_stride;
+    // The wait for stage st + 1 sits between issuing stage st's MMAs and
+    // committing them, so its latency overlaps the tensor work.
+    if (!tc_wait_warp(sm, &sm.full[s], ph, p.status)) return;
     for (int st = 0; st < p.n_st; ++st) {
-      if (!tc_wait_warp(sm, &sm.full[s], ph, p.status)) return;
       tc_fence_after();
       const int nk = 2 * st + 1 < p.n_ks ? 2 : 1;
       const uint32_t b0 = bst + static_cast<uint32_t>(s) * 2u * p.bstage_bytes;
       const uint32_t a0 = tmem_base + p.acol0 + static_cast<uint32_t>(s) * 64u;
-      if (elect_one()) {
+      const bool leader = elect_one();
+      if (leader) {
         for (int h = 0; h < nk; ++h) {
           const uint64_t bdesc = smem_desc_k128(b0 + static_cast<uint32_t>(h) * p.bstage_bytes);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             tc_mma_ts(d_tmem, a0 + 32u * h + 8u * i, bdesc + 2u * i, idesc, (st | h | i) != 0 ? 1u : 0u);
         }
-        tc_commit(smem_addr(&sm.empty[s]));
       }
       __syncwarp();
+      const int sc = s;
       if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
       }
+      const bool more = st + 1 < p.n_st;
+      const bool ok = !more || tc_wait_warp(sm, &sm.full[s], ph, p.status);
+      if (leader) tc_commit(smem_addr(&sm.empty[sc]));
+      __syncwarp();
+      if (!ok) return;
     }
     if (elect_one()) tc_commit(smem_addr(&sm.accf[a]));
     __syncwarp();
