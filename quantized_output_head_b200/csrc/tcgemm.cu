@@ -76,16 +76,8 @@ __device__ __forceinline__ bool tc_aborted(const TcSmem& s) {
   return *reinterpret_cast<volatile int*>(s.abort_flag) != 0;
 }
 
-// Bounded wait of one thread; on expiry raises the timeout status.
-__device__ __forceinline__ bool tc_wait(const TcSmem& s, uint64_t* bar, uint32_t parity, uint32_t* status) {
-  if (tc_aborted(s)) return false;
-  if (mbar_wait(smem_addr(bar), parity)) return true;
-  *reinterpret_cast<volatile int*>(s.abort_flag) = 1;
-  atomicOr(status, static_cast<uint32_t>(ARCHEAD_STATUS_WAIT_TIMEOUT));
-  return false;
-}
-
-// Warp-uniform form.
+// Bounded, warp-uniform wait on an mbarrier phase; on expiry raises the
+// timeout status and the block's abort flag.
 __device__ __forceinline__ bool tc_wait_warp(const TcSmem& s, uint64_t* bar, uint32_t parity, uint32_t* status) {
   bool ok = true;
   if (tc_aborted(s)) ok = false;
