@@ -25,6 +25,9 @@ Readings of points the pages leave open (each also listed in the design notes):
     as printed); its group scales are fp16;
   * the "randomised" truncated SVD of Eq. 4 is replaced by the exact SVD that
     it approximates (§3.2, remark after the proof);
+  * a singular pair (u_i, v_i) is defined only up to a common sign; each is
+    taken with the first largest-magnitude entry of v_i positive, so the
+    quantised factors are a function of the head alone;
   * damping lambda = 1e-2 and metric power p = 0.75 unless given.
 
 Parity pins (tests/test_oracle_pins.py) tie every function here to something
@@ -118,8 +121,16 @@ def damped_metric(H: np.ndarray, lam: float, p: float):
 
 
 def truncated_svd(M: np.ndarray, r: int):
+    """Rank-r truncated SVD (Eckart-Young), singular values descending; each
+    pair's sign fixed so that the first largest-magnitude entry of the right
+    singular vector is positive (the pages leave the sign open)."""
     U, S, Vt = np.linalg.svd(M, full_matrices=False)
-    return U[:, :r], S[:r], Vt[:r]
+    U, S, Vt = U[:, :r].copy(), S[:r], Vt[:r].copy()
+    for i in range(Vt.shape[0]):
+        if Vt[i, np.argmax(np.abs(Vt[i]))] < 0:
+            U[:, i] = -U[:, i]
+            Vt[i] = -Vt[i]
+    return U, S, Vt
 
 
 def correction_factors(E: np.ndarray, T_p: np.ndarray, T_p_inv: np.ndarray, r_r: int):

@@ -113,6 +113,29 @@ def test_identity_metric_is_plain_truncated_svd():
     np.testing.assert_allclose(A @ B, E @ top @ top.T, atol=1e-9)
 
 
+def test_truncated_svd_sign_convention():
+    """Singular pairs are fixed up to a joint sign: with known singular vectors
+    whose largest entries are negative, the oracle returns them negated on
+    both sides (product unchanged, largest entry of each v_i positive)."""
+    rng = np.random.default_rng(12)
+    m, n, r = 40, 12, 4
+    U0, _ = np.linalg.qr(rng.standard_normal((m, n)))
+    V0, _ = np.linalg.qr(rng.standard_normal((n, n)))
+    for i in range(n):                          # make each column's largest entry negative
+        if V0[np.argmax(np.abs(V0[:, i])), i] > 0:
+            V0[:, i] = -V0[:, i]
+    s = np.array([9.0, 7.0, 5.0, 3.0] + [1.0 / (k + 2) for k in range(n - 4)])
+    M = (U0 * s) @ V0.T
+    U, S, Vt = oracle.truncated_svd(M, r)
+    np.testing.assert_allclose(S, s[:r], rtol=1e-12)
+    np.testing.assert_allclose(Vt, -V0[:, :r].T, atol=1e-10)
+    np.testing.assert_allclose(U, -U0[:, :r], atol=1e-10)
+    for i in range(r):
+        assert Vt[i, np.argmax(np.abs(Vt[i]))] > 0
+    # the sign choice leaves the best rank-r approximation unchanged
+    np.testing.assert_allclose((U * S) @ Vt, (U0[:, :r] * s[:r]) @ V0[:, :r].T, atol=1e-10)
+
+
 def _ey_case(seed=5, V=48, d=24, r=4):
     rng = np.random.default_rng(seed)
     H = _aniso(400, d, seed + 1)
