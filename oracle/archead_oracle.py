@@ -80,6 +80,8 @@ def quantize_symmetric(x: np.ndarray, bits: int, group: Optional[int]) -> Tuple[
     """
     qmin, qmax = QRANGE[bits]
     rows, cols = x.shape
+    if cols == 0:                # a rank-0 factor: no codes; its per-row scales are fp16(0) = 0
+        return np.zeros((rows, 0), dtype=np.int8), np.zeros((rows, 1 if group is None else 0), dtype=np.uint16)
     G = cols if group is None else group
     if cols % G:
         raise ValueError("group size must divide the row length")

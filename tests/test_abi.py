@@ -52,6 +52,39 @@ def test_library_exports_every_declared_symbol(qoh):
     assert sorted(qoh.EXPORTED) == names
 
 
+BUILD_HEADER = os.path.join(ROOT, "include", "archead_build.h")
+
+
+def test_builder_library_exports_every_declared_symbol(qoh):
+    import quantized_output_head_b200.builder as bld
+    text = open(BUILD_HEADER).read()
+    names = sorted(set(re.findall(r"ARCHEAD_API\s+[\w\s\*]*?\b(archead_\w+)\s*\(", text)))
+    assert "archead_build_head" in names
+    out = subprocess.run(["nm", "-D", "--defined-only", bld.BUILD_LIB_PATH], capture_output=True, text=True).stdout
+    assert sorted(set(re.findall(r"\bT (archead_\w+)", out))) == names
+    assert sorted(bld.EXPORTED_BUILD) == names
+
+
+def test_builder_argument_checks_need_no_gpu(qoh):
+    """Bad arguments are refused on the host, before any CUDA call."""
+    import ctypes as ct
+    import quantized_output_head_b200.builder as bld
+    lib = bld._blib
+    assert lib.archead_build_quantize(None, 4, 64, 4, 0, None, None, None) == -1
+    assert b"null" in lib.archead_build_last_error()
+    fake = ct.c_void_p(256)                  # never dereferenced: the checks fail first
+    assert lib.archead_build_quantize(fake, 4, 64, 6, 0, fake, fake, None) == -1
+    assert lib.archead_build_quantize(fake, 4, 64, 4, 24, fake, fake, None) == -1
+    assert lib.archead_build_metric(0, 16, fake, 0.01, 0.75, fake, fake, fake, 1 << 20, None) == -1
+    assert lib.archead_build_metric(64, 16, fake, -1.0, 0.75, fake, fake, fake, 1 << 20, None) == -1
+    bad = [qoh.ArcheadDesc(1024, 256, 300, 8, 64, 64),    # r_c > min(V, d)
+           qoh.ArcheadDesc(1024, 256, 32, 8, 48, 64),     # g does not divide d
+           qoh.ArcheadDesc(0, 256, 0, 0, 64, 64)]
+    for desc in bad:
+        assert lib.archead_build_workspace_bytes(ct.byref(desc), 4096) == 0
+        assert lib.archead_build_head(ct.byref(desc), fake, fake, 4096, 0.01, 0.75, None, fake, 1 << 20, None) == -1
+
+
 SHAPES = [
     (1024, 256, 32, 8, 64, 64),
     (151936, 4096, 512, 64, 128, 128),

@@ -1,0 +1,183 @@
+"""GPU construction of a packed head (libarchead_build.so) against the oracle's
+builder: the quantiser bit for bit, the damped metric T_p / T_p^-1 of Eq. 2,
+the correction factors of Eq. 4-5 from the oracle's own remainder E, and the
+whole of Algorithm 1 on the config-1 head and on a 4096 x 1024 head.
+
+Codes and scales are integer decisions taken in fp64 on both sides from values
+that agree to ~1e-12 relative, so they must be equal; the one exception
+accepted is a value the oracle itself places on a rounding boundary (a scale
+ratio within 1e-9 of an fp16 midpoint, a code ratio within 1e-6 of a
+half-integer), where either rounding is correct.
+"""
+import numpy as np
+import pytest
+import torch
+
+import archead_inputs as gen
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+QMAX = {4: 7, 5: 15, 8: 127}
+
+
+@pytest.fixture(scope="module")
+def bld():
+    import quantized_output_head_b200.builder as b
+    return b
+
+
+def _fp16_midpoint_tie(t: np.ndarray) -> np.ndarray:
+    """t (>= 0) lies within 1e-9 relative of the midpoint between two adjacent fp16 values."""
+    bits = oracle.fp16_encode(t).astype(np.int64)
+    f = oracle.fp16_decode(bits.astype(np.uint16))
+    nb = np.where(t >= f, bits + 1, np.maximum(bits - 1, 0)).astype(np.uint16)
+    mid = 0.5 * (f + oracle.fp16_decode(nb))
+    return np.abs(t - mid) <= 1e-9 * np.maximum(t, 1e-300)
+
+
+def assert_quantised_like_oracle(codes_g, scales_g, x, bits, group, what, max_ties=1e-4):
+    """GPU (codes, scale bits) against oracle.quantize_symmetric(x); x are the
+    oracle's unquantised values."""
+    codes_o, s_o = oracle.quantize_symmetric(x, bits, group)
+    codes_g = np.asarray(codes_g).reshape(codes_o.shape)
+    s_g = np.asarray(scales_g).view(np.uint16).reshape(s_o.shape)
+    rows, cols = x.shape
+    if cols == 0 or rows == 0:                   # an empty branch: zero scales, no codes
+        np.testing.assert_array_equal(s_g, s_o)
+        return
+    G = cols if group is None else group
+    ng = cols // G
+    amax = np.abs(x.reshape(rows, ng, G)).max(axis=2)
+    s_bad = s_g != s_o
+    if s_bad.any():
+        tie = _fp16_midpoint_tie(amax / QMAX[bits])
+        assert tie[s_bad].all(), f"{what}: {int((s_bad & ~tie).sum())} scales differ away from a rounding tie"
+    exempt = np.repeat(s_bad, G, axis=1).reshape(rows, cols)
+    c_bad = (codes_g != codes_o) & ~exempt
+    if c_bad.any():
+        s = np.repeat(oracle.fp16_decode(s_o).reshape(rows, ng), G, axis=1)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ratio = np.where(s > 0, x / s, 0.0)
+        near = np.abs(np.abs(ratio - np.floor(ratio)) - 0.5) <= 1e-6
+        diff = np.abs(codes_g.astype(np.int32) - codes_o.astype(np.int32))
+        ok = near & (diff == 1)
+        assert ok[c_bad].all(), f"{what}: {int((c_bad & ~ok).sum())} codes differ away from a rounding tie"
+    n_ties = int(s_bad.sum()) * G + int(c_bad.sum())
+    assert n_ties <= max(1, max_ties * codes_o.size), f"{what}: {n_ties} tie differences"
+
+
+# ------------------------------------------------------------- quantiser
+@pytest.mark.parametrize("bits,group", [(4, 64), (4, 16), (5, None), (8, None), (8, 32)])
+def test_quantize_matches_oracle_bit_for_bit(bld, bits, group):
+    rng = np.random.default_rng(100 + bits)
+    rows, cols = 37, 256
+    x = rng.standard_normal((rows, cols)) * np.exp(rng.uniform(-6, 2, size=(rows, 1)))
+    x[3] = 0.0                                   # all-zero rows: scale 0, codes 0
+    x[5] *= 1e-9                                 # fp16-subnormal scales
+    G = cols if group is None else group
+    # exact half ties under an fp16 scale of 0.5: amax = qmax * 0.5, members (k + 1/2) * 0.5
+    x[7] = 0.0
+    x[7, ::G] = QMAX[bits] * 0.5
+    x[7, 1::G] = 1.25
+    x[7, 2::G] = -0.75
+    x[7, 3::G] = 2.75
+    xt = torch.from_numpy(x).cuda()
+    codes, scales = bld.quantize(xt, bits, 0 if group is None else group)
+    torch.cuda.synchronize()
+    codes_o, s_o = oracle.quantize_symmetric(x, bits, group)
+    np.testing.assert_array_equal(codes.cpu().numpy(), codes_o)
+    np.testing.assert_array_equal(scales.cpu().numpy().view(np.uint16).reshape(s_o.shape), s_o)
+
+
+def test_quantize_rejects_bad_arguments(bld):
+    x = torch.zeros(4, 64, dtype=torch.float64, device="cuda")
+    with pytest.raises(bld.ArcheadBuildError):
+        bld.quantize(x, 6, 0)
+    with pytest.raises(bld.ArcheadBuildError):
+        bld.quantize(x, 4, 24)                   # 24 does not divide 64
+
+
+# ---------------------------------------------------------------- metric
+@pytest.fixture(scope="module")
+def cfg1_inputs():
+    W, H, _, _ = gen.dense_head_inputs()
+    H32 = H.astype(np.float32)
+    return W, H32
+
+
+@pytest.mark.parametrize("lam,p", [(1e-2, 0.75), (0.0, 0.5), (0.3, 1.0)])
+def test_metric_matches_oracle(bld, cfg1_inputs, lam, p):
+    _, H32 = cfg1_inputs
+    T_p, T_inv = bld.metric(torch.from_numpy(H32).cuda(), lam, p)
+    _, _, T_o, Ti_o = oracle.damped_metric(H32.astype(np.float64), lam, p)
+    for got, ref in ((T_p, T_o), (T_inv, Ti_o)):
+        got = got.cpu().numpy()
+        assert np.linalg.norm(got - ref) <= 1e-10 * np.linalg.norm(ref)
+
+
+def test_metric_rejects_singular_covariance(bld):
+    H = torch.zeros(64, 32, dtype=torch.float32, device="cuda")     # C = 0, and no damping
+    with pytest.raises(bld.ArcheadBuildError) as e:
+        bld.metric(H, 0.0, 0.75)
+    assert e.value.status == -1
+
+
+# ------------------------------------------------------------ correction
+@pytest.fixture(scope="module")
+def cfg1_oracle_build(cfg1_inputs):
+    W, H32 = cfg1_inputs
+    return oracle.build_packed_head(W, H32.astype(np.float64), r_c=32, r_r=8, g=64, g_B=64, p=0.75, lam=1e-2)
+
+
+def test_correction_from_oracle_remainder(bld, cfg1_oracle_build):
+    b = cfg1_oracle_build
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    out = bld.correction(dev(b["_E"]), dev(b["_T_p"]), dev(b["_T_p_inv"]), 8, 64)
+    assert_quantised_like_oracle(out["A"].cpu(), out["s_A"].cpu(), b["_A_w"], 8, None, "A")
+    assert_quantised_like_oracle(out["B"].cpu(), out["s_B"].cpu(), b["_B_w"], 8, 64, "B")
+
+
+# ------------------------------------------------------- Algorithm 1 end to end
+def _check_build(bld, W, H32, r_c, r_r, g, g_B, ref):
+    got = bld.to_host(bld.build_head(torch.from_numpy(W.astype(np.float32)).cuda(),
+                                     torch.from_numpy(H32).cuda(), r_c, r_r, g, g_B, p=0.75, lam=1e-2))
+    torch.cuda.synchronize()
+    assert_quantised_like_oracle(got["L"], got["s_L"], ref["_A_c"], 5, None, "L")
+    assert_quantised_like_oracle(got["R"], got["s_R"], ref["_B_c"], 8, None, "R")
+    assert_quantised_like_oracle(got["q"], got["s_res"], W - ref["_A_c"] @ ref["_B_c"], 4, g, "q")
+    assert_quantised_like_oracle(got["A"], got["s_A"], ref["_A_w"], 8, None, "A")
+    assert_quantised_like_oracle(got["B"], got["s_B"], ref["_B_w"], 8, g_B, "B")
+    return got
+
+
+def test_build_head_cfg1(bld, cfg1_inputs, cfg1_oracle_build):
+    W, H32 = cfg1_inputs
+    got = _check_build(bld, W, H32, 32, 8, 64, 64, cfg1_oracle_build)
+    # the built components drive the forward kernels like any other head
+    import quantized_output_head_b200 as qoh
+    shape = (1024, 256, 32, 8, 64, 64)
+    _, _, h_bits, _ = gen.dense_head_inputs()
+    y, rowmax = oracle.logits(got, 64, 64, h_bits)
+    tol = oracle.tolerance(h_bits, rowmax)
+    lg, _ = qoh.PackedHead(*shape, got).logits(torch.from_numpy(h_bits.view(np.int16)).cuda())
+    assert (np.abs(lg.cpu().numpy() - y) <= tol).all()
+
+
+@pytest.mark.parametrize("V,d,r_c,r_r,g,g_B,N", [(4096, 1024, 128, 16, 128, 128, 8192),
+                                                 (1000, 320, 0, 5, 64, 32, 2048),
+                                                 (640, 192, 24, 0, 32, 64, 1024)])
+def test_build_head_other_shapes(bld, V, d, r_c, r_r, g, g_B, N):
+    W, H, _, _ = gen.dense_head_inputs(n_calib=N, V=V, d=d, seed_cfg=7)
+    H32 = H.astype(np.float32)
+    ref = oracle.build_packed_head(W, H32.astype(np.float64), r_c=r_c, r_r=r_r, g=g, g_B=g_B, p=0.75, lam=1e-2)
+    _check_build(bld, W, H32, r_c, r_r, g, g_B, ref)
+
+
+def test_build_head_workspace_too_small(bld, cfg1_inputs):
+    W, H32 = cfg1_inputs
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(bld.ArcheadBuildError) as e:
+        bld.build_head(torch.from_numpy(W.astype(np.float32)).cuda(), torch.from_numpy(H32).cuda(),
+                       32, 8, 64, 64, ws=ws)
+    assert e.value.status == -5
