@@ -25,6 +25,7 @@ the dense head W.
 from __future__ import annotations
 
 import dataclasses
+import math
 from typing import Dict, Optional
 
 import numpy as np
@@ -200,6 +201,27 @@ def dense_head_inputs(n_calib: int = 4096, T: int = 4, seed_cfg: int = 1, V: int
     W = low_rank_std * (G1 @ G2) / np.sqrt(rank) + noise_std * rng.standard_normal((V, d))
     W = W.astype(np.float32).astype(np.float64)
     return W, H, h_bits, targets
+
+
+def dense_head_inputs_device(V: int, d: int, n_calib: int, seed: int = 11, rank: int = 32,
+                             low_rank_std: float = 0.05, noise_std: float = 0.01, device: str = "cuda"):
+    """Full-size dense head and calibration states drawn on the device (the
+    config-1 recipe at any shape: W = rank-``rank`` Gaussian part + i.i.d.
+    noise, H ~ N(0, Q0 diag(10 k^-1.5) Q0^T)), from a seeded torch generator.
+    Returns fp32 tensors W [V, d] and H [n_calib, d]."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(SEED_BASE + seed)
+    G1 = torch.randn(V, rank, device=device, generator=g, dtype=torch.float32)
+    G2 = torch.randn(rank, d, device=device, generator=g, dtype=torch.float32)
+    W = low_rank_std * (G1 @ G2) / math.sqrt(rank)
+    W += noise_std * torch.randn(V, d, device=device, generator=g, dtype=torch.float32)
+    Q, Rm = torch.linalg.qr(torch.randn(d, d, device=device, generator=g, dtype=torch.float64))
+    Q = Q * torch.sign(torch.diagonal(Rm))[None, :]
+    lam = 10.0 * torch.arange(1, d + 1, device=device, dtype=torch.float64) ** -1.5
+    z = torch.randn(n_calib, d, device=device, generator=g, dtype=torch.float64)
+    H = ((z * lam.sqrt()[None, :]) @ Q.T).float()
+    return W, H
 
 
 def random_components(shape: HeadShape, seed: int) -> Dict[str, np.ndarray]:

@@ -17,6 +17,12 @@ Timing is on the device with CUDA events, max over ranks.
 
 --impl reference times the CPU oracle (float64 numpy) on the host cores, on a
 bounded sample of vocabulary rows, scaled to the full head.
+
+--build times the GPU construction of the packed head instead (Algorithm 1:
+damped metric, truncated SVDs, quantisers; fp64) from a seeded dense head of
+the Qwen3-8B shape and 16,384 calibration states (the largest calibration
+budget the pages report), with the oracle's builder on a slice of the head
+rows as the CPU baseline.
 """
 from __future__ import annotations
 
@@ -68,6 +74,10 @@ def parse_args():
     ap.add_argument("--variant", default="archead", choices=["archead", "naive-int4", "core-int4"],
                     help="head format: ARCHead, or one of the pages' storage-matched comparison heads "
                          "(Qwen-shaped configs only)")
+    ap.add_argument("--build", action="store_true", help="time the GPU construction of the packed head")
+    ap.add_argument("--build-steps", type=int, default=5)
+    ap.add_argument("--build-warmup", type=int, default=3)
+    ap.add_argument("--n-calib", type=int, default=16384, help="calibration states for --build")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -288,9 +298,134 @@ def cpu_baseline(cfg, wl, T, comps, h_bits):
                        f"{dt:.1f} s, scaled to the full head")
 
 
+# ------------------------------------------------------------------- build
+BUILD_SHAPE = (151936, 4096, 512, 64, 128, 128)   # Qwen3-8B head: V, d, r_c, r_r, g, g_B
+BUILD_ORACLE_ROWS = 4096
+BUILD_OWN_KERNELS = 13    # launches of the builder's own kernels per build (the rest is cuBLAS / cuSOLVER)
+
+
+def build_flops(V, d, r_c, r_r, N):
+    """fp64 flops of the dense products of one build (eigensolvers not counted):
+    H^T H, W^T W, E^T E (one triangle each), A_c = W V_c, W - A_c B_c,
+    E -= L_hat R_hat, A_w = E (T_p V_w), B_w, and the d x d products of T_p,
+    T_p^-1 and T_p E^T E T_p."""
+    return (N * d * d + 2 * V * d * d + 6 * V * d * r_c + 2 * V * d * r_r
+            + 8 * d ** 3 + 4 * d * d * r_r)
+
+
+def dgemm_peak_tflops(torch, n=8192, reps=8):
+    """fp64 tensor-core throughput of a plain cuBLAS DGEMM, measured here."""
+    a = torch.randn(n, n, dtype=torch.float64, device="cuda")
+    b = torch.randn(n, n, dtype=torch.float64, device="cuda")
+    c = a @ b
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch.matmul(a, b, out=c)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1) / 1e3)
+    del a, b, c
+    return 2 * n ** 3 / best / 1e12
+
+
+def build_cpu_baseline(W, H, shape):
+    """The oracle builder on the first BUILD_ORACLE_ROWS head rows (same d,
+    ranks, groups and calibration states); its V-independent metric step is
+    timed on its own and the rest scaled by V."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    V, d, r_c, r_r, g, g_B = shape
+    Ws = W[:BUILD_ORACLE_ROWS].double().cpu().numpy()
+    Hs = H.double().cpu().numpy()
+    t0 = time.perf_counter()
+    oracle.damped_metric(Hs, 1e-2, 0.75)
+    t_metric = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.build_packed_head(Ws, Hs, r_c=r_c, r_r=r_r, g=g, g_B=g_B, p=0.75, lam=1e-2)
+    t_sample = time.perf_counter() - t0
+    est = t_metric + max(t_sample - t_metric, 0.0) * V / BUILD_ORACLE_ROWS
+    return dict(value=est, unit="s per build", cores=cores, kind="oracle",
+                sample=(f"oracle builder on {BUILD_ORACLE_ROWS} of {V} head rows ({t_sample:.1f} s, of which the "
+                        f"metric {t_metric:.1f} s); the rest scaled by V (the SVDs of a {BUILD_ORACLE_ROWS} x {d} "
+                        f"slice cost less per row than the full head's, so this underestimates the CPU)"))
+
+
+def run_build(args):
+    import torch
+    import quantized_output_head_b200.builder as bld
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != 1:
+        raise SystemExit("--build runs on one GPU (each build is independent: replicas only)")
+    torch.cuda.set_device(0)
+    V, d, r_c, r_r, g, g_B = BUILD_SHAPE
+    N = args.n_calib
+    W, H = gen.dense_head_inputs_device(V, d, N)
+    ws = bld.workspace(V, d, r_c, r_r, g, g_B, N)
+    st = torch.cuda.current_stream()
+    for _ in range(args.build_warmup):
+        bld.build_head(W, H, r_c, r_r, g, g_B, ws=ws)
+    torch.cuda.synchronize()
+    times = []
+    with ClockSampler(0, period=0.05) as clk:
+        for _ in range(args.build_steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            out = bld.build_head(W, H, r_c, r_r, g, g_B, ws=ws)
+            e1.record(st)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / 1e3)
+    sec = sum(times) / len(times)
+    flops = build_flops(V, d, r_c, r_r, N)
+    peak = dgemm_peak_tflops(torch)
+    # End to end: pinned host W and H in, every packed component back to pinned host memory.
+    Wh, Hh = W.cpu().pin_memory(), H.cpu().pin_memory()
+    outs_h = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items()}
+    e_times = []
+    for it in range(0 if args.no_e2e else 2):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        Wd, Hd = Wh.cuda(non_blocking=True), Hh.cuda(non_blocking=True)
+        comps = bld.build_head(Wd, Hd, r_c, r_r, g, g_B, ws=ws)
+        for k, v in comps.items():
+            outs_h[k].copy_(v, non_blocking=True)
+        torch.cuda.synchronize()
+        e_times.append(time.perf_counter() - t0)
+        del Wd, Hd, comps
+    e_sec = min(e_times) if e_times else None
+    cpu = None if args.no_cpu_baseline else build_cpu_baseline(W, H, BUILD_SHAPE)
+    line = dict(
+        metric="ARCHead packed-head build time (Algorithm 1) at V=151936, d=4096, r_c=512, r_r=64, N=16384",
+        value=sec, unit="s per build", n_gpus=1, steps=args.build_steps, warmup=args.build_warmup,
+        ms_per_step=sec * 1e3, higher_is_better=False, scaling="weak", vs_baseline=None, dtype="f64",
+        data="synthetic (seeded dense head: rank-32 Gaussian part + noise; anisotropic calibration states)",
+        config=dict(workload=f"qwen3-8b-head build N{N}", V=V, d=d, r_c=r_c, r_r=r_r, g=g, g_B=g_B, n_calib=N,
+                    p=0.75, lam=1e-2, parallelism="replicas x1", l2="inputs larger than L2 (W 2.5 GB fp32)"),
+        roofline=dict(bound="tensor", achieved=flops / sec / 1e12, peak=peak, unit="TFLOP/s",
+                      frac=flops / sec / 1e12 / peak, traffic=None, kernel="whole build (cuBLAS fp64 products, "
+                      "cuSOLVER eigensolvers, own kernels)", algorithmic_flops_per_launch=flops,
+                      peak_source="measured here: cuBLAS DGEMM 8192^3, best of 8 (fp64 tensor cores)"),
+        cpu_baseline=cpu,
+        e2e=None if e_sec is None else dict(
+            value=e_sec, unit="s per build", h2d_bytes_per_step=(W.numel() + H.numel()) * 4,
+            d2h_bytes_per_step=sum(v.numel() * v.element_size() for v in out.values()),
+            call="builder.build_head with pinned host W, H in and components out"),
+        clocks=clk.summary(), gpu_launches=args.build_steps * BUILD_OWN_KERNELS,
+        step_seconds=times)
+    print(json.dumps(line))
+    return 0
+
+
 # -------------------------------------------------------------------- ours
 def main():
     args = parse_args()
+    if args.build:
+        return run_build(args)
     cfg = args.config
     wl, T = workload(cfg, args.T, args.variant)
     rank = int(os.environ.get("RANK", "0"))

@@ -39,3 +39,35 @@ def check_lse_ce(lse_gpu, ce_gpu, y_ref, tol, targets=None):
         ce_ref = lse_ref - y_ref[np.arange(y_ref.shape[0]), np.asarray(targets)]
         d = np.abs(np.asarray(ce_gpu, np.float64) - ce_ref)
         assert np.all(d <= 2 * bound), f"ce: max |err|/bound = {(d / (2 * bound)).max():.3g}"
+
+
+def check_build_properties(W_rows, comps, rows, T_p, g, g_B, fp16_decode, dequantize, what="build"):
+    """Properties any correct build has, checkable on sampled head rows without
+    the full truncated SVDs (used where the oracle cannot rebuild the head):
+      * B_c has orthonormal rows, so R_hat R_hat^T = I up to INT8 rounding;
+      * A_c = W V_c = W B_c^T: each L_hat row is within ~half an INT5 step of
+        W[v] R_hat^T;
+      * the SC4 codes quantise W - A_c B_c: their deviation from
+        W[v] - (W[v] R_hat^T) R_hat is mostly far below half a step (the rest
+        is R_hat's rounding);
+      * the correction A_w B_w removes most of the activation-metric error
+        ||(E - A_w B_w) T_p||^2 of Eq. 8 on those rows.
+    The bounds were set with margin from heads the oracle builds."""
+    Rh = dequantize(comps["R"], comps["s_R"], None)
+    orth = np.abs(Rh @ Rh.T - np.eye(Rh.shape[0])).max()
+    assert orth < 0.01, f"{what}: R_hat R_hat^T deviates from I by {orth:.3g}"
+    Lh = dequantize(comps["L"][rows], comps["s_L"][rows], None)
+    Ac = W_rows @ Rh.T
+    sL = fp16_decode(comps["s_L"][rows])[:, None]
+    dev_L = np.abs(Lh - Ac) / sL
+    assert dev_L.max() < 0.6, f"{what}: L_hat off W R_hat^T by {dev_L.max():.3g} INT5 steps"
+    Qh = dequantize(comps["q"][rows], comps["s_res"][rows], g)
+    sres = np.repeat(fp16_decode(comps["s_res"][rows]), g, axis=1)
+    dev_q = np.abs(Qh - (W_rows - Ac @ Rh)) / sres
+    assert np.median(dev_q) < 0.3 and dev_q.max() < 2.0, (
+        f"{what}: SC4 codes off the residual (median {np.median(dev_q):.3g}, max {dev_q.max():.3g} steps)")
+    E = W_rows - (Lh @ Rh + Qh)
+    corr = dequantize(comps["A"][rows], comps["s_A"][rows], None) @ dequantize(comps["B"], comps["s_B"], g_B)
+    before = np.sum((E @ T_p) ** 2)
+    after = np.sum(((E - corr) @ T_p) ** 2)
+    assert after < 0.25 * before, f"{what}: the correction leaves {after / before:.3g} of the metric error"

@@ -15,6 +15,7 @@ import torch
 
 import archead_inputs as gen
 import oracle
+from parity import check_build_properties
 
 pytestmark = pytest.mark.gpu
 
@@ -181,3 +182,23 @@ def test_build_head_workspace_too_small(bld, cfg1_inputs):
         bld.build_head(torch.from_numpy(W.astype(np.float32)).cuda(), torch.from_numpy(H32).cuda(),
                        32, 8, 64, 64, ws=ws)
     assert e.value.status == -5
+
+
+
+def test_build_head_qwen_shape_properties(bld):
+    """The full Qwen3-8B-shaped build (V=151936, d=4096, r_c=512, r_r=64, 16384
+    calibration states), in the configuration bench.py --build times: codes in
+    range, finite non-negative scales, and the construction's properties on
+    256 sampled rows (the oracle cannot rebuild a head of this size)."""
+    V, d, r_c, r_r, g, g_B, N = 151936, 4096, 512, 64, 128, 128, 16384
+    W, H = gen.dense_head_inputs_device(V, d, N)
+    comps = bld.to_host(bld.build_head(W, H, r_c, r_r, g, g_B))
+    for k, lo, hi in (("L", -16, 15), ("R", -128, 127), ("q", -8, 7), ("A", -128, 127), ("B", -128, 127)):
+        assert comps[k].min() >= lo and comps[k].max() <= hi, k
+    for k in ("s_L", "s_R", "s_res", "s_A", "s_B"):
+        s = oracle.fp16_decode(comps[k])
+        assert np.isfinite(s).all() and (s >= 0).all(), k
+    rows = np.random.default_rng(3).choice(V, 256, replace=False)
+    W_rows = W[torch.from_numpy(rows).cuda()].double().cpu().numpy()
+    T_p, _ = bld.metric(H, 1e-2, 0.75)
+    check_build_properties(W_rows, comps, rows, T_p.cpu().numpy(), g, g_B, oracle.fp16_decode, oracle.dequantize)

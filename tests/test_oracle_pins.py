@@ -473,3 +473,20 @@ def test_gumbel_sampling_invariants():
     assert np.all((d >= 100) & (d < 300))
     g = oracle.gumbel_noise(42, np.arange(3, dtype=np.uint64), np.arange(8, dtype=np.uint64))
     assert np.all(np.isfinite(g))
+
+
+def test_build_properties_hold_for_the_oracle_build():
+    """The sampled-row properties the full-size GPU build is held to hold for
+    a head the oracle builds (so the bounds are the construction's, not the
+    GPU's)."""
+    from parity import check_build_properties
+    V, d = 4096, 1024
+    W, H, _, _ = gen.dense_head_inputs(n_calib=8192, V=V, d=d, seed_cfg=7)
+    b = oracle.build_packed_head(W, H, r_c=128, r_r=16, g=128, g_B=128)
+    comps = {k: v for k, v in b.items() if not k.startswith("_")}
+    rows = np.random.default_rng(3).choice(V, 256, replace=False)
+    check_build_properties(W[rows], comps, rows, b["_T_p"], 128, 128, oracle.fp16_decode, oracle.dequantize)
+    # a transposed core (A_c from the wrong side) must fail them
+    bad = dict(comps, R=np.ascontiguousarray(comps["R"][::-1]))
+    with pytest.raises(AssertionError):
+        check_build_properties(W[rows], bad, rows, b["_T_p"], 128, 128, oracle.fp16_decode, oracle.dequantize)
