@@ -620,8 +620,8 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
       const bool ok = tok && c < nch;
       load_b_frag_f16(zh, k0, lane, ok, zf[c][s][0][0], zf[c][s][0][1]);
       load_b_frag_f16(zl, k0, lane, ok, zf[c][s][1][0], zf[c][s][1][1]);
-      cb += bias_dot(zf[c][s][0][0], zf[c][s][0][1], kBiasLo + 128.f, kBiasLo + 128.f);
-      cb += bias_dot(zf[c][s][1][0], zf[c][s][1][1], kBiasLo + 128.f, kBiasLo + 128.f);
+      cb += bias_dot(zf[c][s][0][0], zf[c][s][0][1], kInt8Offset, kInt8Offset);
+      cb += bias_dot(zf[c][s][1][0], zf[c][s][1][1], kInt8Offset, kInt8Offset);
     }
   }
   const float2 cbc = column_pair(quad_sum(cb), lane);

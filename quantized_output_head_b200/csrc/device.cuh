@@ -120,15 +120,20 @@ __device__ __forceinline__ uint32_t shift_to(uint32_t x) {
 }
 
 // fp16 fragment unpacking.  A 4-bit field placed under the fp16 exponent of
-// 1024 (0x6400, mantissa step 1 at bit 0) reads as 1024 + u, and one exact fp16
-// subtraction of 1024 leaves u; the field at bits 4-7 under the exponent of 64
-// (0x5400, mantissa step 1 at bit 4) reads as 64 + u with no shift at all.  So
-// per k16 step the A columns 2cc, 2cc+1 (registers a0, a1) carry the bare
-// offset code and the columns 2cc+8, 2cc+9 (a2, a3) the code plus 64; the
-// tensor core sees exact small integers and the constant part (offset, and
-// 64 for the high columns) is removed once per scale group in fp32.
-constexpr float kBiasLo = 0.f;
+// 1024 (0x6400, mantissa step 1 at bit 0) reads as 1024 + u; the field at bits
+// 4-7 under the exponent of 64 (0x5400, mantissa step 1 at bit 4) reads as
+// 64 + u with no shift at all.  So per k16 step the A columns 2cc, 2cc+1
+// (registers a0, a1) carry the offset code plus 1024 and the columns 2cc+8,
+// 2cc+9 (a2, a3) the code plus 64, all exact in fp16; the tensor core
+// multiplies exact integers and the constant part (offset, plus 1024 or 64)
+// is removed once per scale group in fp32.  Keeping the 1024 costs
+// accumulation precision only: the products are exact and the fp32
+// accumulator carries the larger constant (an emulation with truncation after
+// every addition puts the resulting logit error below a quarter of the parity
+// tolerance), and it saves two instructions per k16 step.
+constexpr float kBiasLo = 1024.f;
 constexpr float kBiasHi = 64.f;
+constexpr float kInt8Offset = 128.f;          // offset-binary INT8 after the 1024 is subtracted
 constexpr uint32_t kHalf1024x2 = 0x64006400u;
 
 __device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
@@ -141,9 +146,9 @@ __device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
 // columns) and 16, 20, 24, 28 (high columns).
 __device__ __forceinline__ void unpack_int4_biased(uint32_t w, uint32_t (&a)[4]) {
   const uint32_t w8 = w >> 8;
-  a[0] = hsub2_bits(and_or<0x000F000Fu, 0x64006400u>(w), kHalf1024x2);
+  a[0] = and_or<0x000F000Fu, 0x64006400u>(w);
   a[2] = and_or<0x00F000F0u, 0x54005400u>(w);
-  a[1] = hsub2_bits(and_or<0x000F000Fu, 0x64006400u>(w8), kHalf1024x2);
+  a[1] = and_or<0x000F000Fu, 0x64006400u>(w8);
   a[3] = and_or<0x00F000F0u, 0x54005400u>(w8);
 }
 
@@ -154,11 +159,9 @@ __device__ __forceinline__ void unpack_int4_biased(uint32_t w, uint32_t (&a)[4])
 template <int S>
 __device__ __forceinline__ void unpack_int5_biased(uint32_t w, uint32_t hb, uint32_t (&a)[4]) {
   const uint32_t w8 = w >> 8;
-  a[0] = hsub2_bits(and_or_r(shift_to<4 * S + 0 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w)),
-                    kHalf1024x2);
+  a[0] = and_or_r(shift_to<4 * S + 0 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w));
   a[2] = and_or_r(shift_to<4 * S + 1 - 8>(hb), 0x01000100u, and_or<0x00F000F0u, 0x54005400u>(w));
-  a[1] = hsub2_bits(and_or_r(shift_to<4 * S + 2 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w8)),
-                    kHalf1024x2);
+  a[1] = and_or_r(shift_to<4 * S + 2 - 4>(hb), 0x00100010u, and_or<0x000F000Fu, 0x64006400u>(w8));
   a[3] = and_or_r(shift_to<4 * S + 3 - 8>(hb), 0x01000100u, and_or<0x00F000F0u, 0x54005400u>(w8));
 }
 
