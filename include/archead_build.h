@@ -30,9 +30,11 @@
  * Conventions
  *   - Return value: ARCHEAD_OK or a negative ARCHEAD_E* code of archead.h;
  *     archead_build_last_error() describes the last failure of this thread.
- *   - All matrices are row-major device buffers owned by the caller.  The
- *     library allocates no device memory: scratch comes from the caller's
- *     workspace (archead_build_workspace_bytes, 256-byte aligned).
+ *   - All matrices are row-major device buffers owned by the caller.  Scratch
+ *     comes from the caller's workspace (archead_build_workspace_bytes,
+ *     256-byte aligned); the only device memory allocated inside a call is
+ *     what the cuBLAS and cuSOLVER handles it creates (and destroys before
+ *     returning) reserve for themselves.
  *   - Arithmetic is IEEE fp64 (cuBLAS DGEMM / DSYRK / DSYMM for the dense
  *     products, cuSOLVER DSYEVD for the symmetric eigenproblems, this
  *     library's kernels for everything else).

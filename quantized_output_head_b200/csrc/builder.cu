@@ -221,11 +221,18 @@ int launch_quantize(const double* x, int rows, int cols, int bits, int G, int8_t
 struct Handles {
   cublasHandle_t blas = nullptr;
   cusolverDnHandle_t solver = nullptr;
+  cudaStream_t stream = nullptr;
+  bool bound = false;
+  // Work queued on the stream may still use the handles' scratch when a call
+  // returns early with an error: drain it before the handles go.
   ~Handles() {
+    if (bound) cudaStreamSynchronize(stream);
     if (blas) cublasDestroy(blas);
     if (solver) cusolverDnDestroy(solver);
   }
   int init(cudaStream_t st) {
+    stream = st;
+    bound = true;
     CK_BLAS(cublasCreate(&blas));
     CK_BLAS(cublasSetStream(blas, st));
     CK_SOLVER(cusolverDnCreate(&solver));
