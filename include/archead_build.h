@@ -94,8 +94,13 @@ ARCHEAD_API int archead_build_correction(const archead_desc* desc, const double*
                                          archead_stream_t stream);
 
 /* Algorithm 1 end to end: from the dense head W [V, d] (fp32) and calibration
- * states H [n_calib, d] (fp32), every component of the packed head.
- * desc: d a multiple of g and g_B, 1 <= r_c + r_r <= d, r_c, r_r >= 0. */
+ * states H [n_calib, d] (fp32), every component of the packed head, written
+ * to the caller's device buffers in `out` (those of a rank-0 branch may be
+ * null; its per-row scales, if given, are set to fp16 zero).
+ * desc: g and g_B divide d; 0 <= r_c, r_r <= min(V, d); r_c + r_r >= 1.
+ * EINVAL on a bad argument or a C_lam that is not positive definite, EALIGN /
+ * ENOMEM on a misaligned / too small workspace, ECUDA on a failed CUDA,
+ * cuBLAS or cuSOLVER call (archead_build_last_error names it). */
 ARCHEAD_API int archead_build_head(const archead_desc* desc, const float* W, const float* H, int32_t n_calib,
                                    double lam, double p, const archead_device_components* out, void* workspace,
                                    size_t ws_bytes, archead_stream_t stream);
