@@ -47,6 +47,7 @@ import archead_inputs as gen  # noqa: E402
 
 METRIC = "packed LM-head tokens/s & µs/call at V=151936,d=4096; % HBM or MMA roofline"
 FALLBACK_HBM_GBS = 6650.0
+CPU_SAMPLE_SECONDS = 12.0   # target length of the CPU-oracle sample behind cpu_baseline
 FALLBACK_BF16_TFLOPS = 1590.0
 
 OPS = {  # config -> what one call produces
@@ -287,15 +288,21 @@ def cpu_baseline(cfg, wl, T, comps, h_bits):
     except Exception:
         cores = os.cpu_count()
     shape = wl.shape
-    n_rows = min(shape.V, 32768)
+    # A pilot on a few rows sizes the sample to about CPU_SAMPLE_SECONDS of
+    # oracle work (the whole head when that fits: no scaling at all).
+    pilot = min(shape.V, 2048)
+    t0 = time.perf_counter()
+    oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=np.arange(pilot))
+    t_pilot = max(time.perf_counter() - t0, 1e-3)
+    n_rows = int(min(shape.V, max(pilot, pilot * CPU_SAMPLE_SECONDS / t_pilot)))
     rows = np.arange(n_rows)
     t0 = time.perf_counter()
     oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
     dt = time.perf_counter() - t0
     per_call = dt * shape.V / n_rows
+    scaled = "" if n_rows == shape.V else ", scaled to the full head"
     return dict(value=T / per_call, unit="tokens/s", cores=cores, kind="oracle",
-                sample=f"oracle on {n_rows} of {shape.V} vocabulary rows for {T} token(s), "
-                       f"{dt:.1f} s, scaled to the full head")
+                sample=f"oracle on {n_rows} of {shape.V} vocabulary rows for {T} token(s), {dt:.1f} s{scaled}")
 
 
 # ------------------------------------------------------------------- build
