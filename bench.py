@@ -295,6 +295,7 @@ def cpu_baseline(cfg, wl, T, comps, h_bits):
     oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=np.arange(pilot))
     t_pilot = max(time.perf_counter() - t0, 1e-3)
     n_rows = int(min(shape.V, max(pilot, pilot * CPU_SAMPLE_SECONDS / t_pilot)))
+    n_rows = max(pilot, min(n_rows, int(2e9 // (8 * T))))   # at most ~2 GB of fp64 logits on the host
     rows = np.arange(n_rows)
     t0 = time.perf_counter()
     oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
