@@ -48,6 +48,7 @@ import archead_inputs as gen  # noqa: E402
 METRIC = "packed LM-head tokens/s & µs/call at V=151936,d=4096; % HBM or MMA roofline"
 FALLBACK_HBM_GBS = 6650.0
 CPU_SAMPLE_SECONDS = 12.0   # target length of the CPU-oracle sample behind cpu_baseline
+REFERENCE_SECONDS = 120.0   # target length of a whole --impl reference run
 FALLBACK_BF16_TFLOPS = 1590.0
 
 OPS = {  # config -> what one call produces
@@ -248,6 +249,23 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- reference
+def oracle_call_model(oracle, comps, shape, h_bits, small=256, large=2048):
+    """(fixed seconds per oracle call, seconds per vocabulary row) from two
+    timed calls on `small` and `large` rows (best of two each)."""
+    def best(n):
+        rows = np.arange(min(shape.V, n))
+        ts = []
+        for _ in range(2):
+            t0 = time.perf_counter()
+            oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
+            ts.append(time.perf_counter() - t0)
+        return rows.size, min(ts)
+    n1, t1 = best(small)
+    n2, t2 = best(large)
+    t_row = max((t2 - t1) / max(n2 - n1, 1), 1e-7)
+    return max(t1 - n1 * t_row, 0.0), t_row
+
+
 def run_reference(args, cfg, wl, T):
     """The CPU oracle as it stands, timed on a bounded sample of vocabulary rows."""
     import oracle
@@ -260,16 +278,23 @@ def run_reference(args, cfg, wl, T):
     sh = (shape.V, shape.d, shape.r_c, shape.r_r, shape.g, shape.g_B)
     comps = gen.draw_components(shape, wl.head_seed_cfg)
     h_bits, targets = gen.draw_activations(shape.d, T, shape.V, cfg)
-    rows = np.arange(min(shape.V, 8192))
+    # Each step is a bounded sample of vocabulary rows, sized so that the whole
+    # --warmup + --steps run takes about REFERENCE_SECONDS.  A call of the
+    # oracle has a fixed part (decoding R, B and h) and a part per row; a
+    # two-size pilot separates them, and only the per-row part is scaled to V.
+    t_fixed, t_row = oracle_call_model(oracle, comps, shape, h_bits)
+    per_step = REFERENCE_SECONDS / max(args.steps + args.warmup, 1)
+    rows = np.arange(int(min(shape.V, max(128, (per_step - t_fixed) / t_row))))
     for _ in range(args.warmup):
         oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
     dt = (time.perf_counter() - t0) / args.steps
-    per_call = dt * shape.V / rows.size
+    per_call = t_fixed + max(dt - t_fixed, 0.0) * shape.V / rows.size
     value = T / per_call
-    sample = f"{rows.size} of {shape.V} vocabulary rows x {T} tokens per step, scaled to the full head"
+    sample = (f"{rows.size} of {shape.V} vocabulary rows x {T} tokens per step; the per-row time scaled to the "
+              f"full head, the fixed {t_fixed * 1e3:.0f} ms per call counted once")
     return dict(impl="reference", metric=METRIC, value=value, unit="tokens/s", n_gpus=args.gpus,
                 steps=args.steps, warmup=args.warmup, ms_per_step=per_call * 1e3, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
