@@ -587,28 +587,33 @@ def main():
     status = head.status(ws)
     launches_per_step = ((1 + n_launch) if kind == "decode" else 3) + (1 if sharded else 0)
 
+    # End to end through the host-buffer entry point, every rank at once (each
+    # serves its own batch); the slowest rank's time sets the job's figure.
+    e2e = None
+    if not args.no_e2e and not sharded and args.sample is None:
+        hh = torch.from_numpy(h_bits.view(np.int16)).pin_memory().numpy().view(np.uint16)
+        th = torch.from_numpy(targets).pin_memory().numpy()
+        outs = (torch.empty(T, dtype=torch.float32).pin_memory().numpy(),
+                torch.empty(T, dtype=torch.int32).pin_memory().numpy(),
+                torch.empty(T, dtype=torch.float32).pin_memory().numpy())
+        for _ in range(3):
+            head.lse_argmax_host(hh, th, outs)
+        e_steps = max(10, min(args.steps, 2000))
+        barrier()
+        t0 = time.perf_counter()
+        for _ in range(e_steps):
+            head.lse_argmax_host(hh, th, outs)
+        e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3, dev)
+        e_dt = e_ms / 1e3 / e_steps
+        e2e = dict(value=world * T / e_dt, unit="tokens/s", h2d_bytes_per_step=world * (T * shape.d * 2 + 4 * T),
+                   d2h_bytes_per_step=world * 12 * T, us_per_call=e_dt * 1e6,
+                   call="archead_lse_argmax_host (host buffers, lse+argmax+ce)")
+
     out = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_baseline(cfg, wl, T, comps, h_bits)
-        e2e = None
-        if not args.no_e2e and not sharded and args.sample is None:
-            hh = torch.from_numpy(h_bits.view(np.int16)).pin_memory().numpy().view(np.uint16)
-            th = torch.from_numpy(targets).pin_memory().numpy()
-            outs = (torch.empty(T, dtype=torch.float32).pin_memory().numpy(),
-                    torch.empty(T, dtype=torch.int32).pin_memory().numpy(),
-                    torch.empty(T, dtype=torch.float32).pin_memory().numpy())
-            for _ in range(3):
-                head.lse_argmax_host(hh, th, outs)
-            e_steps = max(10, min(args.steps, 2000))
-            t0 = time.perf_counter()
-            for _ in range(e_steps):
-                head.lse_argmax_host(hh, th, outs)
-            e_dt = (time.perf_counter() - t0) / e_steps
-            e2e = dict(value=T / e_dt, unit="tokens/s", h2d_bytes_per_step=T * shape.d * 2 + 4 * T,
-                       d2h_bytes_per_step=12 * T, us_per_call=e_dt * 1e6,
-                       call="archead_lse_argmax_host (host buffers, lse+argmax+ce)")
         ab, af = algorithmic(sh, T, op)
         out = dict(
             metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
