@@ -305,7 +305,37 @@ def run_reference(args, cfg, wl, T):
                 algorithmic=dict(zip(("bytes", "flops"), algorithmic(sh, T, OPS[cfg]))))
 
 
-def cpu_baseline(cfg, wl, T, comps, h_bits):
+def oracle_parity(oracle, shape, h_bits, y, rowmax, gpu):
+    """The GPU outputs of the timed run against the oracle's values from the
+    baseline sample: max |d logit| / tolerance on the sampled rows and, when
+    the sample is the whole head, max |d LSE| / tolerance and the argmax
+    mismatches beyond the tie rule (a different row is accepted only where the
+    oracle's gap to it is within the two rows' tolerance)."""
+    n_rows = y.shape[1]
+    res = dict(rows=int(n_rows), tokens=int(y.shape[0]))
+    full = n_rows == shape.V
+    if gpu.get("logits") is None and not full:
+        res["note"] = "sampled rows carry no GPU output to compare (no logits written)"
+        return res
+    tol = oracle.tolerance(h_bits, rowmax)
+    if gpu.get("logits") is not None:
+        res["logits_max_err_over_tol"] = float((np.abs(gpu["logits"][:, :n_rows] - y) / tol).max())
+    if full:
+        lse_ref, am_ref, _ = oracle.lse_argmax_ce(y)
+        if gpu.get("lse") is not None:
+            res["lse_max_err_over_tol"] = float((np.abs(gpu["lse"] - lse_ref) / tol.max(axis=1)).max())
+        if gpu.get("argmax") is not None:
+            a = gpu["argmax"].astype(np.int64)
+            t = np.arange(a.size)
+            inside = (a >= 0) & (a < shape.V)
+            ac = np.where(inside, a, 0)
+            gap = y[t, am_ref] - y[t, ac]
+            bad = (a != am_ref) & (~inside | (gap > np.maximum(tol[t, ac], tol[t, am_ref])))
+            res["argmax_mismatches"] = int(bad.sum())
+    return res
+
+
+def cpu_baseline(cfg, wl, T, comps, h_bits, gpu=None):
     import oracle
     try:
         from threadpoolctl import threadpool_info
@@ -323,12 +353,19 @@ def cpu_baseline(cfg, wl, T, comps, h_bits):
     n_rows = max(pilot, min(n_rows, int(2e9 // (8 * T))))   # at most ~2 GB of fp64 logits on the host
     rows = np.arange(n_rows)
     t0 = time.perf_counter()
-    oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
+    y, rowmax = oracle.logits(comps, shape.g, shape.g_B, h_bits, rows=rows)
     dt = time.perf_counter() - t0
     per_call = dt * shape.V / n_rows
     scaled = "" if n_rows == shape.V else ", scaled to the full head"
-    return dict(value=T / per_call, unit="tokens/s", cores=cores, kind="oracle",
-                sample=f"oracle on {n_rows} of {shape.V} vocabulary rows for {T} token(s), {dt:.1f} s{scaled}")
+    cpu = dict(value=T / per_call, unit="tokens/s", cores=cores, kind="oracle",
+               sample=f"oracle on {n_rows} of {shape.V} vocabulary rows for {T} token(s), {dt:.1f} s{scaled}")
+    parity = None
+    if gpu is not None:
+        try:
+            parity = oracle_parity(oracle, shape, h_bits, y, rowmax, gpu)
+        except Exception as e:   # the check must never cost the measurement
+            parity = dict(error=repr(e))
+    return cpu, parity
 
 
 # ------------------------------------------------------------------- build
@@ -611,9 +648,15 @@ def main():
 
     out = None
     if rank == 0:
-        cpu = None
+        cpu = parity = None
         if world == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline(cfg, wl, T, comps, h_bits)
+            gpu_out = None
+            if not sharded:   # the outputs of the last step of the timed run
+                torch.cuda.synchronize()
+                gpu_out = dict(logits=None if logits is None else logits.cpu().numpy().astype(np.float64),
+                               lse=lse.cpu().numpy().astype(np.float64) if op["lse"] else None,
+                               argmax=am.cpu().numpy())
+            cpu, parity = cpu_baseline(cfg, wl, T, comps, h_bits, gpu_out)
         ab, af = algorithmic(sh, T, op)
         out = dict(
             metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
@@ -636,7 +679,7 @@ def main():
                           peak_source=peak_src + (" (sustained bf16)" if bound == "tensor" else "")),
             call=dict(algorithmic_bytes=ab, algorithmic_flops=af, gbs=ab / (ms_per_step / 1e3) / 1e9,
                       hbm_frac=ab / (ms_per_step / 1e3) / 1e9 / hbm),
-            cpu_baseline=cpu, e2e=e2e, clocks=clk.summary(),
+            cpu_baseline=cpu, parity=parity, e2e=e2e, clocks=clk.summary(),
             gpu_launches=args.steps * launches_per_step, device_status=status,
         )
     if world > 1:
