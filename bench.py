@@ -651,7 +651,7 @@ def main():
         cpu = parity = None
         if world == 1 and not args.no_cpu_baseline:
             gpu_out = None
-            if not sharded:   # the outputs of the last step of the timed run
+            if not sharded and args.sample is None:   # the last timed step's outputs are in these buffers
                 torch.cuda.synchronize()
                 gpu_out = dict(logits=None if logits is None else logits.cpu().numpy().astype(np.float64),
                                lse=lse.cpu().numpy().astype(np.float64) if op["lse"] else None,
