@@ -175,3 +175,27 @@ def test_forward_rejects_null_handle(qoh):
     assert L.archead_workspace_bytes(None, 4) == 0
     assert L.archead_forward_kernel(None, 4) == -1
     assert L.archead_status_string(qoh.ARCHEAD_EUNSUP) == b"unsupported shape or device"
+
+
+def test_sampling_and_shard_calls_refuse_bad_arguments_on_the_host(qoh):
+    """These checks return before any CUDA call or handle use (no GPU here)."""
+    import ctypes as ct
+    L = qoh._lib
+    fake = 4096                                  # never dereferenced: the checks fail first
+    for temp in (0.0, -1.0, float("inf"), float("nan")):
+        assert L.archead_sample(fake, fake, 1, temp, 1, 0, fake, None, None, fake, 1 << 20, None) == \
+            qoh.ARCHEAD_EINVAL
+    assert L.archead_sample(fake, fake, 1, 1.0, 1, 0, None, None, None, fake, 1 << 20, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_sample(fake, fake, 1, 1.0, 1, 0, fake + 2, None, None, fake, 1 << 20, None) == \
+        qoh.ARCHEAD_EALIGN
+    assert L.archead_set_vocab_shard(None, 0, 10) == qoh.ARCHEAD_EINVAL
+    assert L.archead_shard_partials(fake, fake, 1, None, None, fake, 1 << 20, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_shard_partials(fake, fake, 1, None, fake + 4, fake, 1 << 20, None) == qoh.ARCHEAD_EALIGN
+    assert L.archead_merge_shards(None, 2, 1, fake, fake, fake, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_merge_shards(fake, 0, 1, fake, fake, fake, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_merge_shards(fake, 2, 0, fake, fake, fake, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_merge_shards(fake, 2, 1, None, None, None, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_merge_shards(fake + 4, 2, 1, fake, fake, fake, None) == qoh.ARCHEAD_EALIGN
+    status = ct.c_uint32(0)
+    assert L.archead_workspace_status(None, 0, None, ct.byref(status)) == qoh.ARCHEAD_EINVAL
+    assert L.archead_workspace_status(fake + 16, 0, None, ct.byref(status)) == qoh.ARCHEAD_EALIGN
