@@ -199,3 +199,15 @@ def test_sampling_and_shard_calls_refuse_bad_arguments_on_the_host(qoh):
     status = ct.c_uint32(0)
     assert L.archead_workspace_status(None, 0, None, ct.byref(status)) == qoh.ARCHEAD_EINVAL
     assert L.archead_workspace_status(fake + 16, 0, None, ct.byref(status)) == qoh.ARCHEAD_EALIGN
+
+
+def test_builder_binding_refuses_host_or_wrongly_typed_tensors(qoh):
+    """The construction binding checks its tensors before it calls the library."""
+    import torch
+    import quantized_output_head_b200.builder as bld
+    with pytest.raises(ValueError):
+        bld.quantize(torch.zeros(4, 64, dtype=torch.float64), 4, 16)          # host tensor
+    with pytest.raises(ValueError):
+        bld.metric(torch.zeros(64, 32, dtype=torch.float64), 0.01, 0.75)      # fp64, host
+    with pytest.raises(ValueError):
+        bld.build_head(torch.zeros(32, 64), torch.zeros(16, 64), 4, 2, 16, 16)
