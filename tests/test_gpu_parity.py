@@ -12,7 +12,7 @@ import torch
 
 import archead_inputs as gen
 import oracle
-from parity import check_argmax, check_lse_ce, check_logits
+from parity import check_argmax, check_argmax_exact, check_lse_ce, check_logits
 
 pytestmark = pytest.mark.gpu
 
@@ -71,6 +71,21 @@ def test_cfg1_host_buffer_entry_matches_device_entry(cfg1):
     assert np.array_equal(ce_h, ce_d.cpu().numpy())
 
 
+def test_cfg1_host_logits_entry_matches_device_entry(cfg1):
+    """archead_logits_host (host buffers in and out) gives the device entry's
+    logits and argmax bit for bit, and both outputs are optional."""
+    head, h_bits, _, y, tol = cfg1
+    lg_d, am_d = head.logits(_dev_hidden(h_bits))
+    lg_h, am_h = head.logits_host(h_bits)
+    assert np.array_equal(lg_h, lg_d.cpu().numpy())
+    assert np.array_equal(am_h, am_d.cpu().numpy())
+    check_logits(lg_h, y, tol)
+    only_am = head.logits_host(h_bits, out=(None, np.empty(h_bits.shape[0], np.int32)))[1]
+    assert np.array_equal(only_am, am_d.cpu().numpy())
+    with pytest.raises(Exception):
+        head.logits_host(h_bits, out=(None, None))
+
+
 # ------------------------------------------------ Qwen-shaped head (2, 3, 5)
 @pytest.fixture(scope="module")
 def qwen(qoh):
@@ -79,11 +94,10 @@ def qwen(qoh):
     h1, t1 = gen.draw_activations(4096, 1, shape.V, 2)
     h64, t64 = gen.draw_activations(4096, 64, shape.V, 3)
     h5, t5 = gen.draw_activations(4096, 4096, shape.V, 5)
-    sample5 = np.linspace(0, 4095, 12).astype(int)
-    stacked = np.concatenate([h1, h64, h5[sample5]], axis=0)
+    stacked = np.concatenate([h1, h64], axis=0)
     y, tol = _oracle(comps, QWEN, stacked)
-    return dict(head=head, h1=h1, t1=t1, h64=h64, t64=t64, h5=h5, t5=t5, sample5=sample5,
-                y1=y[:1], tol1=tol[:1], y64=y[1:65], tol64=tol[1:65], y5=y[65:], tol5=tol[65:])
+    return dict(head=head, comps=comps, h1=h1, t1=t1, h64=h64, t64=t64, h5=h5, t5=t5,
+                y1=y[:1], tol1=tol[:1], y64=y[1:65], tol64=tol[1:65])
 
 
 def test_qwen_decode_T1_logits_argmax(qwen):
@@ -121,14 +135,27 @@ def test_qwen_decode_T64_logits(qwen):
     check_argmax(am.cpu().numpy(), qwen["y64"], qwen["tol64"])
 
 
-def test_qwen_prefill_T4096_sampled(qwen):
-    """Full 4096-token call; the oracle checks 12 evenly spaced tokens over all V."""
+def test_qwen_prefill_T4096_every_token_and_T512_logits(qwen):
+    """Config 5 at full size: LSE, CE and argmax of all 4096 tokens (32 token
+    tiles of the tensor-core launch) over the whole vocabulary, and every logit
+    of a 512-token call (four token tiles), against the oracle.  The oracle runs
+    on batches of 1024 tokens to bound host memory."""
     head = qwen["head"]
-    lse, am, ce = head.lse_argmax(_dev_hidden(qwen["h5"]), torch.from_numpy(qwen["t5"]))
-    s = qwen["sample5"]
-    lse, am, ce = lse.cpu().numpy()[s], am.cpu().numpy()[s], ce.cpu().numpy()[s]
-    check_lse_ce(lse, ce, qwen["y5"], qwen["tol5"], qwen["t5"][s])
-    check_argmax(am, qwen["y5"], qwen["tol5"])
+    h5, t5 = qwen["h5"], qwen["t5"]
+    assert head.forward_kernel(4096) == "tensor_core" and head.forward_kernel(512) == "tensor_core"
+    lse, am, ce = head.lse_argmax(_dev_hidden(h5), torch.from_numpy(t5))
+    lse, am, ce = lse.cpu().numpy(), am.cpu().numpy(), ce.cpu().numpy()
+    lg512, am512 = head.logits(_dev_hidden(h5[:512]))
+    lg512, am512 = lg512.cpu().numpy(), am512.cpu().numpy()
+    for b0 in range(0, 4096, 1024):
+        sl = slice(b0, b0 + 1024)
+        y, tol = _oracle(qwen["comps"], QWEN, h5[sl])
+        check_lse_ce(lse[sl], ce[sl], y, tol, t5[sl])
+        check_argmax(am[sl], y, tol)
+        if b0 == 0:
+            check_logits(lg512, y[:512], tol[:512])
+            check_argmax(am512, y[:512], tol[:512])
+        del y, tol
 
 
 def test_qwen_calls_are_deterministic(qwen):
@@ -370,3 +397,92 @@ def test_forward_argument_errors(qoh):
     with pytest.raises(qoh.ArcheadError) as e:
         head.lse_argmax_into(big[1:129].view(2, 64), None, lse, am, None, ws)
     assert e.value.status == qoh.ARCHEAD_EALIGN
+
+
+# ------------------------------------------- argmax ties and extreme tokens
+def _tie_head(gen_seed, V, d, T, h_bits, spacing):
+    """Components where, for token t, rows b_t - spacing < b_t < b_t + spacing
+    are identical copies of a row whose residual codes follow the sign of h_t
+    (so its logit is the row maximum by a wide margin).  The copies sit at the
+    same position modulo `spacing` (a multiple of 16, the m-tile height, or of
+    128, the tensor-core tile height), in different tiles, so both kernels
+    compute bit-identical logits for them and the lowest index must win."""
+    shape = (V, d, 32, 8, 64, 64)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=gen_seed)
+    h = oracle.bf16_decode(h_bits)
+    triples = []
+    step = (V - 2 * spacing - 16) // T
+    for t in range(T):
+        b = spacing + 8 + step * t + t % 16
+        rows = (b - spacing, b, b + spacing)
+        assert rows[0] >= 0 and rows[2] < V
+        comps["q"][b] = np.where(h[t] >= 0, 7, -8).astype(np.int8)
+        comps["s_res"][b] = gen.f64_to_fp16_bits(np.full(d // 64, 0.006))   # two standard deviations
+        for v in (rows[0], rows[2]):
+            for k in ("L", "s_L", "q", "s_res", "A", "s_A"):
+                comps[k][v] = comps[k][b]
+        triples.append(rows)
+    assert len({v for r in triples for v in r}) == 3 * T   # the triples of different tokens never meet
+    return shape, comps, triples
+
+
+@pytest.mark.parametrize("T,spacing", [(5, 16), (5, 2368), (24, 128), (24, 1280)])
+def test_argmax_ties_resolve_to_lowest_index(qoh, T, spacing):
+    """Equal maxima in different m-tiles / 128-row tiles / blocks: argmax must be
+    exactly the lowest index on both entry points (5 tokens: decode kernel,
+    24 tokens: tensor-core kernel; spacing 2368 = 148 m-tiles puts two copies in
+    the same decode block)."""
+    V, d = 7000, 256
+    h_bits, targets = gen.random_hidden(d, T, seed=41 + T, V=V)
+    shape, comps, triples = _tie_head(40 + T, V, d, T, h_bits, spacing)
+    head = qoh.PackedHead(*shape, comps)
+    assert head.forward_kernel(T) == ("decode" if T <= 8 else "tensor_core")
+    y, tol = _oracle(comps, shape, h_bits)
+    lowest = np.array([r[0] for r in triples])
+    # the construction: the oracle's maximum is the triple, by more than the tolerance
+    _, am_ref, _ = oracle.lse_argmax_ce(y)
+    assert np.array_equal(am_ref, lowest)
+    for t, rows in enumerate(triples):
+        rest = np.delete(y[t], rows)
+        assert y[t, rows[0]] - rest.max() > 4 * tol[t].max()
+    lg, am = head.logits(_dev_hidden(h_bits))
+    lg = lg.cpu().numpy()
+    for t, rows in enumerate(triples):   # the copies are bit-identical on the GPU too
+        assert lg[t, rows[0]] == lg[t, rows[1]] == lg[t, rows[2]]
+    check_logits(lg, y, tol)
+    check_argmax_exact(am.cpu().numpy(), lowest)
+    lse, am2, ce = head.lse_argmax(_dev_hidden(h_bits), torch.from_numpy(targets))
+    check_argmax_exact(am2.cpu().numpy(), lowest, "argmax (fused epilogue)")
+    check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, targets)
+
+
+@pytest.mark.parametrize("T", [5, 24])   # decode kernel, tensor-core kernel
+def test_zero_and_extreme_magnitude_tokens(qoh, T):
+    """Token 0 all zero (every logit exactly 0: argmax 0, LSE = log V), token 1
+    scaled by 2^64, token 2 by 2^-60 (bf16 exact), the rest ordinary."""
+    shape = (3000, 256, 32, 8, 64, 64)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=606)
+    h_bits, targets = gen.random_hidden(256, T, seed=607, V=shape[0])
+    h = gen.bf16_bits_to_f32(h_bits).copy()
+    h[0] = 0.0
+    h[1] *= np.float32(2.0 ** 64)
+    h[2] *= np.float32(2.0 ** -60)
+    h_bits = gen.f32_to_bf16_bits(h)
+    assert np.array_equal(gen.bf16_bits_to_f32(h_bits), h)   # the scaling is exact in bf16
+    head = qoh.PackedHead(*shape, comps)
+    y, tol = _oracle(comps, shape, h_bits)
+    lg, am = head.logits(_dev_hidden(h_bits))
+    lg, am = lg.cpu().numpy(), am.cpu().numpy()
+    lse, am2, ce = head.lse_argmax(_dev_hidden(h_bits), torch.from_numpy(targets))
+    lse, am2, ce = lse.cpu().numpy(), am2.cpu().numpy(), ce.cpu().numpy()
+    # the zero token: exact zeros, every row tied, so the lowest index
+    assert np.all(lg[0] == 0.0)
+    assert am[0] == 0 and am2[0] == 0
+    np.testing.assert_allclose(lse[0], np.log(shape[0]), rtol=1e-6)
+    np.testing.assert_allclose(ce[0], np.log(shape[0]), rtol=1e-6)
+    # every other token within the tolerance (which scales with ||h_t||)
+    check_logits(lg[1:], y[1:], tol[1:])
+    check_argmax(am[1:], y[1:], tol[1:])
+    check_argmax(am2[1:], y[1:], tol[1:])
+    check_lse_ce(lse[1:], ce[1:], y[1:], tol[1:], targets[1:])
+    assert head.status(head.workspace(T)) == 0
