@@ -172,6 +172,18 @@ ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint
                                         int32_t* argmax_host, float* ce_host, void* workspace,
                                         size_t workspace_bytes, archead_stream_t stream);
 
+/* Host-buffer form of archead_logits: hidden [T, d] bf16 is a HOST pointer
+ * (pinned memory recommended) copied to the device inside the workspace; the
+ * logits [T, V] fp32 and argmax [T] int32 are HOST pointers filled before
+ * return (either may be NULL, not both).  workspace (device, 256-byte
+ * aligned) must be >= archead_host_logits_workspace_bytes(handle, T): it
+ * stages the hidden states and the logits on the device.  Synchronises the
+ * stream. */
+ARCHEAD_API size_t archead_host_logits_workspace_bytes(const archead_handle* handle, int32_t T);
+ARCHEAD_API int archead_logits_host(const archead_handle* handle, const uint16_t* hidden_host, int32_t T,
+                                    float* logits_host, int32_t* argmax_host, void* workspace,
+                                    size_t workspace_bytes, archead_stream_t stream);
+
 /* Allocation-free form of archead_logits_lse_argmax, for callers that may not
  * allocate device memory when they run the head (for example while a CUDA
  * graph is being captured under an allocator that forbids it, or inside a
@@ -180,15 +192,25 @@ ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint
  * archead_static_workspace_capacity() bytes (2 MiB) in the library's own device
  * memory, held by every GPU that loads the library until the process exits.
  * The first call on a device, with that device current, looks the array up
- * (cudaGetSymbolAddress) and clears its status word, so make that first call
- * before any stream capture.  All calls on a device share the array: calls
- * that may overlap on the GPU race.  A T whose workspace would not fit the
- * array returns ARCHEAD_ENOMEM.  (No counterpart in the paper: a library
+ * (cudaGetSymbolAddress) and clears its status word with an asynchronous
+ * memset on `stream`, so make that first call before any stream capture.  A
+ * new context on the device (after cudaDeviceReset) is noticed by its handle
+ * and set up again the same way.  All calls on a device share the array:
+ * calls that may overlap on the GPU race.  A T whose workspace would not fit
+ * the array returns ARCHEAD_ENOMEM.  (No counterpart in the paper: a library
  * convenience.) */
 ARCHEAD_API size_t archead_static_workspace_capacity(void);
 ARCHEAD_API int archead_logits_lse_argmax_static(const archead_handle* handle, const uint16_t* hidden,
                                                  int32_t T, const int32_t* targets, float* lse,
                                                  int32_t* argmax, float* ce, archead_stream_t stream);
+
+/* Status word of the fixed array behind archead_logits_lse_argmax_static on
+ * the current device: the OR of ARCHEAD_STATUS_* bits its calls raised since
+ * the last clear (a timed-out wait, or a target id outside [0, V) whose CE is
+ * NaN).  clear != 0 resets it, ordered on `stream`.  Synchronises `stream`.
+ * Returns ARCHEAD_ETIMEOUT if ARCHEAD_STATUS_WAIT_TIMEOUT is set.  (No
+ * counterpart in the paper.) */
+ARCHEAD_API int archead_static_workspace_status(int clear, archead_stream_t stream, uint32_t* status_out);
 
 /* Temperature sampling fused into the vocabulary pass (a consumer of the
  * logits of Eq. 7 with no counterpart in the paper): for each token t,
@@ -248,6 +270,16 @@ ARCHEAD_API int archead_workspace_status(void* workspace, int clear, archead_str
  * pass alone (the low-rank prologue or activation kernel and the final
  * per-token fold excluded).  NULL, NULL switches it off. */
 ARCHEAD_API int archead_set_profile_events(archead_handle* handle, void* before, void* after);
+
+/* Test support for the decode kernel's bounded waits (no counterpart in the
+ * paper).  Every pipeline wait of the decode kernel gives up after
+ * wait_limit_ns (2 s unless set here), raises ARCHEAD_STATUS_WAIT_TIMEOUT in
+ * the workspace status word and makes its block skip the remaining work, so
+ * the call's outputs are invalid but the context stays usable.  With
+ * stall != 0, later decode-kernel calls on this handle first wait on a
+ * barrier that nothing completes, so the limit expires on purpose.  EINVAL if
+ * handle is NULL or wait_limit_ns is 0.  Restore with (2000000000, 0). */
+ARCHEAD_API int archead_test_decode_waits(archead_handle* handle, uint64_t wait_limit_ns, int stall);
 
 /* Free a handle (host memory only; the arena stays with the caller). */
 ARCHEAD_API void archead_free(archead_handle* handle);
