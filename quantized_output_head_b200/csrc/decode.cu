@@ -56,6 +56,7 @@ struct SmemView {
   float4* tokstate;              // [kEpiWarps][kDecodeTokens] per-warp token states of the block
   float2* pickstate;             // [kEpiWarps][kDecodeTokens] per-warp sampling states of the block
   float* hmax;                   // [kMaxDecodeWarps][kDecodeTokens] max|h_t| over each residual warp's columns
+  uint64_t* stall;               // test hook: a barrier nothing arrives on
   int* flags;                    // [0] abort
 };
 
@@ -68,7 +69,8 @@ __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams&
   v.tokstate = reinterpret_cast<float4*>(v.redfree + p.slots);
   v.pickstate = reinterpret_cast<float2*>(v.tokstate + kEpiWarps * kDecodeTokens);
   v.hmax = reinterpret_cast<float*>(v.pickstate + kEpiWarps * kDecodeTokens);
-  v.flags = reinterpret_cast<int*>(v.hmax + kMaxDecodeWarps * kDecodeTokens);
+  v.stall = reinterpret_cast<uint64_t*>(v.hmax + kMaxDecodeWarps * kDecodeTokens);
+  v.flags = reinterpret_cast<int*>(v.stall + 1);
   return v;
 }
 
@@ -83,8 +85,8 @@ __device__ __forceinline__ void raise_timeout(const SmemView& sv, uint32_t* stat
 
 // Warp-uniform bounded wait; false if the block has aborted or the wait expired.
 __device__ __forceinline__ bool warp_wait(const SmemView& sv, uint64_t* bar, uint32_t parity, uint32_t* status,
-                                          int lane) {
-  bool ok = !aborted(sv) && mbar_wait(smem_addr(bar), parity);
+                                          int lane, uint64_t limit_ns) {
+  bool ok = !aborted(sv) && mbar_wait(smem_addr(bar), parity, limit_ns);
   ok = __all_sync(0xffffffffu, ok);
   if (!ok && lane == 0 && !aborted(sv)) raise_timeout(sv, status);
   return ok;
@@ -138,7 +140,7 @@ __device__ __forceinline__ float quad_sum(float v) {
 __device__ __forceinline__ float* group_begin(const SmemView& sv, const DecodeParams& p, int i, int cw, int lane) {
   const int grp = i >> p.mg_log2;
   const int r = grp & (p.slots - 1);
-  if (grp >= p.slots) warp_wait(sv, &sv.redfree[r], ((grp >> p.slots_log2) - 1) & 1, p.status, lane);
+  if (grp >= p.slots) warp_wait(sv, &sv.redfree[r], ((grp >> p.slots_log2) - 1) & 1, p.status, lane, p.wait_limit_ns);
   return sv.part + (r * p.nw_work + cw) * (kGroupTile * 16);
 }
 
@@ -681,9 +683,12 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
   const int m = e / (16 * p.nt);            // m-tile of the group, token t, rows r, r + 1
   const int t = (e >> 4) - m * p.nt, row = e & 15;
   const int ngroups = (n_my + p.mg - 1) >> p.mg_log2;
+  // Test hook: a wait on a barrier that nothing completes runs out its limit,
+  // raises the timeout status and aborts the block.
+  if (p.test_stall) warp_wait(sv, sv.stall, 0, p.status, lane, p.wait_limit_ns);
   for (int grp = 0; grp < ngroups; ++grp) {
     const int r = grp & (p.slots - 1);
-    const bool ok = warp_wait(sv, &sv.reduced[r], (grp >> p.slots_log2) & 1, p.status, lane);
+    const bool ok = warp_wait(sv, &sv.reduced[r], (grp >> p.slots_log2) & 1, p.status, lane, p.wait_limit_ns);
     const float* part = sv.part + r * p.nw_work * (kGroupTile * 16) + e;
     const int i0 = grp << p.mg_log2;
     if (ok && m < p.mg && i0 + m < n_my) {
@@ -835,6 +840,7 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
       mbar_init(smem_addr(&sv.reduced[r]), p.nw_work);
       mbar_init(smem_addr(&sv.redfree[r]), kEpiWarps);
     }
+    mbar_init(smem_addr(sv.stall), 1);
     sv.flags[0] = 0;
     mbar_fence_init();
   }
@@ -870,7 +876,7 @@ void decode_smem_plan(DecodeParams& p, int g_steps) {
 size_t decode_smem_bytes(const DecodeParams& p) {
   return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16 * 4 +
          static_cast<size_t>(2) * p.slots * 8 + kEpiWarps * kDecodeTokens * (16 + 8) +
-         kMaxDecodeWarps * kDecodeTokens * 4 + 16;
+         kMaxDecodeWarps * kDecodeTokens * 4 + 8 + 16;
 }
 
 namespace {

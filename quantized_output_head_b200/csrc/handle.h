@@ -25,6 +25,8 @@ struct archead_handle {
   int v_total;
   cudaEvent_t ev_before;    // optional profiling events (not owned)
   cudaEvent_t ev_after;
+  uint64_t wait_limit_ns;   // decode kernel: limit of every bounded wait (test hook; default kWaitLimitNs)
+  int test_stall;           // decode kernel: test hook, a wait that nothing completes
 };
 
 namespace archead {
@@ -56,8 +58,9 @@ struct WsLayout {
   size_t escale, zhi, zlo, partials, spart;   // decode path
   size_t cinv, xop, tpartials;                // tensor-core path
   size_t total;
-  // host-buffer form only
+  // host-buffer forms only
   size_t h_hidden, h_targets, h_lse, h_argmax, h_ce, host_total;
+  size_t h_logits, host_logits_total;   // logits form: [T, V] fp32 staging after host_total
 };
 
 inline WsLayout ws_layout(const archead_handle& h, int T) {
@@ -88,6 +91,8 @@ inline WsLayout ws_layout(const archead_handle& h, int T) {
   w.h_argmax = o;  o += round_up(t * 4, 256);
   w.h_ce = o;      o += round_up(t * 4, 256);
   w.host_total = o;
+  w.h_logits = o;  o += round_up(t * static_cast<size_t>(h.L.V) * 4, 256);
+  w.host_logits_total = o;
   return w;
 }
 

@@ -319,6 +319,8 @@ extern "C" ARCHEAD_API int archead_pack_load(const archead_desc* desc, const arc
   h->e_B = row_norm_exponent(L, *comps);
   h->row0 = 0;
   h->v_total = L.V;
+  h->wait_limit_ns = kWaitLimitNs;
+  h->test_stall = 0;
   plan_tc(h, *comps, optin);
   e = decode_set_attributes(L.g_steps, static_cast<size_t>(optin));
   if (e == cudaSuccess && h->tc_ok) e = tc_set_attributes();

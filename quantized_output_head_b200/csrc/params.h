@@ -4,6 +4,10 @@
 
 namespace archead {
 
+// A bounded device-side wait gives up after this long (a legitimate wait is
+// microseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
 // Work split of the decode kernel: each residual warp owns kCRes 64-column
 // chunks of d (16 k16 steps), each core warp kCL 64-column chunks of r_c',
 // each correction warp kCA 32-column chunks of r_r'.
@@ -51,6 +55,10 @@ struct DecodeParams {
   // Shared-memory rings: one per compute warp, kRing slices each.
   uint32_t res_slice_bytes, core_slice_bytes, corr_slice_bytes;
   uint32_t core_ring_off, corr_ring_off, ring_bytes;
+  // Bounded waits: limit per wait, and (test hook only) a stall that makes the
+  // epilogue wait on a barrier no one arrives on, so that the limit expires.
+  uint64_t wait_limit_ns;
+  int32_t test_stall;
 };
 
 struct PrologueParams {
