@@ -628,23 +628,39 @@ def main():
     # serves its own batch); the slowest rank's time sets the job's figure.
     e2e = None
     if not args.no_e2e and not sharded and args.sample is None:
+        # The same outputs as the timed step, through the host-buffer entry
+        # point of the same operation (pinned host memory in and out).
         hh = torch.from_numpy(h_bits.view(np.int16)).pin_memory().numpy().view(np.uint16)
         th = torch.from_numpy(targets).pin_memory().numpy()
-        outs = (torch.empty(T, dtype=torch.float32).pin_memory().numpy(),
-                torch.empty(T, dtype=torch.int32).pin_memory().numpy(),
-                torch.empty(T, dtype=torch.float32).pin_memory().numpy())
+        if op["logits"]:
+            outs = (torch.empty((T, shape.V), dtype=torch.float32).pin_memory().numpy(),
+                    torch.empty(T, dtype=torch.int32).pin_memory().numpy())
+
+            def e2e_call():
+                head.logits_host(hh, outs)
+            h2d, d2h = T * shape.d * 2, T * shape.V * 4 + 4 * T
+            what = "archead_logits_host (host buffers, fp32 logits + argmax)"
+        else:
+            outs = (torch.empty(T, dtype=torch.float32).pin_memory().numpy(),
+                    torch.empty(T, dtype=torch.int32).pin_memory().numpy(),
+                    torch.empty(T, dtype=torch.float32).pin_memory().numpy() if op["ce"] else None)
+
+            def e2e_call():
+                head.lse_argmax_host(hh, th if op["ce"] else None, outs)
+            h2d = T * shape.d * 2 + (4 * T if op["ce"] else 0)
+            d2h = 4 * T * (2 + (1 if op["ce"] else 0))
+            what = "archead_lse_argmax_host (host buffers, lse + argmax" + (" + ce)" if op["ce"] else ")")
         for _ in range(3):
-            head.lse_argmax_host(hh, th, outs)
+            e2e_call()
         e_steps = max(10, min(args.steps, 2000))
         barrier()
         t0 = time.perf_counter()
         for _ in range(e_steps):
-            head.lse_argmax_host(hh, th, outs)
+            e2e_call()
         e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3, dev)
         e_dt = e_ms / 1e3 / e_steps
-        e2e = dict(value=world * T / e_dt, unit="tokens/s", h2d_bytes_per_step=world * (T * shape.d * 2 + 4 * T),
-                   d2h_bytes_per_step=world * 12 * T, us_per_call=e_dt * 1e6,
-                   call="archead_lse_argmax_host (host buffers, lse+argmax+ce)")
+        e2e = dict(value=world * T / e_dt, unit="tokens/s", h2d_bytes_per_step=world * h2d,
+                   d2h_bytes_per_step=world * d2h, us_per_call=e_dt * 1e6, call=what)
 
     out = None
     if rank == 0:

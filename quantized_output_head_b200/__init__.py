@@ -33,6 +33,8 @@ EXPORTED = (
     "archead_logits", "archead_logits_lse_argmax", "archead_host_workspace_bytes", "archead_lse_argmax_host",
     "archead_workspace_status", "archead_set_profile_events", "archead_free", "archead_last_cuda_error",
     "archead_status_string", "archead_static_workspace_capacity", "archead_logits_lse_argmax_static",
+    "archead_static_workspace_status", "archead_test_decode_waits", "archead_host_logits_workspace_bytes",
+    "archead_logits_host",
     "archead_forward_kernel", "archead_set_vocab_shard", "archead_shard_partials", "archead_merge_shards",
     "archead_sample",
 )
@@ -59,16 +61,20 @@ _sig = {
     "archead_logits": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "archead_logits_lse_argmax": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "archead_lse_argmax_host": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "archead_host_logits_workspace_bytes": (_sz, [_vp, _i32]),
+    "archead_logits_host": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "archead_workspace_status": (ctypes.c_int, [_vp, ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "archead_set_profile_events": (ctypes.c_int, [_vp, _vp, _vp]),
     "archead_static_workspace_capacity": (_sz, []),
     "archead_logits_lse_argmax_static": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "archead_static_workspace_status": (ctypes.c_int, [ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "archead_forward_kernel": (ctypes.c_int, [_vp, _i32]),
     "archead_set_vocab_shard": (ctypes.c_int, [_vp, _i32, _i32]),
     "archead_sample": (ctypes.c_int, [_vp, _vp, _i32, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, _vp, _vp,
                                       _vp, _vp, _sz, _vp]),
     "archead_shard_partials": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "archead_merge_shards": (ctypes.c_int, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "archead_test_decode_waits": (ctypes.c_int, [_vp, ctypes.c_uint64, ctypes.c_int]),
     "archead_free": (None, [_vp]),
     "archead_last_cuda_error": (ctypes.c_int, []),
     "archead_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -172,12 +178,16 @@ class PackedHead:
     def workspace_bytes(self, T: int) -> int:
         return int(_lib.archead_workspace_bytes(self.handle, int(T)))
 
-    def workspace(self, T: int, host_form: bool = False) -> torch.Tensor:
-        """A zero-initialised workspace big enough for T tokens (cached per size)."""
-        n = (_lib.archead_host_workspace_bytes if host_form else _lib.archead_workspace_bytes)(self.handle, int(T))
+    def workspace(self, T: int, host_form=False) -> torch.Tensor:
+        """A zero-initialised workspace big enough for T tokens (cached per size).
+        host_form: False (device calls), True (archead_lse_argmax_host) or
+        "logits" (archead_logits_host)."""
+        size = {False: _lib.archead_workspace_bytes, True: _lib.archead_host_workspace_bytes,
+                "logits": _lib.archead_host_logits_workspace_bytes}[host_form]
+        n = size(self.handle, int(T))
         if n == 0:
             raise ArcheadError(ARCHEAD_EINVAL, "workspace size")
-        key = ("host" if host_form else "dev", n)
+        key = (str(host_form), n)
         ws = self._ws.get(key)
         if ws is None:
             ws = torch.zeros(n, dtype=torch.uint8, device=self.device)
@@ -238,6 +248,22 @@ class PackedHead:
                                             ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
                "archead_lse_argmax_host")
         return lse, am, ce
+
+    def logits_host(self, hidden_host: np.ndarray,
+                    out: Optional[Tuple[Optional[np.ndarray], Optional[np.ndarray]]] = None,
+                    stream: Optional[torch.cuda.Stream] = None):
+        """Host-buffer logits: numpy bf16 bits [T, d] (ideally pinned) in,
+        (logits [T, V] fp32, argmax [T] int32) numpy out; synchronises the stream."""
+        hb = np.ascontiguousarray(hidden_host).view(np.uint16)
+        T = int(hb.shape[0])
+        if out is None:
+            out = (np.empty((T, self.V), np.float32), np.empty(T, np.int32))
+        lg, am = out
+        ws = self.workspace(T, host_form="logits")
+        _check(_lib.archead_logits_host(self.handle, hb.ctypes.data, T, None if lg is None else lg.ctypes.data,
+                                        None if am is None else am.ctypes.data, ws.data_ptr(), ws.numel(),
+                                        _stream_ptr(stream)), "archead_logits_host")
+        return lg, am
 
     def sample(self, hidden: torch.Tensor, temperature: float, seed: int, offset: int = 0):
         """Gumbel-max temperature sampling fused into the vocabulary pass: returns

@@ -236,6 +236,8 @@ int forward(const archead_handle* h, const uint16_t* hidden, int32_t T, const in
   dp.nw_L = h->nw_L;
   dp.nw_A = h->nw_A;
   dp.nw_work = h->nw_work;
+  dp.wait_limit_ns = h->wait_limit_ns;
+  dp.test_stall = h->test_stall;
   if (h->ev_before != nullptr) {
     e = cudaEventRecord(h->ev_before, stream);
     if (e != cudaSuccess) return set_cuda_error(e);
@@ -336,6 +338,37 @@ extern "C" ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle,
   return ARCHEAD_OK;
 }
 
+extern "C" ARCHEAD_API size_t archead_host_logits_workspace_bytes(const archead_handle* handle, int32_t T) {
+  if (handle == nullptr || T <= 0 || T > kMaxTokens) return 0;
+  return ws_layout(*handle, T).host_logits_total;
+}
+
+extern "C" ARCHEAD_API int archead_logits_host(const archead_handle* handle, const uint16_t* hidden_host, int32_t T,
+                                               float* logits_host, int32_t* argmax_host, void* workspace,
+                                               size_t workspace_bytes, archead_stream_t stream) {
+  if (handle == nullptr || hidden_host == nullptr || workspace == nullptr) return ARCHEAD_EINVAL;
+  if (logits_host == nullptr && argmax_host == nullptr) return ARCHEAD_EINVAL;
+  if (T <= 0 || T > kMaxTokens) return ARCHEAD_EINVAL;
+  if (!aligned(workspace, 256)) return ARCHEAD_EALIGN;
+  const WsLayout w = ws_layout(*handle, T);
+  if (workspace_bytes < w.host_logits_total) return ARCHEAD_ENOMEM;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(workspace);
+  uint16_t* d_hidden = reinterpret_cast<uint16_t*>(wb + w.h_hidden);
+  float* d_logits = logits_host ? reinterpret_cast<float*>(wb + w.h_logits) : nullptr;
+  int32_t* d_argmax = argmax_host ? reinterpret_cast<int32_t*>(wb + w.h_argmax) : nullptr;
+  const size_t t = static_cast<size_t>(T);
+  cudaError_t e = cudaMemcpyAsync(d_hidden, hidden_host, t * handle->L.d * 2, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  const int rc = forward(handle, d_hidden, T, nullptr, d_logits, d_argmax, nullptr, nullptr, workspace, w.total, s);
+  if (rc != ARCHEAD_OK) return rc;
+  if (logits_host) e = cudaMemcpyAsync(logits_host, d_logits, t * handle->L.V * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && argmax_host) e = cudaMemcpyAsync(argmax_host, d_argmax, t * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  return ARCHEAD_OK;
+}
+
 extern "C" ARCHEAD_API int archead_sample(const archead_handle* handle, const uint16_t* hidden, int32_t T,
                                           float temperature, uint64_t seed, uint64_t offset, int32_t* sampled,
                                           float* lse, int32_t* argmax, void* workspace, size_t workspace_bytes,
@@ -394,6 +427,13 @@ extern "C" ARCHEAD_API int archead_set_profile_events(archead_handle* handle, vo
   if (handle == nullptr || ((before == nullptr) != (after == nullptr))) return ARCHEAD_EINVAL;
   handle->ev_before = static_cast<cudaEvent_t>(before);
   handle->ev_after = static_cast<cudaEvent_t>(after);
+  return ARCHEAD_OK;
+}
+
+extern "C" ARCHEAD_API int archead_test_decode_waits(archead_handle* handle, uint64_t wait_limit_ns, int stall) {
+  if (handle == nullptr || wait_limit_ns == 0) return ARCHEAD_EINVAL;
+  handle->wait_limit_ns = wait_limit_ns;
+  handle->test_stall = stall != 0 ? 1 : 0;
   return ARCHEAD_OK;
 }
 
