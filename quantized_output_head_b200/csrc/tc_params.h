@@ -17,8 +17,9 @@ constexpr int kTcBK = 64;             // K columns per k-step (one 128-byte row 
 constexpr int kTcStepsPerStage = 2;   // k-steps per pipeline stage
 constexpr int kTcMaxBN = 128;         // tokens per unit
 constexpr int kTcMaxStages = 8;       // stages in flight between the producers and the MMA (even)
-constexpr int kTcRingSmall = 3;       // ring slots (stages of packed bytes) per dequantising warp, BN <= 64
-constexpr int kTcRingLarge = 2;       // the same for BN > 64
+constexpr int kTcMinRing = 2;         // ring slots (stages of packed bytes) per dequantising warp:
+constexpr int kTcMaxRing = 5;         //   as many as shared memory holds next to the stage buffers
+constexpr int kTcSmemBudget = 232448; // dynamic shared memory a block may use on sm_100a (227 KB)
 constexpr int kTcSlotBytes = 1056;    // one packed k-step of one m-tile block (codes + scales)
 constexpr int kTcDeqWarps = 16;       // two per m-tile block of a unit (even / odd k-steps)
 constexpr int kTcWarps = 22;          // 16 dequantising, 1 TMA, 1 MMA, 4 epilogue

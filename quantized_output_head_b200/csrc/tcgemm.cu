@@ -229,7 +229,9 @@ __device__ __forceinline__ void dequant_step(const TcParams& p, const uint8_t* s
 // lanes 16j..16j+15 lie in the warp's lane quarter w%4) on the global stages
 // of parity w/8; a stage buffer has a fixed parity (the buffer count is even),
 // so each buffer is filled by the same eight warps.  R: ring slots, each the
-// packed bytes of one stage (two k-steps).
+// packed bytes of one stage (two k-steps), filled R - 1 stages ahead with
+// 16-byte cp.async per lane.  (One bulk copy per piece, issued by one lane,
+// measured slower: the copy engine queues many 512-byte copies.)
 template <int R>
 __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int w, int lane) {
   constexpr uint32_t kPair = 2 * kTcSlotBytes;
@@ -343,33 +345,45 @@ __device__ void tma_warp(const TcParams& p, const TcSmem& sm, const CUtensorMap*
 // ---------------------------------------------------------------- MMA warp
 // The whole warp walks the stages (warp-uniform descriptors); one elected lane
 // issues the MMAs and the commits that track them.
+// The issue cost of a tcgen05.mma is mostly the instructions that prepare its
+// operands, so everything per MMA is an immediate offset from two running
+// values: the stage's A column in TMEM and its B descriptor (both advanced by a
+// constant per stage and reset when the buffer index wraps).
 __device__ void mma_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int lane) {
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
   const uint32_t idesc = tc_idesc_f16(kTcBM, p.BN);
-  const uint32_t bst = smem_addr(sm.bst);
+  const uint64_t bd0 = smem_desc_k128(smem_addr(sm.bst));   // buffer 0, first k-step
+  const uint32_t bstep = p.bstage_bytes >> 4;                // descriptor units per X tile (k-step)
+  const uint32_t a_first = tmem_base + p.acol0;
   int s = 0;
   uint32_t ph = 0;
+  uint64_t bd = bd0;
+  uint32_t ad = a_first;
   for (int ui = 0; ui < n_my; ++ui) {
     const uint32_t a = static_cast<uint32_t>(ui) & 1u;
     if (!tc_wait_warp(sm, &sm.acce[a], ((static_cast<uint32_t>(ui) >> 1) & 1u) ^ 1u, p.status)) return;
     tc_fence_after();
-    const uint32_t d_tmem = tmem_base + a * p.acc_stride;
+    const uint32_t d = tmem_base + a * p.acc_stride;
     // The wait for stage st + 1 sits between issuing stage st's MMAs and
     // committing them, so its latency overlaps the tensor work.
     if (!tc_wait_warp(sm, &sm.full[s], ph, p.status)) return;
     for (int st = 0; st < p.n_st; ++st) {
       tc_fence_after();
-      const int nk = 2 * st + 1 < p.n_ks ? 2 : 1;
-      const uint32_t b0 = bst + static_cast<uint32_t>(s) * 2u * p.bstage_bytes;
-      const uint32_t a0 = tmem_base + p.acol0 + static_cast<uint32_t>(s) * 64u;
-      const bool leader = elect_one();
+      const bool two = 2 * st + 1 < p.n_ks;
+      const uint32_t acc0 = st != 0 ? 1u : 0u;
+      const bool leader = elect_one();   // the same lane issues the MMAs and the commit that tracks them
       if (leader) {
-        for (int h = 0; h < nk; ++h) {
-          const uint64_t bdesc = smem_desc_k128(b0 + static_cast<uint32_t>(h) * p.bstage_bytes);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            tc_mma_ts(d_tmem, a0 + 32u * h + 8u * i, bdesc + 2u * i, idesc, (st | h | i) != 0 ? 1u : 0u);
+        tc_mma_ts(d, ad, bd, idesc, acc0);
+        tc_mma_ts(d, ad + 8u, bd + 2u, idesc, 1u);
+        tc_mma_ts(d, ad + 16u, bd + 4u, idesc, 1u);
+        tc_mma_ts(d, ad + 24u, bd + 6u, idesc, 1u);
+        if (two) {
+          const uint64_t b1 = bd + bstep;
+          tc_mma_ts(d, ad + 32u, b1, idesc, 1u);
+          tc_mma_ts(d, ad + 40u, b1 + 2u, idesc, 1u);
+          tc_mma_ts(d, ad + 48u, b1 + 4u, idesc, 1u);
+          tc_mma_ts(d, ad + 56u, b1 + 6u, idesc, 1u);
         }
       }
       __syncwarp();
@@ -377,6 +391,11 @@ __device__ void mma_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base
       if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
+        ad = a_first;
+        bd = bd0;
+      } else {
+        ad += 64u;
+        bd += 2u * bstep;
       }
       const bool more = st + 1 < p.n_st;
       const bool ok = !more || tc_wait_warp(sm, &sm.full[s], ph, p.status);
@@ -553,19 +572,29 @@ __global__ void __launch_bounds__(256) tc_merge_kernel(const float4* partials, i
 // TMEM: two accumulators of acc_stride columns, then one 64-column A tile (two
 // k-steps) per stage buffer; the buffers use what the accumulators leave of the
 // 512 columns.  Shared memory: two X tiles per stage buffer, the dequantising
-// warps' rings, the epilogue tiles and the barriers.
+// warps' rings (as many slots as fit, kTcMinRing..kTcMaxRing), the epilogue
+// tiles and the barriers.
+namespace {
+constexpr uint32_t kTcBarBytes = 256;
+size_t plan_bytes(const TcParams& p) { return static_cast<size_t>(p.bar_off) + kTcBarBytes + 1024; }
+}  // namespace
+
 void tc_smem_plan(TcParams& p) {
   p.acc_stride = static_cast<uint32_t>((p.BN + 31) / 32 * 32);
   p.acol0 = 2 * p.acc_stride;
   p.stages = static_cast<int32_t>(std::min<uint32_t>(kTcMaxStages, (kTmemCols - p.acol0) / 64)) & ~1;
-  p.ring = p.BN <= 64 ? kTcRingSmall : kTcRingLarge;
   p.bstage_bytes = static_cast<uint32_t>(p.BN) * 128u;   // one X tile; multiple of 2048 (BN % 16 == 0)
   p.ring_off = static_cast<uint32_t>(p.stages) * 2u * p.bstage_bytes;
+  for (p.ring = kTcMaxRing; p.ring > kTcMinRing; --p.ring) {
+    p.epi_off = p.ring_off + kTcDeqWarps * p.ring * 2 * kTcSlotBytes;
+    p.bar_off = p.epi_off + 4 * kTcMaxBN * 16 + 4 * 32 * 33 * 4;
+    if (plan_bytes(p) <= static_cast<size_t>(kTcSmemBudget)) return;
+  }
   p.epi_off = p.ring_off + kTcDeqWarps * p.ring * 2 * kTcSlotBytes;
   p.bar_off = p.epi_off + 4 * kTcMaxBN * 16 + 4 * 32 * 33 * 4;
 }
 
-size_t tc_smem_bytes(const TcParams& p) { return static_cast<size_t>(p.bar_off) + 256 + 1024; }
+size_t tc_smem_bytes(const TcParams& p) { return plan_bytes(p); }
 
 size_t tc_smem_max() {
   size_t m = 0;
@@ -580,16 +609,20 @@ size_t tc_smem_max() {
 
 namespace {
 const void* tc_kernel_for(int ring) {
-  return ring == kTcRingSmall ? reinterpret_cast<const void*>(&tc_kernel<kTcRingSmall>)
-                              : reinterpret_cast<const void*>(&tc_kernel<kTcRingLarge>);
+  switch (ring) {
+    case 2: return reinterpret_cast<const void*>(&tc_kernel<2>);
+    case 3: return reinterpret_cast<const void*>(&tc_kernel<3>);
+    case 4: return reinterpret_cast<const void*>(&tc_kernel<4>);
+    default: return reinterpret_cast<const void*>(&tc_kernel<5>);
+  }
 }
 }  // namespace
 
 cudaError_t tc_set_attributes() {
   const int smem = static_cast<int>(tc_smem_max());
-  cudaError_t e = cudaFuncSetAttribute(tc_kernel_for(kTcRingSmall), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(tc_kernel_for(kTcRingLarge), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaSuccess;
+  for (int r = kTcMinRing; r <= kTcMaxRing && e == cudaSuccess; ++r)
+    e = cudaFuncSetAttribute(tc_kernel_for(r), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   return e;
 }
 
