@@ -118,6 +118,24 @@ __device__ __forceinline__ void issue_step(const TcParams& p, uint32_t dst, cons
   }
 }
 
+// A stage of two residual k-steps (ks0, ks0 + 1) of m-tile block blk: the
+// codes of both (1024 contiguous bytes) and the scales of each, 16 bytes per
+// lane, addressed with a few integer operations (the common stage).
+template <int GM>
+__device__ __forceinline__ void issue_res_stage(const TcParams& p, uint32_t dst, const uint8_t* blk, int ks0,
+                                                int lane) {
+  const uint8_t* codes = blk + p.off_res + ks0 * kResChunkBytes + lane * 16;
+  cp_async16(dst + lane * 16, codes);
+  cp_async16(dst + kTcSlotBytes + lane * 16, codes + kResChunkBytes);
+  constexpr int kPieces = 2 << GM;                   // 16-byte scale pieces per k-step
+  if (lane < 2 * kPieces) {
+    const int kk = lane / kPieces, piece = lane % kPieces;
+    const int g0 = ((ks0 + kk) * kTcBK) >> p.g_log2;
+    cp_async16(dst + kk * kTcSlotBytes + kSlotResScales + piece * 16,
+               blk + p.off_sres + g0 * kSresGroupBytes + piece * 16);
+  }
+}
+
 // Scale pair (row gr, row gr + 8) of a slot -> two half2 (s, s) times 2^e.
 __device__ __forceinline__ void scale_pair(const uint8_t* at, float mul, uint32_t& s0, uint32_t& s1) {
   const float2 f = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(at));
@@ -133,18 +151,18 @@ __device__ __forceinline__ void place(const uint32_t (&a)[4], uint32_t s0, uint3
   r[3] = hmul2_bits(a[3], s1);   // lane gr + 8, column 2cc + 1
 }
 
-__device__ __forceinline__ void dequant_residual(const TcParams& p, const uint8_t* slot, int ks, int lane,
-                                                 uint32_t (&r)[16]) {
+// Residual scale groups per 64-column k-step, fixed at compile time: GM = 0
+// (g >= 64: one group, whose scales the slot holds), 1 (g = 32: two), 2
+// (g = 16: four).  k16 step st uses local group st >> (2 - GM).
+template <int GM>
+__device__ __forceinline__ void dequant_residual(const uint8_t* slot, float sc, int lane, uint32_t (&r)[16]) {
   const int gr = lane >> 2;
   const uint4 c = *reinterpret_cast<const uint4*>(slot + lane * 16);
   const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-  const int gsh = p.g_log2;
   uint32_t s0 = 0, s1 = 0;
 #pragma unroll
   for (int st = 0; st < 4; ++st) {
-    // local group of this k16 step (groups are >= 16 columns, powers of two)
-    const int lg = ((ks * kTcBK + 16 * st) >> gsh) - ((ks * kTcBK) >> gsh);
-    if (st == 0 || gsh < 6) scale_pair(slot + kSlotResScales + lg * kSresGroupBytes + gr * 4, p.sc_res, s0, s1);
+    if (st % (4 >> GM) == 0) scale_pair(slot + kSlotResScales + (st >> (2 - GM)) * kSresGroupBytes + gr * 4, sc, s0, s1);
     uint32_t a[4];
     unpack_int4_signed(w[st], a);
     place(a, s0, s1, r + 4 * st);
@@ -218,9 +236,10 @@ __device__ __forceinline__ void cursor_advance(StageCursor& c, const TcParams& p
   cursor_normalize(c, p, n_my, j);
 }
 
+template <int GM>
 __device__ __forceinline__ void dequant_step(const TcParams& p, const uint8_t* slot, int ks, int lane,
                                              uint32_t (&r)[16]) {
-  if (ks < p.ks_core) dequant_residual(p, slot, ks, lane, r);
+  if (ks < p.ks_core) dequant_residual<GM>(slot, p.sc_res, lane, r);
   else if (ks < p.ks_corr) dequant_core(p, slot, lane, r);
   else dequant_corr(p, slot, 2 * (ks - p.ks_corr) + 1 < p.n_A, lane, r);
 }
@@ -232,8 +251,8 @@ __device__ __forceinline__ void dequant_step(const TcParams& p, const uint8_t* s
 // packed bytes of one stage (two k-steps), filled R - 1 stages ahead with
 // 16-byte cp.async per lane.  (One bulk copy per piece, issued by one lane,
 // measured slower: the copy engine queues many 512-byte copies.)
-template <int R>
-__device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int w, int lane) {
+template <int R, int GM>
+__device__ void dequant_loop(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int w, int lane) {
   constexpr uint32_t kPair = 2 * kTcSlotBytes;
   const int j = 2 * (w & 3) + ((w >> 2) & 1);
   const int par = w >> 3;
@@ -241,19 +260,23 @@ __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_
   const uint8_t* ring = sm.rings + static_cast<size_t>(w) * R * kPair;
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
-  const long total = static_cast<long>(n_my) * p.n_st;   // global stages of this CTA
+  const int total = n_my * p.n_st;   // global stages of this CTA
 
   // Prefetch R - 1 of this warp's stages ahead.
   StageCursor pc{0, par, unit_block(p, 0, n_my, j)};
   cursor_normalize(pc, p, n_my, j);
-  long pg = par;
+  int pg = par;
   uint32_t pslot = 0;
   auto issue_next = [&]() {
     if (pg < total && pc.blk != nullptr) {
       const uint32_t dst = ring_s + pslot * kPair;
       const int ks0 = 2 * pc.st;
-      issue_step(p, dst, pc.blk, ks0, lane);
-      if (ks0 + 1 < p.n_ks) issue_step(p, dst + kTcSlotBytes, pc.blk, ks0 + 1, lane);
+      if (ks0 + 1 < p.ks_core) {
+        issue_res_stage<GM>(p, dst, pc.blk, ks0, lane);
+      } else {
+        issue_step(p, dst, pc.blk, ks0, lane);
+        if (ks0 + 1 < p.n_ks) issue_step(p, dst + kTcSlotBytes, pc.blk, ks0 + 1, lane);
+      }
     }
     cp_async_commit();
     if (pg < total) {
@@ -271,7 +294,7 @@ __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_
   int s = par;
   uint32_t ph = 0;
   uint32_t slot_i = 0;
-  for (long g = par; g < total; g += 2) {
+  for (int g = par; g < total; g += 2) {
     issue_next();   // into the slot the previous stage freed
     if (!tc_wait_warp(sm, &sm.empty[s], ph ^ 1u, p.status)) break;
     tc_fence_after();
@@ -280,20 +303,31 @@ __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_
     __syncwarp();
     const int ks0 = 2 * c.st;
     const bool two = ks0 + 1 < p.n_ks;
-    uint32_t r0[16], r1[16];
-    if (c.blk == nullptr) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
-    } else if (two && ks0 + 1 < p.ks_core) {
-      dequant_residual(p, slot, ks0, lane, r0);   // the common case: both k-steps residual
-      dequant_residual(p, slot + kTcSlotBytes, ks0 + 1, lane, r1);
-    } else {
-      dequant_step(p, slot, ks0, lane, r0);
-      if (two) dequant_step(p, slot + kTcSlotBytes, ks0 + 1, lane, r1);
-    }
     const uint32_t ta = tmem_row + static_cast<uint32_t>(s) * 64u;
-    tmem_st_16x256b_x4(ta, r0);
-    if (two) tmem_st_16x256b_x4(ta + 32u, r1);
+    // One k-step at a time into TMEM (a store reads its registers when it
+    // issues), so only one k-step's 16 result registers are live.
+    if (c.blk == nullptr) {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) r[i] = 0u;
+      tmem_st_16x256b_x4(ta, r);
+      if (two) tmem_st_16x256b_x4(ta + 32u, r);
+    } else if (two && ks0 + 1 < p.ks_core) {   // the common case: both k-steps residual
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r[16];
+        dequant_residual<GM>(slot + h * kTcSlotBytes, p.sc_res, lane, r);
+        tmem_st_16x256b_x4(ta + 32u * h, r);
+      }
+    } else {
+      uint32_t r[16];
+      dequant_step<GM>(p, slot, ks0, lane, r);
+      tmem_st_16x256b_x4(ta, r);
+      if (two) {
+        dequant_step<GM>(p, slot + kTcSlotBytes, ks0 + 1, lane, r);
+        tmem_st_16x256b_x4(ta + 32u, r);
+      }
+    }
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();   // every lane is done reading the slot and storing to TMEM
@@ -307,6 +341,13 @@ __device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_
     }
   }
   cp_async_wait_all();
+}
+
+template <int R>
+__device__ void dequant_warp(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int w, int lane) {
+  if (p.g_log2 >= 6) dequant_loop<R, 0>(p, sm, tmem_base, w, lane);
+  else if (p.g_log2 == 5) dequant_loop<R, 1>(p, sm, tmem_base, w, lane);
+  else dequant_loop<R, 2>(p, sm, tmem_base, w, lane);
 }
 
 // ---------------------------------------------------------------- TMA warp
@@ -500,6 +541,8 @@ __device__ void epilogue_warps(const TcParams& p, const TcSmem& sm, uint32_t tme
 
 }  // namespace
 
+// 22 warps: an SM sub-partition holds up to six of them, and its 16,384
+// registers allow 80 per thread.
 template <int R>
 __global__ void __launch_bounds__(kTcWarps * 32, 1)
     tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap xmap) {
