@@ -120,10 +120,9 @@ ARCHEAD_API int archead_pack_image(const archead_desc* desc, const archead_host_
 /* Which kernel a forward call with T tokens runs its vocabulary pass on:
  *   ARCHEAD_KERNEL_DECODE        the streaming decode kernel (up to 8 tokens
  *                                per launch, mma.sync fragments in registers);
- *   ARCHEAD_KERNEL_TENSOR_CORE   the tcgen05 kernel (T >= 17, or T >= 13 when
- *                                d < 4096; and g_B a multiple of 64): weights
- *                                dequantised into tensor memory, 128 rows x up
- *                                to 128 tokens per unit.
+ *   ARCHEAD_KERNEL_TENSOR_CORE   the tcgen05 kernel (T >= 9 and g_B a multiple
+ *                                of 64): weights dequantised into tensor
+ *                                memory, 128 rows x up to 128 tokens per unit.
  * Both compute Eq. 7 of §3.2; -1 if handle is null or T <= 0.  (A library
  * query with no counterpart in the paper.) */
 enum { ARCHEAD_KERNEL_DECODE = 0, ARCHEAD_KERNEL_TENSOR_CORE = 1 };

@@ -1,8 +1,7 @@
 // Forward entry points of the C ABI (include/archead.h): argument checks,
 // workspace carving, and one of two launch sequences on the caller's stream,
 // with no host synchronisation:
-//   T < tc_min_tokens() (17 for d >= 4096, else 13; any T when g_B is not a
-//   multiple of 64):
+//   T < kTcMinTokens (9; any T when g_B is not a multiple of 64):
 //     prologue (z_c, z_r, E_t)  ->  decode launches of <= 8 tokens each
 //   otherwise:
 //     activation operand [h | z_c | z_r]  ->  tensor-core pass  ->  per-token fold

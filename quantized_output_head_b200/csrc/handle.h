@@ -31,20 +31,12 @@ struct archead_handle {
 
 namespace archead {
 
-// Calls with at least tc_min_tokens() tokens take the tensor-core path when
-// the shape allows it; smaller ones the decode kernel, which streams the whole
-// head once per 8 tokens.  Two decode launches beat one tensor-core launch
-// (up to 16 tokens) only when every residual warp has its full 256 columns of
-// d (d >= 4096: Qwen-shaped head, 13 / 16 tokens 266 / 286 us against ~297);
-// on narrower heads each decode launch streams slower (d = 2560: 0.44 of HBM
-// against 0.50) and one decode launch is the limit (16 tokens: 330 us against
-// 306 us on the tensor cores).
-constexpr int kFullWidthD = 4096;
-constexpr int kTcMinTokensNarrow = 13;
-inline int tc_min_tokens(const archead_handle& h) {
-  return h.L.d >= kFullWidthD ? kTcMinTokens : kTcMinTokensNarrow;
-}
-inline bool use_tc(const archead_handle& h, int T) { return h.tc_ok && T >= tc_min_tokens(h); }
+// Calls with at least kTcMinTokens tokens take the tensor-core path when the
+// shape allows it; smaller ones the decode kernel, which streams the whole
+// head once per 8 tokens.  At the Qwen shape one decode launch (8 tokens)
+// takes ~125 us and the tensor-core pass ~177 us for any count up to 128, so
+// a second decode launch (9-16 tokens: 214-286 us) loses to it.
+inline bool use_tc(const archead_handle& h, int T) { return h.tc_ok && T >= kTcMinTokens; }
 
 // K columns of the tensor-core path: d + r_c' + r_r' rounded up to 64.
 inline int tc_kc(const Layout& L) { return L.d + L.rcp + static_cast<int>(round_up(L.rrp, 64)); }

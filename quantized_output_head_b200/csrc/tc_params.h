@@ -23,7 +23,7 @@ constexpr int kTcSmemBudget = 232448; // dynamic shared memory a block may use o
 constexpr int kTcSlotBytes = 1056;    // one packed k-step of one m-tile block (codes + scales)
 constexpr int kTcDeqWarps = 16;       // two per m-tile block of a unit (even / odd k-steps)
 constexpr int kTcWarps = 22;          // 16 dequantising, 1 TMA, 1 MMA, 4 epilogue
-constexpr int kTcMinTokens = 17;      // calls with fewer tokens take the decode kernel (up to two launches)
+constexpr int kTcMinTokens = 9;       // calls with fewer tokens take the decode kernel (one launch)
 
 struct TcParams {
   const uint8_t* mtiles;      // arena: m-tile blocks

@@ -114,13 +114,12 @@ def test_qwen_decode_T1_fused(qwen):
     check_argmax(am.cpu().numpy(), qwen["y1"], qwen["tol1"])
 
 
-@pytest.mark.parametrize("T", sorted(set(gen.SWEEP_T) | {13, 16, 17}))
+@pytest.mark.parametrize("T", sorted(set(gen.SWEEP_T) | {9, 16, 17}))
 def test_qwen_decode_sweep_fused(qwen, T):
-    """Config 3's token counts, plus the wide-head dispatch boundary: 13 and 16
-    tokens take two decode launches, 17 the tensor-core kernel."""
+    """Config 3's token counts, plus the dispatch boundary: up to 8 tokens take
+    one decode launch, 9 and more the tensor-core kernel."""
     head = qwen["head"]
-    if T in (13, 16, 17):
-        assert head.forward_kernel(T) == ("decode" if T <= 16 else "tensor_core")
+    assert head.forward_kernel(T) == ("decode" if T <= 8 else "tensor_core")
     h, tg = qwen["h64"][:T], qwen["t64"][:T]
     lse, am, ce = head.lse_argmax(_dev_hidden(h), torch.from_numpy(tg))
     y, tol = qwen["y64"][:T], qwen["tol64"][:T]
@@ -236,7 +235,7 @@ def test_small_shapes(qoh, V, d, r_c, r_r, g, g_B, T):
     assert np.array_equal(am.cpu().numpy(), am2.cpu().numpy())
 
 
-# Calls of >= 13 tokens (>= 17 when d >= 4096) take the tensor-core kernel when g_B is a multiple of 64.
+# Calls of >= 9 tokens take the tensor-core kernel when g_B is a multiple of 64.
 SMALL_TC = [
     # V,    d,   r_c, r_r, g,   g_B, T
     (1000, 320, 32, 8, 64, 64, 17),       # ragged vocabulary, one 32-column correction chunk
@@ -244,9 +243,9 @@ SMALL_TC = [
     (1500, 512, 64, 0, 32, 64, 130),      # no correction, g = 32, two token tiles
     (4099, 512, 128, 64, 256, 128, 40),   # g = 256, last 128-row tile nearly empty
     (300, 128, 64, 32, 128, 128, 200),    # three 128-row tiles, the last partial
-    (777, 192, 64, 64, 64, 64, 13),       # fewest tokens of the tensor-core path (d < 4096), odd k-step count
-    (777, 192, 64, 64, 64, 64, 12),       # most tokens of the decode kernel on a narrow head (two launches)
-    (1003, 320, 100, 40, 16, 10, 20),     # g_B = 10: 13+ tokens through the decode kernel
+    (777, 192, 64, 64, 64, 64, 9),        # fewest tokens of the tensor-core path, odd k-step count
+    (777, 192, 64, 64, 64, 64, 8),        # most tokens of the decode kernel (one launch)
+    (1003, 320, 100, 40, 16, 10, 20),     # g_B = 10: 9+ tokens through the decode kernel (three launches)
 ]
 
 
