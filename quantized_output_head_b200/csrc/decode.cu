@@ -47,6 +47,7 @@ namespace archead {
 namespace {
 
 constexpr int kGroupTile = 8;    // m-tiles x tokens per partial-logit group (mg * nt)
+constexpr int kMergeLoads = 8;   // partials a lane of the last block loads at once (grids up to 256 blocks in one round)
 
 struct SmemView {
   uint8_t* rings;                // per compute warp: kRing slices
@@ -295,6 +296,27 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
   const uint8_t* g_scales = base + p.off_sres + rs.grp0 * kSresGroupBytes + lane * 16;
   const bool scale_lane = lane * 16 < rs.ng * kSresGroupBytes;
   const bool full = rs.nchunks == kCRes;
+  // The residual warps read every column of h between them, so they find E_t
+  // (max|h_t| < 2^E_t, the same value the prologue computes) without waiting
+  // for the prologue: a max over each warp's columns, then over the warps.
+  // The h loads go out first, ahead of the ring's copies, so E_t is known by
+  // the time the first m-tile has landed.
+  const bool tok = gr < p.nt;
+  const uint16_t* hrow = p.hidden + static_cast<size_t>(p.t0 + (tok ? gr : 0)) * p.d;
+  uint32_t hf[kCRes][4][2];   // bf16 pairs of this warp's columns, then fp16 fragments
+#pragma unroll
+  for (int c = 0; c < kCRes; ++c) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint32_t bits = 0u;
+        if (tok && c < rs.nchunks)
+          bits = *reinterpret_cast<const uint32_t*>(hrow + (rs.chunk0 + c) * kResChunkK + s * 16 + 2 * (lane & 3) + 8 * j);
+        hf[c][s][j] = bits;
+      }
+    }
+  }
   // Start streaming before the prologue's results are needed.
 #pragma unroll
   for (int k = 0; k < kRing; ++k) {
@@ -306,27 +328,16 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
   }
   g_codes += kRing * stride;
   g_scales += kRing * stride;
-  // The residual warps read every column of h between them, so they find E_t
-  // (max|h_t| < 2^E_t, the same value the prologue computes) without waiting
-  // for the prologue: a max over each warp's columns, then over the warps.
-  const bool tok = gr < p.nt;
-  const uint16_t* hrow = p.hidden + static_cast<size_t>(p.t0 + (tok ? gr : 0)) * p.d;
-  uint32_t hf[kCRes][4][2];   // bf16 pairs of this warp's columns, then fp16 fragments
   float mx = 0.f;
 #pragma unroll
-  for (int c = 0; c < kCRes; ++c) {
+  for (int c = 0; c < kCRes; ++c)
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < 4; ++s)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        uint32_t bits = 0u;
-        if (tok && c < rs.nchunks)
-          bits = *reinterpret_cast<const uint32_t*>(hrow + (rs.chunk0 + c) * kResChunkK + s * 16 + 2 * (lane & 3) + 8 * j);
-        hf[c][s][j] = bits;
+        const uint32_t bits = hf[c][s][j];
         mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(bits << 16)), fabsf(__uint_as_float(bits & 0xFFFF0000u))));
       }
-    }
-  }
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   if ((lane & 3) == 0) sv.hmax[wres * kDecodeTokens + gr] = mx;
@@ -789,22 +800,37 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
   if (prev != gridDim.x - 1) return;
 
   // Last block: merge the per-block partials of every token of this launch.
+  // A lane issues all of its loads of a round (kMergeLoads partials) before
+  // merging any, so a 148-block grid costs one L2 round trip, not five.
   __threadfence();
+  const int nblk = static_cast<int>(gridDim.x);
   for (int t = 0; t < p.nt; ++t) {
     const float4* part = p.partials + static_cast<size_t>(p.t0 + t) * gridDim.x;
     LseState a = lse_init();
-    for (int b = lane; b < static_cast<int>(gridDim.x); b += 32) {
-      const float4 q = __ldcg(part + b);
-      a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
+    for (int b0 = 0; b0 < nblk; b0 += 32 * kMergeLoads) {
+      float4 q[kMergeLoads];
+#pragma unroll
+      for (int u = 0; u < kMergeLoads; ++u) {
+        const int b = b0 + lane + 32 * u;
+        q[u] = b < nblk ? __ldcg(part + b) : make_float4(-INFINITY, 0.f, __int_as_float(0x7fffffff), 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kMergeLoads; ++u) a = lse_merge(a, LseState{q[u].x, q[u].y, __float_as_int(q[u].z)});
     }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) a = lse_merge(a, lse_shfl_xor(a, m));
     if (p.sampled != nullptr) {
       const float2* sp = p.spart + static_cast<size_t>(p.t0 + t) * gridDim.x;
       PickState b = pick_init();
-      for (int blk = lane; blk < static_cast<int>(gridDim.x); blk += 32) {
-        const float2 q = __ldcg(sp + blk);
-        b = pick_merge(b, PickState{q.x, __float_as_int(q.y)});
+      for (int b0 = 0; b0 < nblk; b0 += 32 * kMergeLoads) {
+        float2 q[kMergeLoads];
+#pragma unroll
+        for (int u = 0; u < kMergeLoads; ++u) {
+          const int blk = b0 + lane + 32 * u;
+          q[u] = blk < nblk ? __ldcg(sp + blk) : make_float2(-INFINITY, __int_as_float(0x7fffffff));
+        }
+#pragma unroll
+        for (int u = 0; u < kMergeLoads; ++u) b = pick_merge(b, PickState{q[u].x, __float_as_int(q[u].y)});
       }
 #pragma unroll
       for (int m = 16; m >= 1; m >>= 1) b = pick_merge(b, pick_shfl_xor(b, m));
