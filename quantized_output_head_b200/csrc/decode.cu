@@ -47,7 +47,8 @@ namespace archead {
 namespace {
 
 constexpr int kGroupTile = 8;    // m-tiles x tokens per partial-logit group (mg * nt)
-constexpr int kMergeLoads = 8;   // partials a lane of the last block loads at once (grids up to 256 blocks in one round)
+constexpr int kMergeLoads = 5;   // partials per token a lane of the last block loads at once (grids up to 160 blocks in one round)
+constexpr int kMergeLoadsOne = 8;   // the same when one warp merges one token at a time
 
 struct SmemView {
   uint8_t* rings;                // per compute warp: kRing slices
@@ -58,7 +59,7 @@ struct SmemView {
   float2* pickstate;             // [kEpiWarps][kDecodeTokens] per-warp sampling states of the block
   float* hmax;                   // [kMaxDecodeWarps][kDecodeTokens] max|h_t| over each residual warp's columns
   uint64_t* stall;               // test hook: a barrier nothing arrives on
-  int* flags;                    // [0] abort
+  int* flags;                    // [0] abort, [1] this block merges the partials
 };
 
 __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams& p) {
@@ -685,6 +686,11 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
 // token, rows r and r + 1), so a lane keeps one running state and reads each
 // warp's region with one 8-byte load.
 static_assert(kGroupTile * 16 == 64 * kEpiWarps, "two elements per epilogue lane");
+// kShared: the last block merges on both epilogue warps (launches of three or
+// more tokens); otherwise on one.  Two instances, so that the code of one
+// path does not change the other's (the one-token kernel measured ~6 us slower
+// with both paths compiled into it).
+template <bool kShared>
 __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int ew, int lane) {
   const int e = 2 * (32 * ew + lane);
   LseState st = lse_init();
@@ -771,82 +777,187 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     }
   }
   named_bar_sync(1, kEpiWarps * 32);
-  if (ew != 0) return;
-  // The prologue resets the completion ticket, and the previous launch on this
-  // workspace must be done with it: wait for the preceding grid here.
-  grid_dependency_wait();
-  for (int t = 0; t < p.nt; ++t) {
-    LseState a = lse_init();
-    PickState b = pick_init();
+  if constexpr (!kShared) {
+    // One warp writes the block's partials, takes the ticket and, in the last
+    // block, merges.
+    if (ew != 0) return;
+    // The prologue resets the completion ticket, and the previous launch on this
+    // workspace must be done with it: wait for the preceding grid here.
+    grid_dependency_wait();
+    for (int t = 0; t < p.nt; ++t) {
+      LseState a = lse_init();
+      PickState b = pick_init();
 #pragma unroll
-    for (int w = 0; w < kEpiWarps; ++w) {
-      const float4 q = sv.tokstate[w * kDecodeTokens + t];
-      a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
-      const float2 r = sv.pickstate[w * kDecodeTokens + t];
-      b = pick_merge(b, PickState{r.x, __float_as_int(r.y)});
+      for (int w = 0; w < kEpiWarps; ++w) {
+        const float4 q = sv.tokstate[w * kDecodeTokens + t];
+        a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
+        const float2 r = sv.pickstate[w * kDecodeTokens + t];
+        b = pick_merge(b, PickState{r.x, __float_as_int(r.y)});
+      }
+      if (lane == 0) {
+        p.partials[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] =
+            make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
+        if (p.sampled != nullptr)
+          p.spart[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] = make_float2(b.z, __int_as_float(b.idx));
+      }
     }
-    if (lane == 0) {
-      p.partials[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] =
-          make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
-      if (p.sampled != nullptr)
-        p.spart[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] = make_float2(b.z, __int_as_float(b.idx));
+    __threadfence();
+    __syncwarp();
+    unsigned prev = 0;
+    if (lane == 0) prev = atomicAdd(p.counter, 1u);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev != gridDim.x - 1) return;
+
+    // Last block: merge the per-block partials of every token of this launch.
+    // A lane issues all of its loads of a round (kMergeLoadsOne partials) before
+    // merging any, so a 148-block grid costs one L2 round trip, not five.
+    __threadfence();
+    const int nblk = static_cast<int>(gridDim.x);
+    for (int t = 0; t < p.nt; ++t) {
+      const float4* part = p.partials + static_cast<size_t>(p.t0 + t) * gridDim.x;
+      LseState a = lse_init();
+      for (int b0 = 0; b0 < nblk; b0 += 32 * kMergeLoadsOne) {
+        float4 q[kMergeLoadsOne];
+#pragma unroll
+        for (int u = 0; u < kMergeLoadsOne; ++u) {
+          const int b = b0 + lane + 32 * u;
+          q[u] = b < nblk ? __ldcg(part + b) : make_float4(-INFINITY, 0.f, __int_as_float(0x7fffffff), 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kMergeLoadsOne; ++u) a = lse_merge(a, LseState{q[u].x, q[u].y, __float_as_int(q[u].z)});
+      }
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) a = lse_merge(a, lse_shfl_xor(a, m));
+      if (p.sampled != nullptr) {
+        const float2* sp = p.spart + static_cast<size_t>(p.t0 + t) * gridDim.x;
+        PickState b = pick_init();
+        for (int b0 = 0; b0 < nblk; b0 += 32 * kMergeLoadsOne) {
+          float2 q[kMergeLoadsOne];
+#pragma unroll
+          for (int u = 0; u < kMergeLoadsOne; ++u) {
+            const int blk = b0 + lane + 32 * u;
+            q[u] = blk < nblk ? __ldcg(sp + blk) : make_float2(-INFINITY, __int_as_float(0x7fffffff));
+          }
+#pragma unroll
+          for (int u = 0; u < kMergeLoadsOne; ++u) b = pick_merge(b, PickState{q[u].x, __float_as_int(q[u].y)});
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) b = pick_merge(b, pick_shfl_xor(b, m));
+        if (lane == 0) p.sampled[p.t0 + t] = b.idx;
+      }
+      if (lane == 0) {
+        const int tg = p.t0 + t;
+        const float lse = a.m + logf(a.s);
+        const int gidx = a.idx + p.row0;
+        // target logit when the target row is one of this head's rows
+        const int tl = p.targets != nullptr ? p.targets[tg] - p.row0 : -1;
+        const float tgt = (tl >= 0 && tl < p.V) ? __ldcg(p.tgt + tg) : __int_as_float(0x7fc00000);
+        if (p.lse != nullptr) p.lse[tg] = lse;
+        if (p.argmax != nullptr) p.argmax[tg] = gidx;
+        if (p.ce != nullptr) p.ce[tg] = lse - tgt;
+        if (p.shard_out != nullptr) p.shard_out[tg] = make_float4(lse, a.m, __int_as_float(gidx), tgt);
+      }
     }
+    if (lane == 0) *p.counter = 0u;
+    return;
   }
-  __threadfence();
-  __syncwarp();
-  unsigned prev = 0;
-  if (lane == 0) prev = atomicAdd(p.counter, 1u);
-  prev = __shfl_sync(0xffffffffu, prev, 0);
-  if (prev != gridDim.x - 1) return;
+  if (ew == 0) {
+    // The prologue resets the completion ticket, and the previous launch on
+    // this workspace must be done with it: wait for the preceding grid here.
+    grid_dependency_wait();
+    for (int t = 0; t < p.nt; ++t) {
+      LseState a = lse_init();
+      PickState b = pick_init();
+#pragma unroll
+      for (int w = 0; w < kEpiWarps; ++w) {
+        const float4 q = sv.tokstate[w * kDecodeTokens + t];
+        a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
+        const float2 r = sv.pickstate[w * kDecodeTokens + t];
+        b = pick_merge(b, PickState{r.x, __float_as_int(r.y)});
+      }
+      if (lane == 0) {
+        p.partials[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] =
+            make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
+        if (p.sampled != nullptr)
+          p.spart[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] = make_float2(b.z, __int_as_float(b.idx));
+      }
+    }
+    __threadfence();
+    __syncwarp();
+    unsigned prev = 0;
+    if (lane == 0) prev = atomicAdd(p.counter, 1u);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (lane == 0) sv.flags[1] = prev == gridDim.x - 1 ? 1 : 0;
+  }
+  named_bar_sync(1, kEpiWarps * 32);
+  if (*reinterpret_cast<volatile int*>(&sv.flags[1]) == 0) return;
 
   // Last block: merge the per-block partials of every token of this launch.
-  // A lane issues all of its loads of a round (kMergeLoads partials) before
-  // merging any, so a 148-block grid costs one L2 round trip, not five.
+  // The tokens are split over the epilogue warps, two per warp per round, and
+  // a lane issues all of its loads of a round before merging any, so a
+  // 148-block grid costs one L2 round trip per round (not one per partial).
   __threadfence();
   const int nblk = static_cast<int>(gridDim.x);
-  for (int t = 0; t < p.nt; ++t) {
-    const float4* part = p.partials + static_cast<size_t>(p.t0 + t) * gridDim.x;
-    LseState a = lse_init();
+  for (int tp = ew; tp < p.nt; tp += 2 * kEpiWarps) {
+    const int tq = tp + kEpiWarps;   // the round's second token (may be past nt)
+    const bool two = tq < p.nt;
+    const float4* part0 = p.partials + static_cast<size_t>(p.t0 + tp) * gridDim.x;
+    const float4* part1 = p.partials + static_cast<size_t>(p.t0 + (two ? tq : tp)) * gridDim.x;
+    LseState a0 = lse_init(), a1 = lse_init();
     for (int b0 = 0; b0 < nblk; b0 += 32 * kMergeLoads) {
-      float4 q[kMergeLoads];
+      float4 q0[kMergeLoads], q1[kMergeLoads];
 #pragma unroll
       for (int u = 0; u < kMergeLoads; ++u) {
         const int b = b0 + lane + 32 * u;
-        q[u] = b < nblk ? __ldcg(part + b) : make_float4(-INFINITY, 0.f, __int_as_float(0x7fffffff), 0.f);
+        const float4 none = make_float4(-INFINITY, 0.f, __int_as_float(0x7fffffff), 0.f);
+        q0[u] = b < nblk ? __ldcg(part0 + b) : none;
+        q1[u] = (two && b < nblk) ? __ldcg(part1 + b) : none;
       }
 #pragma unroll
-      for (int u = 0; u < kMergeLoads; ++u) a = lse_merge(a, LseState{q[u].x, q[u].y, __float_as_int(q[u].z)});
+      for (int u = 0; u < kMergeLoads; ++u) {
+        a0 = lse_merge(a0, LseState{q0[u].x, q0[u].y, __float_as_int(q0[u].z)});
+        a1 = lse_merge(a1, LseState{q1[u].x, q1[u].y, __float_as_int(q1[u].z)});
+      }
     }
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) a = lse_merge(a, lse_shfl_xor(a, m));
-    if (p.sampled != nullptr) {
-      const float2* sp = p.spart + static_cast<size_t>(p.t0 + t) * gridDim.x;
-      PickState b = pick_init();
-      for (int b0 = 0; b0 < nblk; b0 += 32 * kMergeLoads) {
-        float2 q[kMergeLoads];
+    for (int m = 16; m >= 1; m >>= 1) {
+      a0 = lse_merge(a0, lse_shfl_xor(a0, m));
+      a1 = lse_merge(a1, lse_shfl_xor(a1, m));
+    }
 #pragma unroll
-        for (int u = 0; u < kMergeLoads; ++u) {
-          const int blk = b0 + lane + 32 * u;
-          q[u] = blk < nblk ? __ldcg(sp + blk) : make_float2(-INFINITY, __int_as_float(0x7fffffff));
+    for (int k = 0; k < 2; ++k) {
+      const int t = k == 0 ? tp : tq;
+      if (k == 1 && !two) break;
+      const LseState a = k == 0 ? a0 : a1;
+      if (p.sampled != nullptr) {
+        const float2* sp = p.spart + static_cast<size_t>(p.t0 + t) * gridDim.x;
+        PickState b = pick_init();
+        for (int b0 = 0; b0 < nblk; b0 += 32 * kMergeLoads) {
+          float2 q[kMergeLoads];
+#pragma unroll
+          for (int u = 0; u < kMergeLoads; ++u) {
+            const int blk = b0 + lane + 32 * u;
+            q[u] = blk < nblk ? __ldcg(sp + blk) : make_float2(-INFINITY, __int_as_float(0x7fffffff));
+          }
+#pragma unroll
+          for (int u = 0; u < kMergeLoads; ++u) b = pick_merge(b, PickState{q[u].x, __float_as_int(q[u].y)});
         }
 #pragma unroll
-        for (int u = 0; u < kMergeLoads; ++u) b = pick_merge(b, PickState{q[u].x, __float_as_int(q[u].y)});
+        for (int m = 16; m >= 1; m >>= 1) b = pick_merge(b, pick_shfl_xor(b, m));
+        if (lane == 0) p.sampled[p.t0 + t] = b.idx;
       }
-#pragma unroll
-      for (int m = 16; m >= 1; m >>= 1) b = pick_merge(b, pick_shfl_xor(b, m));
-      if (lane == 0) p.sampled[p.t0 + t] = b.idx;
-    }
-    if (lane == 0) {
-      const int tg = p.t0 + t;
-      const float lse = a.m + logf(a.s);
-      const int gidx = a.idx + p.row0;
-      // target logit when the target row is one of this head's rows
-      const int tl = p.targets != nullptr ? p.targets[tg] - p.row0 : -1;
-      const float tgt = (tl >= 0 && tl < p.V) ? __ldcg(p.tgt + tg) : __int_as_float(0x7fc00000);
-      if (p.lse != nullptr) p.lse[tg] = lse;
-      if (p.argmax != nullptr) p.argmax[tg] = gidx;
-      if (p.ce != nullptr) p.ce[tg] = lse - tgt;
-      if (p.shard_out != nullptr) p.shard_out[tg] = make_float4(lse, a.m, __int_as_float(gidx), tgt);
+      if (lane == 0) {
+        const int tg = p.t0 + t;
+        const float lse = a.m + logf(a.s);
+        const int gidx = a.idx + p.row0;
+        // target logit when the target row is one of this head's rows
+        const int tl = p.targets != nullptr ? p.targets[tg] - p.row0 : -1;
+        const float tgt = (tl >= 0 && tl < p.V) ? __ldcg(p.tgt + tg) : __int_as_float(0x7fc00000);
+        if (p.lse != nullptr) p.lse[tg] = lse;
+        if (p.argmax != nullptr) p.argmax[tg] = gidx;
+        if (p.ce != nullptr) p.ce[tg] = lse - tgt;
+        if (p.shard_out != nullptr) p.shard_out[tg] = make_float4(lse, a.m, __int_as_float(gidx), tgt);
+      }
     }
   }
   if (lane == 0) *p.counter = 0u;
@@ -854,7 +965,7 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
 
 }  // namespace
 
-template <int G>
+template <int G, bool kShared>
 __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const SmemView sv = smem_view(smem, p);
@@ -873,7 +984,7 @@ __global__ void __launch_bounds__(kMaxDecodeWarps * 32, 1) decode_kernel(const D
   __syncthreads();
 
   if (warp < kEpiWarps) {
-    epilogue_warp(p, sv, n_my, warp, lane);
+    epilogue_warp<kShared>(p, sv, n_my, warp, lane);
     return;
   }
   const int cw = warp - kEpiWarps;
@@ -907,23 +1018,28 @@ size_t decode_smem_bytes(const DecodeParams& p) {
 
 namespace {
 template <int G>
-const void* kernel_ptr() {
-  return reinterpret_cast<const void*>(&decode_kernel<G>);
+const void* kernel_ptr(bool shared) {
+  return shared ? reinterpret_cast<const void*>(&decode_kernel<G, true>)
+                : reinterpret_cast<const void*>(&decode_kernel<G, false>);
 }
-const void* kernel_for(int g_steps) {
+const void* kernel_for(int g_steps, bool shared) {
   switch (g_steps) {
-    case 1: return kernel_ptr<1>();
-    case 2: return kernel_ptr<2>();
-    case 4: return kernel_ptr<4>();
-    case 8: return kernel_ptr<8>();
-    default: return kernel_ptr<16>();
+    case 1: return kernel_ptr<1>(shared);
+    case 2: return kernel_ptr<2>(shared);
+    case 4: return kernel_ptr<4>(shared);
+    case 8: return kernel_ptr<8>(shared);
+    default: return kernel_ptr<16>(shared);
   }
 }
 }  // namespace
 
 cudaError_t decode_set_attributes(int g_steps, size_t smem) {
-  return cudaFuncSetAttribute(kernel_for(g_steps), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(kernel_for(g_steps, false), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kernel_for(g_steps, true), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+  return e;
 }
 
 cudaError_t launch_decode(int g_steps, const DecodeParams& p, int grid, size_t smem, cudaStream_t stream) {
@@ -938,7 +1054,7 @@ cudaError_t launch_decode(int g_steps, const DecodeParams& p, int grid, size_t s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   void* args[] = {const_cast<DecodeParams*>(&p)};
-  return cudaLaunchKernelExC(&cfg, kernel_for(g_steps), args);
+  return cudaLaunchKernelExC(&cfg, kernel_for(g_steps, p.nt > 2), args);
 }
 
 }  // namespace archead
