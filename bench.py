@@ -635,21 +635,18 @@ def main():
         if op["logits"]:
             outs = (torch.empty((T, shape.V), dtype=torch.float32).pin_memory().numpy(),
                     torch.empty(T, dtype=torch.int32).pin_memory().numpy())
-
-            def e2e_call():
-                head.logits_host(hh, outs)
+            e2e_call = head.prepare_logits_host(hh, outs)
             h2d, d2h = T * shape.d * 2, T * shape.V * 4 + 4 * T
-            what = "archead_logits_host (host buffers, fp32 logits + argmax)"
+            what = "archead_logits_host (host buffers, fp32 logits + argmax; prepared call)"
         else:
             outs = (torch.empty(T, dtype=torch.float32).pin_memory().numpy(),
                     torch.empty(T, dtype=torch.int32).pin_memory().numpy(),
                     torch.empty(T, dtype=torch.float32).pin_memory().numpy() if op["ce"] else None)
-
-            def e2e_call():
-                head.lse_argmax_host(hh, th if op["ce"] else None, outs)
+            e2e_call = head.prepare_lse_argmax_host(hh, th if op["ce"] else None, outs)
             h2d = T * shape.d * 2 + (4 * T if op["ce"] else 0)
             d2h = 4 * T * (2 + (1 if op["ce"] else 0))
-            what = "archead_lse_argmax_host (host buffers, lse + argmax" + (" + ce)" if op["ce"] else ")")
+            what = ("archead_lse_argmax_host (host buffers, lse + argmax" + (" + ce" if op["ce"] else "") +
+                    "; prepared call)")
         for _ in range(3):
             e2e_call()
         e_steps = max(10, min(args.steps, 2000))

@@ -265,6 +265,33 @@ class PackedHead:
                                         _stream_ptr(stream)), "archead_logits_host")
         return lg, am
 
+    def prepare_logits_host(self, hidden_host: np.ndarray, out: Tuple[Optional[np.ndarray], Optional[np.ndarray]],
+                            stream: Optional[torch.cuda.Stream] = None):
+        """archead_logits_host bound to fixed host buffers (pinned memory lets
+        the library replay one captured launch sequence): returns a callable
+        that runs the call again on the current contents of those buffers.
+        The buffers, the workspace and the stream are resolved once here."""
+        hb = np.ascontiguousarray(hidden_host).view(np.uint16)
+        T = int(hb.shape[0])
+        lg, am = out
+        ws = self.workspace(T, host_form="logits")
+        args = (self.handle, hb.ctypes.data, T, None if lg is None else lg.ctypes.data,
+                None if am is None else am.ctypes.data, ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+        return _bound_call(_lib.archead_logits_host, args, (hb, lg, am, ws), "archead_logits_host")
+
+    def prepare_lse_argmax_host(self, hidden_host: np.ndarray, targets_host: Optional[np.ndarray],
+                                out: Tuple[np.ndarray, np.ndarray, Optional[np.ndarray]],
+                                stream: Optional[torch.cuda.Stream] = None):
+        """archead_lse_argmax_host bound to fixed host buffers; see prepare_logits_host."""
+        hb = np.ascontiguousarray(hidden_host).view(np.uint16)
+        T = int(hb.shape[0])
+        tg = None if targets_host is None else np.ascontiguousarray(targets_host, dtype=np.int32)
+        lse, am, ce = out
+        ws = self.workspace(T, host_form=True)
+        args = (self.handle, hb.ctypes.data, T, None if tg is None else tg.ctypes.data, lse.ctypes.data,
+                am.ctypes.data, None if ce is None else ce.ctypes.data, ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+        return _bound_call(_lib.archead_lse_argmax_host, args, (hb, tg, lse, am, ce, ws), "archead_lse_argmax_host")
+
     def sample(self, hidden: torch.Tensor, temperature: float, seed: int, offset: int = 0):
         """Gumbel-max temperature sampling fused into the vocabulary pass: returns
         (sampled [T] int32, lse [T], argmax [T]) of this head's rows; token t
@@ -325,6 +352,17 @@ class PackedHead:
         if rc not in (ARCHEAD_OK, ARCHEAD_ETIMEOUT):
             _check(rc, "archead_workspace_status")
         return int(v.value)
+
+
+def _bound_call(fn, args, keep, what):
+    """A no-argument call of `fn(*args)` that raises on a non-OK status; `keep`
+    holds the buffers the arguments point into."""
+    def call():
+        rc = fn(*args)
+        if rc != ARCHEAD_OK:
+            raise ArcheadError(rc, what)
+    call.buffers = keep
+    return call
 
 
 # ------------------------------------------------------- vocabulary shards

@@ -12,6 +12,8 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
+#include <new>
 
 #include "handle.h"
 
@@ -267,6 +269,107 @@ int set_cuda_error(cudaError_t e) {
   return ARCHEAD_ECUDA;
 }
 
+// ---------------------------------------------------- host-buffer sequences
+// A host-buffer call is a fixed sequence (copies in, the forward launches,
+// copies out).  When every host buffer is pinned, the sequence is captured
+// once per distinct argument set on a private stream and replayed with one
+// graph launch on the caller's stream: one driver call instead of five to
+// seven, so the GPU runs the steps back to back.  Any capture failure falls
+// back to the direct sequence (and is remembered for that argument set).
+struct HostGraphKey {
+  int kind, T;
+  const void* in[2];
+  void* out[3];
+  void* ws;
+  size_t ws_bytes;
+  bool operator==(const HostGraphKey& o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
+};
+
+struct HostGraphCache {
+  static constexpr int kEntries = 4;
+  std::mutex mu;
+  cudaStream_t cap = nullptr;   // capture stream (non-blocking), created on first use
+  struct Entry {
+    bool used = false, failed = false;
+    HostGraphKey key{};
+    cudaGraphExec_t exec = nullptr;
+  } e[kEntries];
+  int next = 0;
+};
+
+HostGraphCache* host_graph_cache_new() { return new (std::nothrow) HostGraphCache(); }
+
+void host_graph_cache_free(HostGraphCache* c) {
+  if (c == nullptr) return;
+  for (auto& en : c->e)
+    if (en.exec != nullptr) cudaGraphExecDestroy(en.exec);
+  if (c->cap != nullptr) cudaStreamDestroy(c->cap);
+  delete c;
+}
+
+namespace {
+
+bool pinned(const void* p) {
+  if (p == nullptr) return true;
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+// Runs `enqueue` through the cache: a replay, or a capture then a replay.
+// Returns ARCHEAD_OK with the sequence launched on `s`, kNoGraph when the
+// caller should run the direct sequence, or an error.
+constexpr int kNoGraph = 1;
+template <class F>
+int via_graph(const archead_handle* h, const HostGraphKey& key, cudaStream_t s, F enqueue) {
+  HostGraphCache* c = h->graphs;
+  if (c == nullptr || h->ev_before != nullptr) return kNoGraph;   // profiling events are per call
+  std::lock_guard<std::mutex> lock(c->mu);
+  for (auto& en : c->e) {
+    if (en.used && en.key == key) {
+      if (en.failed) return kNoGraph;
+      const cudaError_t e = cudaGraphLaunch(en.exec, s);
+      return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
+    }
+  }
+  HostGraphCache::Entry& en = c->e[c->next];
+  c->next = (c->next + 1) % HostGraphCache::kEntries;
+  if (en.exec != nullptr) cudaGraphExecDestroy(en.exec);
+  en = HostGraphCache::Entry{};
+  en.used = true;
+  en.key = key;
+  en.failed = true;
+  if (c->cap == nullptr && cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking) != cudaSuccess) {
+    c->cap = nullptr;
+    cudaGetLastError();
+    return kNoGraph;
+  }
+  cudaGraph_t g = nullptr;
+  if (cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaGetLastError();
+    return kNoGraph;
+  }
+  const int rc = enqueue(c->cap);
+  const cudaError_t ee = cudaStreamEndCapture(c->cap, &g);
+  cudaGetLastError();   // a capture that failed leaves no sticky error; clear the record
+  if (rc == ARCHEAD_OK && ee == cudaSuccess && g != nullptr &&
+      cudaGraphInstantiate(&en.exec, g, 0) == cudaSuccess) {
+    en.failed = false;
+  } else {
+    en.exec = nullptr;
+    cudaGetLastError();
+  }
+  if (g != nullptr) cudaGraphDestroy(g);
+  if (en.failed) return kNoGraph;
+  const cudaError_t e = cudaGraphLaunch(en.exec, s);
+  return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
+}
+
+}  // namespace
+
 }  // namespace archead
 
 using namespace archead;
@@ -315,6 +418,8 @@ extern "C" ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle,
   if (!aligned(workspace, 256)) return ARCHEAD_EALIGN;
   const WsLayout w = ws_layout(*handle, T);
   if (workspace_bytes < w.host_total) return ARCHEAD_ENOMEM;
+  const int dc = check_device(handle);
+  if (dc != ARCHEAD_OK) return dc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* wb = static_cast<uint8_t*>(workspace);
   uint16_t* d_hidden = reinterpret_cast<uint16_t*>(wb + w.h_hidden);
@@ -323,18 +428,27 @@ extern "C" ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle,
   int32_t* d_argmax = reinterpret_cast<int32_t*>(wb + w.h_argmax);
   float* d_ce = ce_host ? reinterpret_cast<float*>(wb + w.h_ce) : nullptr;
   const size_t t = static_cast<size_t>(T);
-  cudaError_t e = cudaMemcpyAsync(d_hidden, hidden_host, t * handle->L.d * 2, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess && d_targets)
-    e = cudaMemcpyAsync(d_targets, targets_host, t * 4, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return set_cuda_error(e);
-  const int rc = forward(handle, d_hidden, T, d_targets, nullptr, d_argmax, d_lse, d_ce, workspace, w.total, s);
+  auto enqueue = [&](cudaStream_t q) -> int {
+    cudaError_t e = cudaMemcpyAsync(d_hidden, hidden_host, t * handle->L.d * 2, cudaMemcpyHostToDevice, q);
+    if (e == cudaSuccess && d_targets) e = cudaMemcpyAsync(d_targets, targets_host, t * 4, cudaMemcpyHostToDevice, q);
+    if (e != cudaSuccess) return set_cuda_error(e);
+    const int rc = forward(handle, d_hidden, T, d_targets, nullptr, d_argmax, d_lse, d_ce, workspace, w.total, q);
+    if (rc != ARCHEAD_OK) return rc;
+    e = cudaMemcpyAsync(lse_host, d_lse, t * 4, cudaMemcpyDeviceToHost, q);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(argmax_host, d_argmax, t * 4, cudaMemcpyDeviceToHost, q);
+    if (e == cudaSuccess && ce_host) e = cudaMemcpyAsync(ce_host, d_ce, t * 4, cudaMemcpyDeviceToHost, q);
+    return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
+  };
+  int rc = kNoGraph;
+  if (pinned(hidden_host) && pinned(targets_host) && pinned(lse_host) && pinned(argmax_host) && pinned(ce_host)) {
+    const HostGraphKey key{0, T, {hidden_host, targets_host}, {lse_host, argmax_host, ce_host}, workspace,
+                           workspace_bytes};
+    rc = via_graph(handle, key, s, enqueue);
+  }
+  if (rc == kNoGraph) rc = enqueue(s);
   if (rc != ARCHEAD_OK) return rc;
-  e = cudaMemcpyAsync(lse_host, d_lse, t * 4, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(argmax_host, d_argmax, t * 4, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess && ce_host) e = cudaMemcpyAsync(ce_host, d_ce, t * 4, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return set_cuda_error(e);
-  return ARCHEAD_OK;
+  const cudaError_t e = cudaStreamSynchronize(s);
+  return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
 }
 
 extern "C" ARCHEAD_API size_t archead_host_logits_workspace_bytes(const archead_handle* handle, int32_t T) {
@@ -351,21 +465,33 @@ extern "C" ARCHEAD_API int archead_logits_host(const archead_handle* handle, con
   if (!aligned(workspace, 256)) return ARCHEAD_EALIGN;
   const WsLayout w = ws_layout(*handle, T);
   if (workspace_bytes < w.host_logits_total) return ARCHEAD_ENOMEM;
+  const int dc = check_device(handle);
+  if (dc != ARCHEAD_OK) return dc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* wb = static_cast<uint8_t*>(workspace);
   uint16_t* d_hidden = reinterpret_cast<uint16_t*>(wb + w.h_hidden);
   float* d_logits = logits_host ? reinterpret_cast<float*>(wb + w.h_logits) : nullptr;
   int32_t* d_argmax = argmax_host ? reinterpret_cast<int32_t*>(wb + w.h_argmax) : nullptr;
   const size_t t = static_cast<size_t>(T);
-  cudaError_t e = cudaMemcpyAsync(d_hidden, hidden_host, t * handle->L.d * 2, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return set_cuda_error(e);
-  const int rc = forward(handle, d_hidden, T, nullptr, d_logits, d_argmax, nullptr, nullptr, workspace, w.total, s);
+  auto enqueue = [&](cudaStream_t q) -> int {
+    cudaError_t e = cudaMemcpyAsync(d_hidden, hidden_host, t * handle->L.d * 2, cudaMemcpyHostToDevice, q);
+    if (e != cudaSuccess) return set_cuda_error(e);
+    const int rc = forward(handle, d_hidden, T, nullptr, d_logits, d_argmax, nullptr, nullptr, workspace, w.total, q);
+    if (rc != ARCHEAD_OK) return rc;
+    if (logits_host) e = cudaMemcpyAsync(logits_host, d_logits, t * handle->L.V * 4, cudaMemcpyDeviceToHost, q);
+    if (e == cudaSuccess && argmax_host) e = cudaMemcpyAsync(argmax_host, d_argmax, t * 4, cudaMemcpyDeviceToHost, q);
+    return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
+  };
+  int rc = kNoGraph;
+  if (pinned(hidden_host) && pinned(logits_host) && pinned(argmax_host)) {
+    const HostGraphKey key{1, T, {hidden_host, nullptr}, {logits_host, argmax_host, nullptr}, workspace,
+                           workspace_bytes};
+    rc = via_graph(handle, key, s, enqueue);
+  }
+  if (rc == kNoGraph) rc = enqueue(s);
   if (rc != ARCHEAD_OK) return rc;
-  if (logits_host) e = cudaMemcpyAsync(logits_host, d_logits, t * handle->L.V * 4, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess && argmax_host) e = cudaMemcpyAsync(argmax_host, d_argmax, t * 4, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return set_cuda_error(e);
-  return ARCHEAD_OK;
+  const cudaError_t e = cudaStreamSynchronize(s);
+  return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
 }
 
 extern "C" ARCHEAD_API int archead_sample(const archead_handle* handle, const uint16_t* hidden, int32_t T,

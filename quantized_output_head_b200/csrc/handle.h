@@ -8,6 +8,11 @@
 #include "params.h"
 #include "tc_params.h"
 
+namespace archead {
+struct HostGraphCache;
+}  // namespace archead
+using archead::HostGraphCache;
+
 struct archead_handle {
   archead::Layout L;
   const uint8_t* arena;     // device, not owned
@@ -27,6 +32,7 @@ struct archead_handle {
   cudaEvent_t ev_after;
   uint64_t wait_limit_ns;   // decode kernel: limit of every bounded wait (test hook; default kWaitLimitNs)
   int test_stall;           // decode kernel: test hook, a wait that nothing completes
+  struct HostGraphCache* graphs;   // host-buffer entry points: captured sequences (api.cu), owned
 };
 
 namespace archead {
@@ -111,5 +117,9 @@ cudaError_t launch_shard_merge(const float4* parts, int n, int T, float* lse, in
 
 // Thread-local record of the last CUDA error (api.cu).
 int set_cuda_error(cudaError_t e);
+
+// Cache of captured host-buffer call sequences of a handle (api.cu).
+HostGraphCache* host_graph_cache_new();
+void host_graph_cache_free(HostGraphCache* c);
 
 }  // namespace archead

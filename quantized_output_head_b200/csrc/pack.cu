@@ -321,6 +321,7 @@ extern "C" ARCHEAD_API int archead_pack_load(const archead_desc* desc, const arc
   h->v_total = L.V;
   h->wait_limit_ns = kWaitLimitNs;
   h->test_stall = 0;
+  h->graphs = nullptr;
   plan_tc(h, *comps, optin);
   e = decode_set_attributes(L.g_steps, static_cast<size_t>(optin));
   if (e == cudaSuccess && h->tc_ok) e = tc_set_attributes();
@@ -342,8 +343,17 @@ extern "C" ARCHEAD_API int archead_pack_load(const archead_desc* desc, const arc
     delete h;
     return set_cuda_error(e);
   }
+  h->graphs = host_graph_cache_new();
+  if (h->graphs == nullptr) {
+    delete h;
+    return ARCHEAD_ENOMEM;
+  }
   *out = h;
   return ARCHEAD_OK;
 }
 
-extern "C" ARCHEAD_API void archead_free(archead_handle* handle) { delete handle; }
+extern "C" ARCHEAD_API void archead_free(archead_handle* handle) {
+  if (handle == nullptr) return;
+  host_graph_cache_free(handle->graphs);
+  delete handle;
+}

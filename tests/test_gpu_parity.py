@@ -86,6 +86,42 @@ def test_cfg1_host_logits_entry_matches_device_entry(cfg1):
         head.logits_host(h_bits, out=(None, None))
 
 
+def _pinned(a):
+    t = torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    return t, t.numpy()
+
+
+def test_cfg1_host_entries_replay_with_pinned_buffers(cfg1):
+    """Pinned host buffers take the captured-sequence path (a capture on the
+    first call, a replay after it): new inputs in the same buffers give the
+    device entry points' results bit for bit, twice in a row, for both
+    host-buffer entry points and their prepared forms."""
+    head, h_bits, targets, y, tol = cfg1
+    T = h_bits.shape[0]
+    _, hh = _pinned(h_bits.view(np.int16))
+    _, th = _pinned(targets)
+    keep = [_pinned(np.zeros((T, head.V), np.float32)), _pinned(np.zeros(T, np.int32)),
+            _pinned(np.zeros(T, np.float32)), _pinned(np.zeros(T, np.int32)), _pinned(np.zeros(T, np.float32))]
+    lg, am, lse, am2, ce = [k[1] for k in keep]
+    logits_call = head.prepare_logits_host(hh, (lg, am))
+    lse_call = head.prepare_lse_argmax_host(hh, th, (lse, am2, ce))
+    rng = np.random.default_rng(3)
+    for rep in range(3):
+        src = h_bits if rep == 0 else np.roll(h_bits, rep, axis=1)   # new inputs into the same buffers
+        hh.view(np.uint16)[:] = src
+        th[:] = rng.integers(0, head.V, size=T, dtype=np.int32)
+        logits_call()
+        lse_call()
+        lg_d, am_d = head.logits(_dev_hidden(src))
+        lse_d, am2_d, ce_d = head.lse_argmax(_dev_hidden(src), torch.from_numpy(th.copy()))
+        assert np.array_equal(lg, lg_d.cpu().numpy()) and np.array_equal(am, am_d.cpu().numpy())
+        assert np.array_equal(lse, lse_d.cpu().numpy()) and np.array_equal(am2, am2_d.cpu().numpy())
+        assert np.array_equal(ce, ce_d.cpu().numpy())
+    # the unprepared forms with the same pinned buffers replay the same sequences
+    head.logits_host(hh, (lg, am))
+    assert np.array_equal(lg, lg_d.cpu().numpy())
+
+
 # ------------------------------------------------ Qwen-shaped head (2, 3, 5)
 @pytest.fixture(scope="module")
 def qwen(qoh):
