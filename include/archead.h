@@ -26,8 +26,10 @@
  *   - Return value: ARCHEAD_OK (0) or a negative ARCHEAD_E* code.  No C++
  *     exception crosses this boundary.
  *   - Device pointers are plain CUDA device addresses owned by the caller; the
- *     library allocates no device memory.  Host pointers are only read during
- *     the call (or, for the *_host entry point, until it returns).
+ *     library allocates no device memory (the host-buffer forms may keep
+ *     captured CUDA graphs and one stream per handle, driver resources that
+ *     archead_free releases).  Host pointers are only read during the call
+ *     (or, for the *_host entry points, until it returns).
  *   - Forward calls are asynchronous on the given stream and never synchronise
  *     the host (except archead_lse_argmax_host, which is the host-buffer form).
  *     A fault inside a kernel surfaces at the caller's next synchronisation.
@@ -164,7 +166,10 @@ ARCHEAD_API int archead_logits_lse_argmax(const archead_handle* handle, const ui
  * are HOST pointers (pinned memory recommended), copied to the device inside
  * the workspace; lse / argmax / ce are HOST pointers filled before return.
  * workspace must be >= archead_host_workspace_bytes(handle, T).  Synchronises
- * the stream. */
+ * the stream.  When every host buffer is pinned, the call's fixed sequence
+ * (copies in, the forward launches, copies out) is captured once per distinct
+ * set of arguments (the last four are kept per handle) and replayed with one
+ * graph launch; otherwise, or if the capture fails, it runs directly. */
 ARCHEAD_API size_t archead_host_workspace_bytes(const archead_handle* handle, int32_t T);
 ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint16_t* hidden_host,
                                         int32_t T, const int32_t* targets_host, float* lse_host,
@@ -177,7 +182,8 @@ ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint
  * return (either may be NULL, not both).  workspace (device, 256-byte
  * aligned) must be >= archead_host_logits_workspace_bytes(handle, T): it
  * stages the hidden states and the logits on the device.  Synchronises the
- * stream. */
+ * stream.  Pinned host buffers take the captured sequence as
+ * archead_lse_argmax_host does. */
 ARCHEAD_API size_t archead_host_logits_workspace_bytes(const archead_handle* handle, int32_t T);
 ARCHEAD_API int archead_logits_host(const archead_handle* handle, const uint16_t* hidden_host, int32_t T,
                                     float* logits_host, int32_t* argmax_host, void* workspace,
@@ -280,7 +286,8 @@ ARCHEAD_API int archead_set_profile_events(archead_handle* handle, void* before,
  * handle is NULL or wait_limit_ns is 0.  Restore with (2000000000, 0). */
 ARCHEAD_API int archead_test_decode_waits(archead_handle* handle, uint64_t wait_limit_ns, int stall);
 
-/* Free a handle (host memory only; the arena stays with the caller). */
+/* Free a handle and the captured sequences of its host-buffer calls (the arena
+ * stays with the caller). */
 ARCHEAD_API void archead_free(archead_handle* handle);
 
 /* The last cudaError_t seen by a call that returned ARCHEAD_ECUDA (thread-local). */
