@@ -18,17 +18,19 @@
 // block + grid, ...): every compute warp owns a fixed slice of every m-tile
 // block, so it streams its own bytes:
 //   residual warps    16 k16 steps of d each; their fp16 h fragments stay in
-//                     registers for the whole launch; between them they read
-//                     all of h, so they find each token's exponent E_t
-//                     themselves and start without waiting for the prologue
+//                     registers for the whole launch, each warp's columns
+//                     under a power of two of their own (from their own
+//                     maximum), so a warp starts as soon as its h and first
+//                     m-tile have landed, waiting for no other warp and not
+//                     for the prologue
 //   core warps        kCL 64-column chunks of r_c' each
 //   correction warps  kCA 32-column chunks of r_r' each (these and the core
 //                     warps wait for the prologue's z)
 // Residual and core warps take m-tiles in interleaved pairs (two independent
 // MMA chains).  Each compute warp prefetches its slice of the next kRing
 // m-tiles into a private shared-memory ring with cp.async (16 B per lane, L2
-// only) and waits only on its own copies: no producer warp and no block-wide
-// synchronisation.  After an m-tile the warp stores its 16 x nt partial logits
+// only, evict-first: the head is read once) and waits only on its own copies:
+// no producer warp and no block-wide synchronisation.  After an m-tile the warp stores its 16 x nt partial logits
 // in its own region of a slot and arrives on reduced[r].  Warps 0-1, the
 // epilogue, each take half of a slot's elements (two adjacent per lane), sum
 // the warps' regions in warp order (deterministic), push the logits into
@@ -55,9 +57,8 @@ struct SmemView {
   float* part;                   // [slots][nw_work][mg][nt][16 rows] per-warp partial logits
   uint64_t* reduced;             // [slots] compute warps -> epilogue warps
   uint64_t* redfree;             // [slots] epilogue warps -> compute warps
-  float4* tokstate;              // [kEpiWarps][kDecodeTokens] per-warp token states of the block
-  float2* pickstate;             // [kEpiWarps][kDecodeTokens] per-warp sampling states of the block
-  float* hmax;                   // [kMaxDecodeWarps][kDecodeTokens] max|h_t| over each residual warp's columns
+  float4* tokstate;              // [4 kEpiWarps] LSE state of each epilogue octet (q = 4 ew + lane / 8)
+  float2* pickstate;             // [4 kEpiWarps] sampling state of each epilogue octet
   uint64_t* stall;               // test hook: a barrier nothing arrives on
   int* flags;                    // [0] abort, [1] this block merges the partials
 };
@@ -70,8 +71,7 @@ __device__ __forceinline__ SmemView smem_view(uint8_t* smem, const DecodeParams&
   v.redfree = v.reduced + p.slots;
   v.tokstate = reinterpret_cast<float4*>(v.redfree + p.slots);
   v.pickstate = reinterpret_cast<float2*>(v.tokstate + kEpiWarps * kDecodeTokens);
-  v.hmax = reinterpret_cast<float*>(v.pickstate + kEpiWarps * kDecodeTokens);
-  v.stall = reinterpret_cast<uint64_t*>(v.hmax + kMaxDecodeWarps * kDecodeTokens);
+  v.stall = reinterpret_cast<uint64_t*>(v.pickstate + kEpiWarps * kDecodeTokens);
   v.flags = reinterpret_cast<int*>(v.stall + 1);
   return v;
 }
@@ -193,8 +193,8 @@ __device__ __forceinline__ void issue_res(uint32_t dst, const uint8_t* codes, co
                                           bool scale_lane) {
 #pragma unroll
   for (int c = 0; c < kCRes; ++c)
-    if (kFull || c < nchunks) cp_async16(dst + c * kResChunkBytes, codes + c * kResChunkBytes);
-  if (scale_lane) cp_async16(dst + kCRes * kResChunkBytes, scales);
+    if (kFull || c < nchunks) cp_async16_hint(dst + c * kResChunkBytes, codes + c * kResChunkBytes, l2_evict_first_policy());
+  if (scale_lane) cp_async16_hint(dst + kCRes * kResChunkBytes, scales, l2_evict_first_policy());
 }
 
 // One m-tile of a residual warp: 16 k16 steps over its 4 chunks, flushing
@@ -297,11 +297,11 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
   const uint8_t* g_scales = base + p.off_sres + rs.grp0 * kSresGroupBytes + lane * 16;
   const bool scale_lane = lane * 16 < rs.ng * kSresGroupBytes;
   const bool full = rs.nchunks == kCRes;
-  // The residual warps read every column of h between them, so they find E_t
-  // (max|h_t| < 2^E_t, the same value the prologue computes) without waiting
-  // for the prologue: a max over each warp's columns, then over the warps.
-  // The h loads go out first, ahead of the ring's copies, so E_t is known by
-  // the time the first m-tile has landed.
+  // Each warp scales its own columns of h_t by 2^(kScaleExp - E), with
+  // max|h_t| < 2^E over those columns: exact for bf16 inputs, and undone on
+  // the warp's fp32 partial sums (a power of two), so warps need not agree on
+  // E.  The h loads go out first, ahead of the ring's copies, so E is known
+  // by the time the first m-tile has landed.
   const bool tok = gr < p.nt;
   const uint16_t* hrow = p.hidden + static_cast<size_t>(p.t0 + (tok ? gr : 0)) * p.d;
   uint32_t hf[kCRes][4][2];   // bf16 pairs of this warp's columns, then fp16 fragments
@@ -341,14 +341,10 @@ __device__ void residual_warp(const DecodeParams& p, const SmemView& sv, int n_m
       }
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  if ((lane & 3) == 0) sv.hmax[wres * kDecodeTokens + gr] = mx;
-  named_bar_sync(2, p.nw_res * 32);
   float hs = 0.f;
   if (tok) {
-    float m = 0.f;
-    for (int w = 0; w < p.nw_res; ++w) m = fmaxf(m, sv.hmax[w * kDecodeTokens + gr]);
     int E = 0;
-    frexpf(m, &E);
+    frexpf(mx, &E);
     hs = ldexpf(1.f, kScaleExp - E);
   }
   // fp16 h fragments of this warp's columns, and the constant-part sum of each
@@ -453,9 +449,9 @@ __device__ __forceinline__ void issue_core(uint32_t dst, const uint8_t* g_nib, c
                                            const uint8_t* g_sl, int nch, bool hi_lane, bool sl_lane) {
 #pragma unroll
   for (int c = 0; c < kCL; ++c)
-    if (c < nch) cp_async16(dst + c * kLNibChunkBytes, g_nib + c * kLNibChunkBytes);
-  if (hi_lane) cp_async16(dst + kCL * kLNibChunkBytes, g_hi);
-  if (sl_lane) cp_async16(dst + kCL * (kLNibChunkBytes + kLHiChunkBytes), g_sl);
+    if (c < nch) cp_async16_hint(dst + c * kLNibChunkBytes, g_nib + c * kLNibChunkBytes, l2_evict_first_policy());
+  if (hi_lane) cp_async16_hint(dst + kCL * kLNibChunkBytes, g_hi, l2_evict_first_policy());
+  if (sl_lane) cp_async16_hint(dst + kCL * (kLNibChunkBytes + kLHiChunkBytes), g_sl, l2_evict_first_policy());
 }
 
 // One core chunk (4 k16 steps, fp16 pair hi + lo of z) of one m-tile slot into acc.
@@ -597,8 +593,8 @@ __device__ __forceinline__ void issue_corr(uint32_t dst, const uint8_t* g_codes,
                                            bool sa_lane) {
 #pragma unroll
   for (int c = 0; c < kCA; ++c)
-    if (c < nch) cp_async16(dst + c * kAChunkBytes, g_codes + c * kAChunkBytes);
-  if (sa_lane) cp_async16(dst + kCA * kAChunkBytes, g_sa);
+    if (c < nch) cp_async16_hint(dst + c * kAChunkBytes, g_codes + c * kAChunkBytes, l2_evict_first_policy());
+  if (sa_lane) cp_async16_hint(dst + kCA * kAChunkBytes, g_sa, l2_evict_first_policy());
 }
 
 __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n_my, int wa, int cw, int lane) {
@@ -686,10 +682,42 @@ __device__ void correction_warp(const DecodeParams& p, const SmemView& sv, int n
 // token, rows r and r + 1), so a lane keeps one running state and reads each
 // warp's region with one 8-byte load.
 static_assert(kGroupTile * 16 == 64 * kEpiWarps, "two elements per epilogue lane");
+static_assert(4 * kEpiWarps >= kDecodeTokens, "every token of a launch has an epilogue octet");
 // kShared: the last block merges on both epilogue warps (launches of three or
 // more tokens); otherwise on one.  Two instances, so that the code of one
 // path does not change the other's (the one-token kernel measured ~6 us slower
 // with both paths compiled into it).
+// The prologue resets the completion ticket (after the previous launch on the
+// workspace is done with it), so the ticket may be taken only once the
+// prologue grid is complete.  The core and correction warps wait for that
+// grid (griddepcontrol.wait) before they produce a partial, and the epilogue
+// takes the ticket after it has consumed every partial of the block, so a
+// second wait is needed only when the block has no such warp or no m-tile.
+__device__ __forceinline__ bool ticket_needs_wait(const DecodeParams& p, int n_my) {
+  return p.nw_work == p.nw_res || n_my == 0;
+}
+
+// The block's partial of token t, from the octets q = t, t + nt, ... < 8
+// merged in increasing q (deterministic), written by lane t of the calling
+// warp; the warp barrier orders the stores before lane 0's ticket.
+__device__ __forceinline__ void write_block_partials(const DecodeParams& p, const SmemView& sv, int lane) {
+  if (lane < p.nt) {
+    LseState a = lse_init();
+    PickState b = pick_init();
+#pragma unroll 1
+    for (int q = lane; q < 4 * kEpiWarps; q += p.nt) {
+      const float4 s = sv.tokstate[q];
+      a = lse_merge(a, LseState{s.x, s.y, __float_as_int(s.z)});
+      const float2 r = sv.pickstate[q];
+      b = pick_merge(b, PickState{r.x, __float_as_int(r.y)});
+    }
+    const size_t at = static_cast<size_t>(p.t0 + lane) * gridDim.x + blockIdx.x;
+    p.partials[at] = make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
+    if (p.sampled != nullptr) p.spart[at] = make_float2(b.z, __int_as_float(b.idx));
+  }
+  __syncwarp();
+}
+
 template <bool kShared>
 __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_my, int ew, int lane) {
   const int e = 2 * (32 * ew + lane);
@@ -751,67 +779,35 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&sv.redfree[r]));
   }
-  // Per token: merge each octet of lanes (16 rows of one token); octet
-  // q = 4 ew + (lane >> 3) carries token q mod nt.  Each warp leaves one state
-  // per token in shared memory; warp 0 merges them in warp order.
-#pragma unroll
+  // Merge each octet of lanes (16 rows of one token; octet q = 4 ew + lane / 8
+  // carries token q mod nt) and leave its state in shared memory.  The code
+  // from here on runs once per launch, after the packed head has streamed
+  // through L2, so its instructions are fetched cold: its loops stay rolled.
+#pragma unroll 1
   for (int o = 4; o >= 1; o >>= 1) {
     st = lse_merge(st, lse_shfl_xor(st, o));
     pk = pick_merge(pk, pick_shfl_xor(pk, o));
   }
-  for (int tt = 0; tt < p.nt; ++tt) {
-    LseState a = lse_init();
-    PickState b = pick_init();
-#pragma unroll
-    for (int oc = 0; oc < 4; ++oc) {
-      const LseState q = lse_shfl_idx(st, 8 * oc);
-      const PickState r = pick_shfl_idx(pk, 8 * oc);
-      if ((4 * ew + oc) % p.nt == tt) {
-        a = lse_merge(a, q);
-        b = pick_merge(b, r);
-      }
-    }
-    if (lane == 0) {
-      sv.tokstate[ew * kDecodeTokens + tt] = make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
-      sv.pickstate[ew * kDecodeTokens + tt] = make_float2(b.z, __int_as_float(b.idx));
-    }
+  if ((lane & 7) == 0) {
+    sv.tokstate[4 * ew + (lane >> 3)] = make_float4(st.m, st.s, __int_as_float(st.idx), 0.f);
+    sv.pickstate[4 * ew + (lane >> 3)] = make_float2(pk.z, __int_as_float(pk.idx));
   }
   named_bar_sync(1, kEpiWarps * 32);
   if constexpr (!kShared) {
     // One warp writes the block's partials, takes the ticket and, in the last
     // block, merges.
     if (ew != 0) return;
-    // The prologue resets the completion ticket, and the previous launch on this
-    // workspace must be done with it: wait for the preceding grid here.
-    grid_dependency_wait();
-    for (int t = 0; t < p.nt; ++t) {
-      LseState a = lse_init();
-      PickState b = pick_init();
-#pragma unroll
-      for (int w = 0; w < kEpiWarps; ++w) {
-        const float4 q = sv.tokstate[w * kDecodeTokens + t];
-        a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
-        const float2 r = sv.pickstate[w * kDecodeTokens + t];
-        b = pick_merge(b, PickState{r.x, __float_as_int(r.y)});
-      }
-      if (lane == 0) {
-        p.partials[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] =
-            make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
-        if (p.sampled != nullptr)
-          p.spart[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] = make_float2(b.z, __int_as_float(b.idx));
-      }
-    }
-    __threadfence();
-    __syncwarp();
+    if (ticket_needs_wait(p, n_my)) grid_dependency_wait();
+    write_block_partials(p, sv, lane);
     unsigned prev = 0;
-    if (lane == 0) prev = atomicAdd(p.counter, 1u);
+    if (lane == 0) prev = ticket_acq_rel(p.counter);
     prev = __shfl_sync(0xffffffffu, prev, 0);
     if (prev != gridDim.x - 1) return;
+    __syncwarp();   // the lanes' loads below come after lane 0's acquire
 
     // Last block: merge the per-block partials of every token of this launch.
     // A lane issues all of its loads of a round (kMergeLoadsOne partials) before
     // merging any, so a 148-block grid costs one L2 round trip, not five.
-    __threadfence();
     const int nblk = static_cast<int>(gridDim.x);
     for (int t = 0; t < p.nt; ++t) {
       const float4* part = p.partials + static_cast<size_t>(p.t0 + t) * gridDim.x;
@@ -826,7 +822,7 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
 #pragma unroll
         for (int u = 0; u < kMergeLoadsOne; ++u) a = lse_merge(a, LseState{q[u].x, q[u].y, __float_as_int(q[u].z)});
       }
-#pragma unroll
+#pragma unroll 1
       for (int m = 16; m >= 1; m >>= 1) a = lse_merge(a, lse_shfl_xor(a, m));
       if (p.sampled != nullptr) {
         const float2* sp = p.spart + static_cast<size_t>(p.t0 + t) * gridDim.x;
@@ -841,7 +837,7 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
 #pragma unroll
           for (int u = 0; u < kMergeLoadsOne; ++u) b = pick_merge(b, PickState{q[u].x, __float_as_int(q[u].y)});
         }
-#pragma unroll
+#pragma unroll 1
         for (int m = 16; m >= 1; m >>= 1) b = pick_merge(b, pick_shfl_xor(b, m));
         if (lane == 0) p.sampled[p.t0 + t] = b.idx;
       }
@@ -862,41 +858,17 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
     return;
   }
   if (ew == 0) {
-    // The prologue resets the completion ticket, and the previous launch on
-    // this workspace must be done with it: wait for the preceding grid here.
-    grid_dependency_wait();
-    for (int t = 0; t < p.nt; ++t) {
-      LseState a = lse_init();
-      PickState b = pick_init();
-#pragma unroll
-      for (int w = 0; w < kEpiWarps; ++w) {
-        const float4 q = sv.tokstate[w * kDecodeTokens + t];
-        a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
-        const float2 r = sv.pickstate[w * kDecodeTokens + t];
-        b = pick_merge(b, PickState{r.x, __float_as_int(r.y)});
-      }
-      if (lane == 0) {
-        p.partials[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] =
-            make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
-        if (p.sampled != nullptr)
-          p.spart[static_cast<size_t>(p.t0 + t) * gridDim.x + blockIdx.x] = make_float2(b.z, __int_as_float(b.idx));
-      }
-    }
-    __threadfence();
-    __syncwarp();
-    unsigned prev = 0;
-    if (lane == 0) prev = atomicAdd(p.counter, 1u);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (lane == 0) sv.flags[1] = prev == gridDim.x - 1 ? 1 : 0;
+    if (ticket_needs_wait(p, n_my)) grid_dependency_wait();
+    write_block_partials(p, sv, lane);
+    if (lane == 0) sv.flags[1] = ticket_acq_rel(p.counter) == gridDim.x - 1 ? 1 : 0;
   }
-  named_bar_sync(1, kEpiWarps * 32);
+  named_bar_sync(1, kEpiWarps * 32);   // also orders both warps' loads below after the acquire
   if (*reinterpret_cast<volatile int*>(&sv.flags[1]) == 0) return;
 
   // Last block: merge the per-block partials of every token of this launch.
   // The tokens are split over the epilogue warps, two per warp per round, and
   // a lane issues all of its loads of a round before merging any, so a
   // 148-block grid costs one L2 round trip per round (not one per partial).
-  __threadfence();
   const int nblk = static_cast<int>(gridDim.x);
   for (int tp = ew; tp < p.nt; tp += 2 * kEpiWarps) {
     const int tq = tp + kEpiWarps;   // the round's second token (may be past nt)
@@ -919,7 +891,7 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
         a1 = lse_merge(a1, LseState{q1[u].x, q1[u].y, __float_as_int(q1[u].z)});
       }
     }
-#pragma unroll
+#pragma unroll 1
     for (int m = 16; m >= 1; m >>= 1) {
       a0 = lse_merge(a0, lse_shfl_xor(a0, m));
       a1 = lse_merge(a1, lse_shfl_xor(a1, m));
@@ -942,7 +914,7 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
 #pragma unroll
           for (int u = 0; u < kMergeLoads; ++u) b = pick_merge(b, PickState{q[u].x, __float_as_int(q[u].y)});
         }
-#pragma unroll
+#pragma unroll 1
         for (int m = 16; m >= 1; m >>= 1) b = pick_merge(b, pick_shfl_xor(b, m));
         if (lane == 0) p.sampled[p.t0 + t] = b.idx;
       }
@@ -1012,8 +984,7 @@ void decode_smem_plan(DecodeParams& p, int g_steps) {
 
 size_t decode_smem_bytes(const DecodeParams& p) {
   return static_cast<size_t>(p.ring_bytes) + static_cast<size_t>(p.slots) * p.nw_work * kGroupTile * 16 * 4 +
-         static_cast<size_t>(2) * p.slots * 8 + kEpiWarps * kDecodeTokens * (16 + 8) +
-         kMaxDecodeWarps * kDecodeTokens * 4 + 8 + 16;
+         static_cast<size_t>(2) * p.slots * 8 + kEpiWarps * kDecodeTokens * (16 + 8) + 8 + 16;
 }
 
 namespace {

@@ -72,6 +72,18 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+// The same with an L2 cache policy (createpolicy): data read once per launch
+// is marked evict-first, so what the launch reuses (its own instructions, the
+// activations, the partials) stays in L2 while the packed head streams through.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -81,6 +93,17 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Completion ticket: one gpu-scope acquire-release add, returning the old
+// value.  The release half publishes the calling thread's earlier writes and,
+// cumulatively, those ordered before them by a block or warp barrier; the
+// acquire half orders the caller's later reads (and, after a barrier, its
+// block's) after every earlier releaser's writes.
+__device__ __forceinline__ unsigned ticket_acq_rel(unsigned* counter) {
+  unsigned prev;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(counter) : "memory");
+  return prev;
 }
 
 // ------------------------------------------------------------ named barrier
@@ -204,11 +227,13 @@ __device__ __forceinline__ void lse_push(LseState& st, float y, int v) {
     st.s += __expf(y - st.m);
   }
 }
+// Merge of two states, with the same fast exponential (a state with no
+// element, s = 0, contributes nothing and its exp(-inf - m) is not used).
 __device__ __forceinline__ LseState lse_merge(const LseState& a, const LseState& b) {
   LseState r;
   r.m = fmaxf(a.m, b.m);
-  const float sa = (a.s == 0.f) ? 0.f : a.s * expf(a.m - r.m);
-  const float sb = (b.s == 0.f) ? 0.f : b.s * expf(b.m - r.m);
+  const float sa = (a.s == 0.f) ? 0.f : a.s * __expf(a.m - r.m);
+  const float sb = (b.s == 0.f) ? 0.f : b.s * __expf(b.m - r.m);
   r.s = sa + sb;
   if (a.m > b.m) r.idx = a.idx;
   else if (b.m > a.m) r.idx = b.idx;

@@ -18,8 +18,10 @@ constexpr int kMaxDecodeWarps = 24;      // launch bound of the decode kernel
 constexpr int kEpiWarps = 2;             // decode epilogue warps (share each group of partial logits)
 constexpr int kDecodeTokens = 8;         // N of one m16n8k16 fragment
 constexpr int kRing = 4;                 // m-tiles in flight per compute warp
-// h is scaled per token by 2^(kScaleExp - E_t), E_t the binary exponent of
-// max|h_t| (max|h_t| < 2^E_t), so the fp16 copy is below 2^kScaleExp.
+// fp16 copies of h are scaled by 2^(kScaleExp - E), E the binary exponent of
+// the maximum of |h_t| over the columns they cover (the whole row for the
+// prologue's E_t, a residual warp's own columns in the decode kernel), so
+// they stay below 2^kScaleExp.
 constexpr int kScaleExp = 14;
 
 struct DecodeParams {
