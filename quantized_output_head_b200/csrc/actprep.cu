@@ -13,11 +13,19 @@
 // y[t,v]·2^c_t with no fp16 overflow.
 //
 // grid.y = Kz'/64 + 1: blocks y < Kz'/64 compute 64 entries of z for the 16
-// tokens with m16n8k16 MMAs (tokens as M, z rows as N, fp16 h scaled by
-// 2^(kScaleExp - E_t), exact int8 codes as fp16, fp32 accumulation; the
-// group scales of B are applied in fp32 at each group end); block y = last
+// tokens with m16n8k16 MMAs (tokens as M, z rows as N, fp16 h scaled by a
+// power of two, exact int8 codes as fp16, fp32 accumulation; the group
+// scales of B are applied in fp32 at each group end); block y = last
 // converts h.  Within every 16-column block X is stored in the column order
 // of the dequantised weights in tensor memory (tc_kpos).
+//
+// grid.z splits the columns of d when there are few tokens, so that the
+// short z computation spreads over the SMs: split s scales h by
+// 2^(kScaleExp - E_s) with E_s from its own columns, writes its fp32 sums
+// and E_s, and the last split to arrive (acquire-release ticket) adds the
+// splits in order, each times 2^(E_s - E_t) (E_t = max_s E_s), and writes X.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -30,6 +38,8 @@
 namespace archead {
 
 namespace {
+
+constexpr int kNoExp = -(1 << 20);   // exponent of a split whose columns are all zero
 
 // bf16 pair -> fp16 pair times 2^e (exact while the result is a normal fp16).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t bits, float scale) {
@@ -125,27 +135,36 @@ __device__ __forceinline__ void z_block(const ActParams& p, int n0, int b0, int 
 
 }  // namespace
 
-__global__ void __launch_bounds__(256) act_prep_kernel(const ActParams p) {
+__global__ void __launch_bounds__(256, 1) act_prep_kernel(const ActParams p) {
   __shared__ float red[8][16][64];
   __shared__ int s_E[16];
+  __shared__ bool s_nz[16];
+  __shared__ int s_last;
   // The tensor-core kernel may start streaming the packed head right away; it
   // waits (griddepcontrol.wait) before it reads anything written here.
   grid_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * 16;
-  if (p.targets != nullptr && blockIdx.x == 0 && blockIdx.y == 0) {
+  const bool conv = blockIdx.y == gridDim.y - 1;
+  if (conv && blockIdx.z != 0) return;
+  // 64-column blocks [kb0, kb1) of d: this split's (all of d for the h segment)
+  const int nb = p.d / 64;
+  const int kb0 = conv ? 0 : static_cast<int>(blockIdx.z) * nb / static_cast<int>(gridDim.z);
+  const int kb1 = conv ? nb : (static_cast<int>(blockIdx.z) + 1) * nb / static_cast<int>(gridDim.z);
+  if (p.targets != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
     for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
       const int v = p.targets[t];
       if (v < 0 || v >= p.v_total) atomicOr(p.status, static_cast<uint32_t>(ARCHEAD_STATUS_BAD_TARGET));
     }
   }
-  // E_t of the tile's tokens: |bf16| orders like its bit pattern without the sign.
+  // E of the tile's tokens over columns [64 kb0, 64 kb1) (E_t for the whole
+  // row): |bf16| orders like its bit pattern without the sign.
   for (int tt = 0; tt < 2; ++tt) {
     const int tl = 2 * warp + tt, t = t0 + tl;
     uint32_t mx = 0;
     if (t < p.T) {
       const uint4* row = reinterpret_cast<const uint4*>(p.hidden + static_cast<size_t>(t) * p.d);
-      for (int i = lane; i < p.d / 8; i += 32) {
+      for (int i = 8 * kb0 + lane; i < 8 * kb1; i += 32) {
         const uint4 v = row[i];
         mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
         mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
@@ -158,11 +177,12 @@ __global__ void __launch_bounds__(256) act_prep_kernel(const ActParams p) {
       int E = 0;
       if (m16 != 0) frexpf(__uint_as_float(m16 << 16), &E);   // max|h_t| < 2^E
       s_E[tl] = E;
+      s_nz[tl] = m16 != 0;
     }
   }
   __syncthreads();
 
-  if (blockIdx.y == gridDim.y - 1) {
+  if (conv) {
     // h segment: X[t, j] = h[t, j]·2^(c_t - alpha), c_t = kScaleExp - E_t + mseg.
     if (threadIdx.x < 16 && t0 + static_cast<int>(threadIdx.x) < p.T)
       p.cinv[t0 + threadIdx.x] = ldexpf(1.f, s_E[threadIdx.x] - kScaleExp - p.mseg);
@@ -187,8 +207,7 @@ __global__ void __launch_bounds__(256) act_prep_kernel(const ActParams p) {
   // z segment: rows n0 .. n0 + 63 of (R | B), all of one kind (r_c' is a multiple of 64).
   const int n0 = blockIdx.y * 64;
   const int gr = lane >> 2;
-  const int nb = p.d / 64;
-  const int b0 = warp * nb / 8, b1 = (warp + 1) * nb / 8;
+  const int b0 = kb0 + warp * (kb1 - kb0) / 8, b1 = kb0 + (warp + 1) * (kb1 - kb0) / 8;
   const int ta = t0 + gr, tb = t0 + gr + 8;
   const float hs[2] = {ta < p.T ? ldexpf(1.f, kScaleExp - s_E[gr]) : 0.f,
                        tb < p.T ? ldexpf(1.f, kScaleExp - s_E[gr + 8]) : 0.f};
@@ -211,16 +230,52 @@ __global__ void __launch_bounds__(256) act_prep_kernel(const ActParams p) {
     red[warp][gr + 8][8 * n + 2 * cc + 1] = acc[n][3];
   }
   __syncthreads();
+  const int zb = static_cast<int>(blockIdx.x * (gridDim.y - 1) + blockIdx.y);   // tile x z block
+  if (gridDim.z > 1) {
+    // This split's sums (in the 2^(kScaleExp - E_s) domain) and exponents.
+    float* mine = p.zpart + (static_cast<size_t>(zb) * gridDim.z + blockIdx.z) * kActPartFloats;
+    for (int idx = threadIdx.x; idx < 16 * 64; idx += blockDim.x) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) s += red[w][idx >> 6][idx & 63];
+      mine[idx] = s;
+    }
+    // (a split whose columns are all zero carries no exponent)
+    if (threadIdx.x < 16) mine[16 * 64 + threadIdx.x] = __int_as_float(s_nz[threadIdx.x] ? s_E[threadIdx.x] : kNoExp);
+    __syncthreads();   // the block's stores come before thread 0's release
+    if (threadIdx.x == 0) s_last = ticket_acq_rel(p.zticket + zb) == gridDim.z - 1 ? 1 : 0;
+    __syncthreads();   // and every thread's loads below after its acquire
+    if (!s_last) return;
+    const float* all = p.zpart + static_cast<size_t>(zb) * gridDim.z * kActPartFloats;
+    if (threadIdx.x < 16) {
+      int E = kNoExp;
+      for (int z = 0; z < static_cast<int>(gridDim.z); ++z)
+        E = max(E, __float_as_int(__ldcg(all + static_cast<size_t>(z) * kActPartFloats + 16 * 64 + threadIdx.x)));
+      s_E[threadIdx.x] = E == kNoExp ? 0 : E;   // E_t (0 for an all-zero token, as for a whole row)
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < 16 * 64; idx += blockDim.x) {
+      const int tl = idx >> 6;
+      float s = 0.f;
+      for (int z = 0; z < static_cast<int>(gridDim.z); ++z) {
+        const float* part = all + static_cast<size_t>(z) * kActPartFloats;
+        s += ldexpf(__ldcg(part + idx), __float_as_int(__ldcg(part + 16 * 64 + tl)) - s_E[tl]);
+      }
+      red[0][tl][idx & 63] = s;
+    }
+    if (threadIdx.x == 0) p.zticket[zb] = 0u;   // every split has arrived: ready for the next call
+    __syncthreads();
+  }
   // X[t, d + n] = z·2^(c_t - beta|gamma): with c_t = kScaleExp - E_t + mseg the
   // token exponent cancels against the 2^(kScaleExp - E_t) of h.
   const float sc_core = ldexpf(1.f, p.mseg - p.beta);
   const float sc_corr = ldexpf(1.f, p.mseg - p.gamma);
+  const int nw = gridDim.z > 1 ? 1 : 8;   // warp partials still to add
   for (int idx = threadIdx.x; idx < 16 * 64; idx += blockDim.x) {
     const int tl = idx >> 6, c = idx & 63, t = t0 + tl, n = n0 + c;
     if (t >= p.T) continue;
     float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) s += red[w][tl][c];
+    for (int w = 0; w < nw; ++w) s += red[w][tl][c];
     float val = 0.f;
     if (n < p.rcp) val = s * __half2float(__ushort_as_half(p.s_R[n])) * sc_core;
     else if (n < p.Kz) val = s * sc_corr;
@@ -229,10 +284,18 @@ __global__ void __launch_bounds__(256) act_prep_kernel(const ActParams p) {
   }
 }
 
-cudaError_t launch_act_prep(const ActParams& p, cudaStream_t stream) {
-  const dim3 grid((p.T + 15) / 16, (p.Kc - p.d) / 64 + 1);
+cudaError_t launch_act_prep(const ActParams& p, int splits, cudaStream_t stream) {
+  const dim3 grid((p.T + 15) / 16, (p.Kc - p.d) / 64 + 1, splits);
   act_prep_kernel<<<grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
+}
+
+int act_prep_splits(int T, int d, int Kc, int num_sms, size_t scratch_bytes) {
+  const int tiles = ((T + 15) / 16) * ((Kc - d) / 64);
+  if (tiles == 0 || tiles > kActTickets) return 1;
+  int s = std::min(std::min(kActMaxSplits, d / 64), std::max(1, num_sms / tiles));
+  while (s > 1 && static_cast<size_t>(s) * tiles * kActPartFloats * 4 > scratch_bytes) --s;
+  return s;
 }
 
 }  // namespace archead

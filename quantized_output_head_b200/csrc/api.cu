@@ -68,7 +68,13 @@ int forward_tc(const archead_handle* h, const uint16_t* hidden, int32_t T, const
   ap.beta = h->tc_beta;
   ap.gamma = h->tc_gamma;
   ap.mseg = h->tc_mseg;
-  cudaError_t e = launch_act_prep(ap, stream);
+  // The K-split partials borrow the region of the tensor-core partials: the
+  // tensor-core kernel writes there only after this grid has completed.
+  const size_t part_bytes = static_cast<size_t>(T) * tc_n_mt128(L) * 16;
+  const int splits = act_prep_splits(T, L.d, Kc, h->num_sms, part_bytes);
+  ap.zpart = reinterpret_cast<float*>(wb + w.tpartials);
+  ap.zticket = reinterpret_cast<uint32_t*>(wb + kActTicketOff);
+  cudaError_t e = launch_act_prep(ap, splits, stream);
   if (e != cudaSuccess) return set_cuda_error(e);
 
   TcParams tp{};

@@ -61,6 +61,10 @@ struct WsLayout {
   size_t h_logits, host_logits_total;   // logits form: [T, V] fp32 staging after host_total
 };
 
+// The K-split tickets of the activation kernel sit in the zero-filled head of
+// the workspace, between the status word and the target logits.
+static_assert(kActTicketOff >= 8 && kActTicketOff + 4 * kActTickets <= 256, "ticket block of the workspace head");
+
 inline WsLayout ws_layout(const archead_handle& h, int T) {
   WsLayout w{};
   const size_t t = static_cast<size_t>(T);
@@ -102,7 +106,10 @@ cudaError_t launch_decode(int g_steps, const DecodeParams& p, int grid, size_t s
 cudaError_t launch_prologue(const PrologueParams& p, cudaStream_t stream);
 
 // Tensor-core path (actprep.cu, tcgemm.cu).
-cudaError_t launch_act_prep(const ActParams& p, cudaStream_t stream);
+cudaError_t launch_act_prep(const ActParams& p, int splits, cudaStream_t stream);
+// K splits of the activation kernel for T tokens; their partials need
+// splits x tiles x z blocks x kActPartFloats floats of scratch_bytes.
+int act_prep_splits(int T, int d, int Kc, int num_sms, size_t scratch_bytes);
 void tc_smem_plan(TcParams& p);
 size_t tc_smem_bytes(const TcParams& p);
 size_t tc_smem_max();

@@ -24,6 +24,10 @@ constexpr int kTcSlotBytes = 1056;    // one packed k-step of one m-tile block (
 constexpr int kTcDeqWarps = 16;       // two per m-tile block of a unit (even / odd k-steps)
 constexpr int kTcWarps = 22;          // 16 dequantising, 1 TMA, 1 MMA, 4 epilogue
 constexpr int kTcMinTokens = 9;       // calls with fewer tokens take the decode kernel (one launch)
+constexpr int kActMaxSplits = 8;      // K splits of one block of z in the activation kernel
+constexpr int kActPartFloats = 16 * 64 + 16;   // one split's partial sums and token exponents
+constexpr int kActTicketOff = 64;     // workspace byte offset of the K-split tickets (inside the zeroed head)
+constexpr int kActTickets = 48;       // tickets available there: K splits need tiles x z blocks <= this
 
 struct TcParams {
   const uint8_t* mtiles;      // arena: m-tile blocks
@@ -55,6 +59,8 @@ struct ActParams {
   uint32_t* status;
   uint16_t* xop;              // [T, Kc] fp16 activation operand
   float* cinv;                // [T] 2^-c_t
+  float* zpart;               // K-split partials: [tile][z block][split] x (16 x 64 sums, 16 exponents)
+  uint32_t* zticket;          // [tile][z block] completion tickets of the K splits (zero between calls)
   int32_t T, d, rcp, Kz, Kc, g_B, V;
   int32_t v_total;                             // target ids are checked against [0, v_total)
   int32_t alpha, beta, gamma, mseg;

@@ -584,26 +584,44 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1)
   }
 }
 
-// Per-token fold of the partials: LSE, first argmax, cross-entropy.
-__global__ void __launch_bounds__(256) tc_merge_kernel(const float4* partials, int n_mt128, int T,
-                                                       const int32_t* targets, const float* tgt, int V, int row0,
-                                                       float* lse, int32_t* argmax, float* ce, float4* shard_out) {
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+// Per-token fold of the partials: LSE, first argmax, cross-entropy.  One
+// block per token: a thread folds the partials m = tid, tid + 256, ... (loads
+// of a round issued together), then the warps (shuffle tree) and the block's
+// eight warp states in warp order, so the order is fixed whatever the timing.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeRound = 8;   // partials a thread loads before folding any
+__global__ void __launch_bounds__(kMergeThreads) tc_merge_kernel(const float4* partials, int n_mt128, int T,
+                                                                 const int32_t* targets, const float* tgt, int V,
+                                                                 int row0, float* lse, int32_t* argmax, float* ce,
+                                                                 float4* shard_out) {
+  __shared__ float4 ws[kMergeThreads / 32];
+  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   grid_dependency_wait();
-  if (t >= T) return;
+  const float4* part = partials + static_cast<size_t>(t) * n_mt128;
   LseState a = lse_init();
-  for (int m = lane; m < n_mt128; m += 32) {
-    const float4 q = partials[static_cast<size_t>(t) * n_mt128 + m];
-    a = lse_merge(a, LseState{q.x, q.y, __float_as_int(q.z)});
+  for (int m0 = 0; m0 < n_mt128; m0 += kMergeThreads * kMergeRound) {
+    float4 q[kMergeRound];
+#pragma unroll
+    for (int u = 0; u < kMergeRound; ++u) {
+      const int m = m0 + static_cast<int>(threadIdx.x) + kMergeThreads * u;
+      q[u] = m < n_mt128 ? __ldcg(part + m) : make_float4(-INFINITY, 0.f, __int_as_float(0x7fffffff), 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kMergeRound; ++u) a = lse_merge(a, LseState{q[u].x, q[u].y, __float_as_int(q[u].z)});
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) a = lse_merge(a, lse_shfl_xor(a, o));
-  if (lane == 0) {
+  if (lane == 0) ws[warp] = make_float4(a.m, a.s, __int_as_float(a.idx), 0.f);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    a = lse_init();
+#pragma unroll 1
+    for (int w = 0; w < kMergeThreads / 32; ++w) a = lse_merge(a, LseState{ws[w].x, ws[w].y, __float_as_int(ws[w].z)});
     const float l = a.m + logf(a.s);
     const int gidx = a.idx + row0;
     // target logit when the target row is one of this head's rows
     const int tl = targets != nullptr ? targets[t] - row0 : -1;
-    const float tv = (tl >= 0 && tl < V) ? tgt[t] : __int_as_float(0x7fc00000);
+    const float tv = (tl >= 0 && tl < V) ? __ldcg(tgt + t) : __int_as_float(0x7fc00000);
     if (lse != nullptr) lse[t] = l;
     if (argmax != nullptr) argmax[t] = gidx;
     if (ce != nullptr) ce[t] = l - tv;
@@ -715,9 +733,20 @@ cudaError_t launch_tc(const TcParams& p, const CUtensorMap& map, int grid, cudaS
 cudaError_t launch_tc_merge(const float4* partials, int n_mt128, int T, const int32_t* targets, const float* tgt,
                             int V, int row0, float* lse, int32_t* argmax, float* ce, float4* shard_out,
                             cudaStream_t stream) {
-  tc_merge_kernel<<<(T + 7) / 8, 256, 0, stream>>>(partials, n_mt128, T, targets, tgt, V, row0, lse, argmax, ce,
-                                                   shard_out);
-  return cudaGetLastError();
+  // Launched as a programmatic dependent of the tensor-core kernel: its blocks
+  // take the SMs that kernel frees and wait (griddepcontrol.wait) for its
+  // partials.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(T);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_merge_kernel, partials, n_mt128, T, targets, tgt, V, row0, lse, argmax, ce,
+                            shard_out);
 }
 
 // Per token, fold the states of n vocabulary shards (stacked in increasing row
