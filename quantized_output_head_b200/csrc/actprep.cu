@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(256, 1) act_prep_kernel(const ActParams p) {
   __shared__ float red[8][16][64];
   __shared__ int s_E[16];
   __shared__ bool s_nz[16];
+  __shared__ int s_Ez[kActMaxSplits][16];
   __shared__ int s_last;
   // The tensor-core kernel may start streaming the packed head right away; it
   // waits (griddepcontrol.wait) before it reads anything written here.
@@ -146,33 +147,54 @@ __global__ void __launch_bounds__(256, 1) act_prep_kernel(const ActParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * 16;
   const bool conv = blockIdx.y == gridDim.y - 1;
-  if (conv && blockIdx.z != 0) return;
-  // 64-column blocks [kb0, kb1) of d: this split's (all of d for the h segment)
+  // 64-column blocks [kb0, kb1) of d: this split's (its share of the h
+  // segment for the converting blocks, whose exponents cover all of d)
   const int nb = p.d / 64;
-  const int kb0 = conv ? 0 : static_cast<int>(blockIdx.z) * nb / static_cast<int>(gridDim.z);
-  const int kb1 = conv ? nb : (static_cast<int>(blockIdx.z) + 1) * nb / static_cast<int>(gridDim.z);
+  const int kb0 = static_cast<int>(blockIdx.z) * nb / static_cast<int>(gridDim.z);
+  const int kb1 = (static_cast<int>(blockIdx.z) + 1) * nb / static_cast<int>(gridDim.z);
+  const int eb0 = conv ? 0 : kb0, eb1 = conv ? nb : kb1;
   if (p.targets != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
     for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
       const int v = p.targets[t];
       if (v < 0 || v >= p.v_total) atomicOr(p.status, static_cast<uint32_t>(ARCHEAD_STATUS_BAD_TARGET));
     }
   }
-  // E of the tile's tokens over columns [64 kb0, 64 kb1) (E_t for the whole
-  // row): |bf16| orders like its bit pattern without the sign.
-  for (int tt = 0; tt < 2; ++tt) {
-    const int tl = 2 * warp + tt, t = t0 + tl;
-    uint32_t mx = 0;
-    if (t < p.T) {
-      const uint4* row = reinterpret_cast<const uint4*>(p.hidden + static_cast<size_t>(t) * p.d);
-      for (int i = 8 * kb0 + lane; i < 8 * kb1; i += 32) {
-        const uint4 v = row[i];
-        mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, v.w & 0x7FFF7FFFu);
-      }
+  // E of the tile's tokens over columns [64 eb0, 64 eb1) (E_t for the whole
+  // row): |bf16| orders like its bit pattern without the sign.  Warp w takes
+  // tokens 2w and 2w + 1, a lane kEU 16-byte pieces of each per round, all
+  // loads of a round in flight together.
+  constexpr int kEU = 4;
+  uint32_t mx[2] = {0u, 0u};
+  {
+    const uint4* rows[2];
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      const int t = t0 + 2 * warp + tt;
+      rows[tt] = t < p.T ? reinterpret_cast<const uint4*>(p.hidden + static_cast<size_t>(t) * p.d) : nullptr;
     }
-    const uint32_t m16 = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
+    for (int i0 = 8 * eb0 + lane; i0 < 8 * eb1; i0 += 32 * kEU) {
+      uint4 v[2][kEU];
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+          const int i = i0 + 32 * u;
+          v[tt][u] = (rows[tt] != nullptr && i < 8 * eb1) ? rows[tt][i] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+          mx[tt] = __vmaxu2(mx[tt], v[tt][u].x & 0x7FFF7FFFu);
+          mx[tt] = __vmaxu2(mx[tt], v[tt][u].y & 0x7FFF7FFFu);
+          mx[tt] = __vmaxu2(mx[tt], v[tt][u].z & 0x7FFF7FFFu);
+          mx[tt] = __vmaxu2(mx[tt], v[tt][u].w & 0x7FFF7FFFu);
+        }
+    }
+  }
+  for (int tt = 0; tt < 2; ++tt) {
+    const int tl = 2 * warp + tt;
+    const uint32_t m16 = __reduce_max_sync(0xffffffffu, max(mx[tt] & 0xFFFFu, mx[tt] >> 16));
     if (lane == 0) {
       int E = 0;
       if (m16 != 0) frexpf(__uint_as_float(m16 << 16), &E);   // max|h_t| < 2^E
@@ -183,23 +205,40 @@ __global__ void __launch_bounds__(256, 1) act_prep_kernel(const ActParams p) {
   __syncthreads();
 
   if (conv) {
-    // h segment: X[t, j] = h[t, j]·2^(c_t - alpha), c_t = kScaleExp - E_t + mseg.
-    if (threadIdx.x < 16 && t0 + static_cast<int>(threadIdx.x) < p.T)
+    // h segment, 16-column blocks [4 kb0, 4 kb1) of this split:
+    // X[t, j] = h[t, j]·2^(c_t - alpha), c_t = kScaleExp - E_t + mseg.
+    if (blockIdx.z == 0 && threadIdx.x < 16 && t0 + static_cast<int>(threadIdx.x) < p.T)
       p.cinv[t0 + threadIdx.x] = ldexpf(1.f, s_E[threadIdx.x] - kScaleExp - p.mseg);
-    const int nb16 = p.d / 16;
-    for (int item = threadIdx.x; item < 16 * nb16; item += blockDim.x) {
-      const int tl = item / nb16, b = item - tl * nb16, t = t0 + tl;
-      if (t >= p.T) break;
-      const float sc = ldexpf(1.f, kScaleExp - s_E[tl] + p.mseg - p.alpha);
-      const uint4* src = reinterpret_cast<const uint4*>(p.hidden + static_cast<size_t>(t) * p.d + b * 16);
-      const uint4 lo = src[0], hi = src[1];
-      const uint32_t in[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};   // column pairs 2i, 2i+1
-      uint32_t out[8];
+    const int nbr = 4 * (kb1 - kb0), n_items = 16 * nbr;
+    constexpr int kCU = 2;   // items of a thread in flight together
+    for (int item0 = threadIdx.x; item0 < n_items; item0 += kCU * blockDim.x) {
+      uint4 lo[kCU], hi[kCU];
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) out[jj] = bf16x2_to_f16x2(in[(jj >> 1) + 4 * (jj & 1)], sc);
-      uint4* dst = reinterpret_cast<uint4*>(p.xop + static_cast<size_t>(t) * p.Kc + b * 16);
-      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+      for (int u = 0; u < kCU; ++u) {
+        const int item = item0 + u * static_cast<int>(blockDim.x);
+        const int tl = item / nbr, t = t0 + tl;
+        lo[u] = hi[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (item < n_items && t < p.T) {
+          const uint4* src =
+              reinterpret_cast<const uint4*>(p.hidden + static_cast<size_t>(t) * p.d + (4 * kb0 + item - tl * nbr) * 16);
+          lo[u] = src[0];
+          hi[u] = src[1];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kCU; ++u) {
+        const int item = item0 + u * static_cast<int>(blockDim.x);
+        const int tl = item / nbr, t = t0 + tl;
+        if (item >= n_items || t >= p.T) continue;
+        const float sc = ldexpf(1.f, kScaleExp - s_E[tl] + p.mseg - p.alpha);
+        const uint32_t in[8] = {lo[u].x, lo[u].y, lo[u].z, lo[u].w, hi[u].x, hi[u].y, hi[u].z, hi[u].w};   // column pairs 2i, 2i+1
+        uint32_t out[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) out[jj] = bf16x2_to_f16x2(in[(jj >> 1) + 4 * (jj & 1)], sc);
+        uint4* dst = reinterpret_cast<uint4*>(p.xop + static_cast<size_t>(t) * p.Kc + (4 * kb0 + item - tl * nbr) * 16);
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+      }
     }
     return;
   }
@@ -246,21 +285,28 @@ __global__ void __launch_bounds__(256, 1) act_prep_kernel(const ActParams p) {
     if (threadIdx.x == 0) s_last = ticket_acq_rel(p.zticket + zb) == gridDim.z - 1 ? 1 : 0;
     __syncthreads();   // and every thread's loads below after its acquire
     if (!s_last) return;
-    const float* all = p.zpart + static_cast<size_t>(zb) * gridDim.z * kActPartFloats;
+    const int nz = static_cast<int>(gridDim.z);
+    const float* all = p.zpart + static_cast<size_t>(zb) * nz * kActPartFloats;
+    if (static_cast<int>(threadIdx.x) < 16 * nz)
+      s_Ez[threadIdx.x >> 4][threadIdx.x & 15] =
+          __float_as_int(__ldcg(all + static_cast<size_t>(threadIdx.x >> 4) * kActPartFloats + 16 * 64 + (threadIdx.x & 15)));
+    __syncthreads();
     if (threadIdx.x < 16) {
       int E = kNoExp;
-      for (int z = 0; z < static_cast<int>(gridDim.z); ++z)
-        E = max(E, __float_as_int(__ldcg(all + static_cast<size_t>(z) * kActPartFloats + 16 * 64 + threadIdx.x)));
+      for (int z = 0; z < nz; ++z) E = max(E, s_Ez[z][threadIdx.x]);
       s_E[threadIdx.x] = E == kNoExp ? 0 : E;   // E_t (0 for an all-zero token, as for a whole row)
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < 16 * 64; idx += blockDim.x) {
       const int tl = idx >> 6;
+      float v[kActMaxSplits];
+#pragma unroll
+      for (int z = 0; z < kActMaxSplits; ++z)
+        v[z] = z < nz ? __ldcg(all + static_cast<size_t>(z) * kActPartFloats + idx) : 0.f;
       float s = 0.f;
-      for (int z = 0; z < static_cast<int>(gridDim.z); ++z) {
-        const float* part = all + static_cast<size_t>(z) * kActPartFloats;
-        s += ldexpf(__ldcg(part + idx), __float_as_int(__ldcg(part + 16 * 64 + tl)) - s_E[tl]);
-      }
+#pragma unroll
+      for (int z = 0; z < kActMaxSplits; ++z)
+        if (z < nz) s += ldexpf(v[z], s_Ez[z][tl] - s_E[tl]);
       red[0][tl][idx & 63] = s;
     }
     if (threadIdx.x == 0) p.zticket[zb] = 0u;   // every split has arrived: ready for the next call
