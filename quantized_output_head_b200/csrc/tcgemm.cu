@@ -90,6 +90,26 @@ __device__ __forceinline__ bool tc_wait_warp(const TcSmem& s, uint64_t* bar, uin
   return ok;
 }
 
+// The same, with the common case (the phase has completed) in one try and one
+// vote; the abort flag is read only when the phase is still pending.
+__device__ __forceinline__ bool tc_wait_fast(const TcSmem& s, uint64_t* bar, uint32_t parity, uint32_t* status) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(smem_addr(bar), parity))) return true;
+  return tc_wait_warp(s, bar, parity, status);
+}
+
+// Shared-memory loads by 32-bit address (ordered after the copy waits and the
+// warp barrier before them).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+
 // ------------------------------------------------------- dequantising warps
 // Packed bytes of one k-step of one m-tile block -> ring slot (kTcSlotBytes):
 //   residual   [0,512) codes, [512, 512 + 32 * groups) group scales
@@ -115,24 +135,6 @@ __device__ __forceinline__ void issue_step(const TcParams& p, uint32_t dst, cons
     cp_async16(dst + lane * 16, blk + p.off_A + a * kAChunkBytes + lane * 16);
     if (a + 1 < p.n_A) cp_async16(dst + 512 + lane * 16, blk + p.off_A + (a + 1) * kAChunkBytes + lane * 16);
     if (lane < 2) cp_async16(dst + kSlotCorrScales + lane * 16, blk + p.off_sA + lane * 16);
-  }
-}
-
-// A stage of two residual k-steps (ks0, ks0 + 1) of m-tile block blk: the
-// codes of both (1024 contiguous bytes) and the scales of each, 16 bytes per
-// lane, addressed with a few integer operations (the common stage).
-template <int GM>
-__device__ __forceinline__ void issue_res_stage(const TcParams& p, uint32_t dst, const uint8_t* blk, int ks0,
-                                                int lane) {
-  const uint8_t* codes = blk + p.off_res + ks0 * kResChunkBytes + lane * 16;
-  cp_async16(dst + lane * 16, codes);
-  cp_async16(dst + kTcSlotBytes + lane * 16, codes + kResChunkBytes);
-  constexpr int kPieces = 2 << GM;                   // 16-byte scale pieces per k-step
-  if (lane < 2 * kPieces) {
-    const int kk = lane / kPieces, piece = lane % kPieces;
-    const int g0 = ((ks0 + kk) * kTcBK) >> p.g_log2;
-    cp_async16(dst + kk * kTcSlotBytes + kSlotResScales + piece * 16,
-               blk + p.off_sres + g0 * kSresGroupBytes + piece * 16);
   }
 }
 
@@ -163,6 +165,28 @@ __device__ __forceinline__ void dequant_residual(const uint8_t* slot, float sc, 
 #pragma unroll
   for (int st = 0; st < 4; ++st) {
     if (st % (4 >> GM) == 0) scale_pair(slot + kSlotResScales + (st >> (2 - GM)) * kSresGroupBytes + gr * 4, sc, s0, s1);
+    uint32_t a[4];
+    unpack_int4_signed(w[st], a);
+    place(a, s0, s1, r + 4 * st);
+  }
+}
+
+// The same from the slot's shared-memory address: codes at slot + code_off
+// (code_off = 16 lane), this lane's scale pair at slot + scale_off
+// (scale_off = kSlotResScales + 4 gr).
+template <int GM>
+__device__ __forceinline__ void dequant_residual_s(uint32_t slot, uint32_t code_off, uint32_t scale_off, float sc,
+                                                   uint32_t (&r)[16]) {
+  const uint4 c = lds128(slot + code_off);
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  uint32_t s0 = 0, s1 = 0;
+#pragma unroll
+  for (int st = 0; st < 4; ++st) {
+    if (st % (4 >> GM) == 0) {
+      const float2 f = half2_bits_to_float2(lds32(slot + scale_off + (st >> (2 - GM)) * kSresGroupBytes));
+      s0 = pack_half2(f.x * sc, f.x * sc);
+      s1 = pack_half2(f.y * sc, f.y * sc);
+    }
     uint32_t a[4];
     unpack_int4_signed(w[st], a);
     place(a, s0, s1, r + 4 * st);
@@ -218,24 +242,6 @@ __device__ __forceinline__ const uint8_t* unit_block(const TcParams& p, int ui, 
   return mt16 < p.n_mtiles ? p.mtiles + static_cast<size_t>(mt16) * p.mblk_bytes : nullptr;
 }
 
-// Cursor over the global stages g = par, par + 2, ... of this CTA's units
-// (stage st of a unit holds k-steps 2st and 2st + 1).
-struct StageCursor {
-  int ui, st;
-  const uint8_t* blk;
-};
-__device__ __forceinline__ void cursor_normalize(StageCursor& c, const TcParams& p, int n_my, int j) {
-  while (c.st >= p.n_st) {
-    c.st -= p.n_st;
-    ++c.ui;
-    c.blk = unit_block(p, c.ui, n_my, j);
-  }
-}
-__device__ __forceinline__ void cursor_advance(StageCursor& c, const TcParams& p, int n_my, int j) {
-  c.st += 2;
-  cursor_normalize(c, p, n_my, j);
-}
-
 template <int GM>
 __device__ __forceinline__ void dequant_step(const TcParams& p, const uint8_t* slot, int ks, int lane,
                                              uint32_t (&r)[16]) {
@@ -246,11 +252,13 @@ __device__ __forceinline__ void dequant_step(const TcParams& p, const uint8_t* s
 
 // Warp w dequantises m-tile block j = 2(w%4) + (w/4)%2 of every unit (TMEM
 // lanes 16j..16j+15 lie in the warp's lane quarter w%4) on the global stages
-// of parity w/8; a stage buffer has a fixed parity (the buffer count is even),
-// so each buffer is filled by the same eight warps.  R: ring slots, each the
-// packed bytes of one stage (two k-steps), filled R - 1 stages ahead with
-// 16-byte cp.async per lane.  (One bulk copy per piece, issued by one lane,
-// measured slower: the copy engine queues many 512-byte copies.)
+// g = ui * n_st + st of parity w/8; a stage buffer has a fixed parity (the
+// buffer count is even), so each buffer is filled by the same eight warps.  R:
+// ring slots, each the packed bytes of one stage (two k-steps), filled R - 1
+// of the warp's stages ahead with 16-byte cp.async per lane.  (One bulk copy
+// per piece, issued by one lane, measured slower: the copy engine queues many
+// 512-byte copies.)  The stages whose two k-steps are both residual (all but a
+// few per unit) run a loop of their own with no per-stage segment tests.
 template <int R, int GM>
 __device__ void dequant_loop(const TcParams& p, const TcSmem& sm, uint32_t tmem_base, int w, int lane) {
   constexpr uint32_t kPair = 2 * kTcSlotBytes;
@@ -260,86 +268,138 @@ __device__ void dequant_loop(const TcParams& p, const TcSmem& sm, uint32_t tmem_
   const uint8_t* ring = sm.rings + static_cast<size_t>(w) * R * kPair;
   const int n_my = (p.n_units - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                    static_cast<int>(gridDim.x);
-  const int total = n_my * p.n_st;   // global stages of this CTA
+  const int n_st = p.n_st;
+  const int n_rst = p.ks_core >> 1;   // stages of two residual k-steps
 
-  // Prefetch R - 1 of this warp's stages ahead.
-  StageCursor pc{0, par, unit_block(p, 0, n_my, j)};
-  cursor_normalize(pc, p, n_my, j);
-  int pg = par;
+  // Prefetch cursor: unit ordinal pu, stage pst, R - 1 of this warp's stages
+  // ahead.  A residual stage is the codes of two k-steps (1024 contiguous
+  // bytes, 16 per lane) and the scales of each (lanes below 2 kPieces).
+  constexpr int kPieces = 2 << GM;                  // 16-byte scale pieces per k-step
+  const int kk = lane / kPieces, piece = lane % kPieces;
+  const bool scale_lane = lane < 2 * kPieces;
+  const uint32_t code_dst = 16u * lane, scale_dst = kk * kTcSlotBytes + kSlotResScales + piece * 16;
+  int pu = 0, pst = par;
+  const uint8_t* pblk = nullptr;
+  const uint8_t* pcode = nullptr;    // this lane's codes of k-step 0 of the unit
+  const uint8_t* pscale = nullptr;   // its scale piece of group 0
+  auto rebase = [&]() {
+    pblk = unit_block(p, pu, n_my, j);
+    if (pblk != nullptr) {
+      pcode = pblk + p.off_res + 16 * lane;
+      pscale = pblk + p.off_sres + 16 * piece;
+    }
+  };
+  rebase();
   uint32_t pslot = 0;
   auto issue_next = [&]() {
-    if (pg < total && pc.blk != nullptr) {
-      const uint32_t dst = ring_s + pslot * kPair;
-      const int ks0 = 2 * pc.st;
-      if (ks0 + 1 < p.ks_core) {
-        issue_res_stage<GM>(p, dst, pc.blk, ks0, lane);
-      } else {
-        issue_step(p, dst, pc.blk, ks0, lane);
-        if (ks0 + 1 < p.n_ks) issue_step(p, dst + kTcSlotBytes, pc.blk, ks0 + 1, lane);
+    if (pu < n_my) {
+      if (pblk != nullptr) {
+        const uint32_t dst = ring_s + pslot * kPair;
+        const int ks0 = 2 * pst;
+        if (pst < n_rst) {
+          const uint8_t* c = pcode + ks0 * kResChunkBytes;
+          cp_async16(dst + code_dst, c);
+          cp_async16(dst + kTcSlotBytes + code_dst, c + kResChunkBytes);
+          if (scale_lane) cp_async16(dst + scale_dst, pscale + (((ks0 + kk) * kTcBK) >> p.g_log2) * kSresGroupBytes);
+        } else {
+          issue_step(p, dst, pblk, ks0, lane);
+          if (ks0 + 1 < p.n_ks) issue_step(p, dst + kTcSlotBytes, pblk, ks0 + 1, lane);
+        }
+      }
+      pst += 2;
+      if (pst >= n_st) {
+        pst -= n_st;
+        ++pu;
+        rebase();
       }
     }
     cp_async_commit();
-    if (pg < total) {
-      pg += 2;
-      cursor_advance(pc, p, n_my, j);
-    }
-    if (++pslot == R) pslot = 0;
+    pslot = pslot + 1 == R ? 0u : pslot + 1;
   };
 #pragma unroll 1
   for (int k = 0; k < R - 1; ++k) issue_next();
 
   const uint32_t tmem_row = tmem_base + (static_cast<uint32_t>(16 * j) << 16) + p.acol0;
-  StageCursor c{0, par, unit_block(p, 0, n_my, j)};
-  cursor_normalize(c, p, n_my, j);
+  const uint32_t code_off = 16u * lane, scale_off = kSlotResScales + 4u * (lane >> 2);
   int s = par;
   uint32_t ph = 0;
   uint32_t slot_i = 0;
-  for (int g = par; g < total; g += 2) {
-    issue_next();   // into the slot the previous stage freed
-    if (!tc_wait_warp(sm, &sm.empty[s], ph ^ 1u, p.status)) break;
-    tc_fence_after();
-    const uint8_t* slot = ring + slot_i * kPair;
-    cp_async_wait<R - 1>();
-    __syncwarp();
-    const int ks0 = 2 * c.st;
-    const bool two = ks0 + 1 < p.n_ks;
-    const uint32_t ta = tmem_row + static_cast<uint32_t>(s) * 64u;
-    // One k-step at a time into TMEM (a store reads its registers when it
-    // issues), so only one k-step's 16 result registers are live.
-    if (c.blk == nullptr) {
-      uint32_t r[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) r[i] = 0u;
-      tmem_st_16x256b_x4(ta, r);
-      if (two) tmem_st_16x256b_x4(ta + 32u, r);
-    } else if (two && ks0 + 1 < p.ks_core) {   // the common case: both k-steps residual
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t r[16];
-        dequant_residual<GM>(slot + h * kTcSlotBytes, p.sc_res, lane, r);
-        tmem_st_16x256b_x4(ta + 32u * h, r);
-      }
-    } else {
-      uint32_t r[16];
-      dequant_step<GM>(p, slot, ks0, lane, r);
-      tmem_st_16x256b_x4(ta, r);
-      if (two) {
-        dequant_step<GM>(p, slot + kTcSlotBytes, ks0 + 1, lane, r);
-        tmem_st_16x256b_x4(ta + 32u, r);
-      }
-    }
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();   // every lane is done reading the slot and storing to TMEM
-    if (lane == 0) mbar_arrive(smem_addr(&sm.full[s]));
-    if (++slot_i == R) slot_i = 0;
-    cursor_advance(c, p, n_my, j);
+  // After a stage: the next ring slot and stage buffer.
+  auto advance = [&]() {
+    slot_i = slot_i + 1 == R ? 0u : slot_i + 1;
     s += 2;
     if (s >= p.stages) {
       s -= p.stages;
       ph ^= 1u;
     }
+  };
+  for (int ui = 0; ui < n_my; ++ui) {
+    const uint8_t* blk = unit_block(p, ui, n_my, j);
+    int st = (par + ui * n_st) & 1;   // global stage ui * n_st + st has parity par
+    // Residual stages.
+    for (; st < n_rst; st += 2) {
+      issue_next();   // into the slot the previous stage freed
+      if (!tc_wait_fast(sm, &sm.empty[s], ph ^ 1u, p.status)) goto done;
+      tc_fence_after();
+      cp_async_wait<R - 1>();
+      __syncwarp();
+      const uint32_t ta = tmem_row + static_cast<uint32_t>(s) * 64u;
+      // One k-step at a time into TMEM (a store reads its registers when it
+      // issues), so only one k-step's 16 result registers are live.
+      if (blk != nullptr) {
+        const uint32_t slot = ring_s + slot_i * kPair;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[16];
+          dequant_residual_s<GM>(slot + h * kTcSlotBytes, code_off, scale_off, p.sc_res, r);
+          tmem_st_16x256b_x4(ta + 32u * h, r);
+        }
+      } else {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = 0u;
+        tmem_st_16x256b_x4(ta, r);
+        tmem_st_16x256b_x4(ta + 32u, r);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();   // every lane is done reading the slot and storing to TMEM
+      if (lane == 0) mbar_arrive(smem_addr(&sm.full[s]));
+      advance();
+    }
+    // The rest: a residual / core boundary, core and correction k-steps.
+    for (; st < n_st; st += 2) {
+      issue_next();
+      if (!tc_wait_warp(sm, &sm.empty[s], ph ^ 1u, p.status)) goto done;
+      tc_fence_after();
+      cp_async_wait<R - 1>();
+      __syncwarp();
+      const int ks0 = 2 * st;
+      const bool two = ks0 + 1 < p.n_ks;
+      const uint32_t ta = tmem_row + static_cast<uint32_t>(s) * 64u;
+      uint32_t r[16];
+      if (blk == nullptr) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = 0u;
+        tmem_st_16x256b_x4(ta, r);
+        if (two) tmem_st_16x256b_x4(ta + 32u, r);
+      } else {
+        const uint8_t* slot = ring + slot_i * kPair;
+        dequant_step<GM>(p, slot, ks0, lane, r);
+        tmem_st_16x256b_x4(ta, r);
+        if (two) {
+          dequant_step<GM>(p, slot + kTcSlotBytes, ks0 + 1, lane, r);
+          tmem_st_16x256b_x4(ta + 32u, r);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&sm.full[s]));
+      advance();
+    }
   }
+done:
   cp_async_wait_all();
 }
 
