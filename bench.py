@@ -19,7 +19,8 @@ Timing is on the device with CUDA events, max over ranks.
 bounded sample of vocabulary rows, scaled to the full head.
 
 --build times the GPU construction of the packed head instead (Algorithm 1:
-damped metric, truncated SVDs, quantisers; fp64) from a seeded dense head of
+damped metric, the randomised truncated SVDs of Eq. 4 (--svd exact for the
+exact ones), quantisers; fp64) from a seeded dense head of
 the Qwen3-8B shape and 16,384 calibration states (the largest calibration
 budget the pages report), with the oracle's builder on a slice of the head
 rows as the CPU baseline.
@@ -80,6 +81,10 @@ def parse_args():
     ap.add_argument("--build-steps", type=int, default=5)
     ap.add_argument("--build-warmup", type=int, default=3)
     ap.add_argument("--n-calib", type=int, default=16384, help="calibration states for --build")
+    ap.add_argument("--svd", choices=("randomized", "exact"), default="randomized",
+                    help="truncated SVDs of --build: the pages' randomised one (default) or the exact one")
+    ap.add_argument("--svd-oversample", type=int, default=None, help="randomised SVD: sketch columns beyond r")
+    ap.add_argument("--svd-power-iters", type=int, default=None, help="randomised SVD: subspace iteration steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -374,13 +379,28 @@ BUILD_ORACLE_ROWS = 4096
 BUILD_OWN_KERNELS = 13    # launches of the builder's own kernels per build (the rest is cuBLAS / cuSOLVER)
 
 
-def build_flops(V, d, r_c, r_r, N):
-    """fp64 flops of the dense products of one build (eigensolvers not counted):
-    H^T H, W^T W, E^T E (one triangle each), A_c = W V_c, W - A_c B_c,
+def sketch_cols(d, r, oversample):
+    """Columns of the randomised SVD's sketch (archead_svd_opts: r + oversample,
+    rounded up to a multiple of 64 above 64, at most d)."""
+    k = r + oversample
+    return min(d, (k + 63) // 64 * 64 if k > 64 else k)
+
+
+def build_flops(V, d, r_c, r_r, N, svd="exact", oversample=0, power_iters=0):
+    """fp64 flops of the dense products of one build (eigensolvers and QR not
+    counted): H^T H, W^T W, E^T E (one triangle each), A_c = W V_c, W - A_c B_c,
     E -= L_hat R_hat, A_w = E (T_p V_w), B_w, and the d x d products of T_p,
-    T_p^-1 and T_p E^T E T_p."""
-    return (N * d * d + 2 * V * d * d + 6 * V * d * r_c + 2 * V * d * r_r
-            + 8 * d ** 3 + 4 * d * d * r_r)
+    T_p^-1 and T_p E^T E T_p; for the randomised SVDs also, per factorisation
+    of rank r with k sketch columns, power_iters + 2 products G Q (d x d x k),
+    the projection Q^T G Q and the Ritz vectors (d x k x k each)."""
+    f = (N * d * d + 2 * V * d * d + 6 * V * d * r_c + 2 * V * d * r_r
+         + 8 * d ** 3 + 4 * d * d * r_r)
+    if svd == "randomized":
+        for r in (r_c, r_r):
+            if r > 0:
+                k = sketch_cols(d, r, oversample)
+                f += 2 * d * d * k * (power_iters + 2) + 4 * d * k * k
+    return f
 
 
 def dgemm_peak_tflops(torch, n=8192, reps=8):
@@ -438,20 +458,26 @@ def run_build(args):
     W, H = gen.dense_head_inputs_device(V, d, N)
     ws = bld.workspace(V, d, r_c, r_r, g, g_B, N)
     st = torch.cuda.current_stream()
+    svd_kw = dict(svd=args.svd)
+    if args.svd == "randomized":
+        svd_kw.update(oversample=bld.RANDOMIZED_OVERSAMPLE if args.svd_oversample is None else args.svd_oversample,
+                      power_iters=(bld.RANDOMIZED_POWER_ITERS if args.svd_power_iters is None
+                                   else args.svd_power_iters))
     for _ in range(args.build_warmup):
-        bld.build_head(W, H, r_c, r_r, g, g_B, ws=ws)
+        bld.build_head(W, H, r_c, r_r, g, g_B, ws=ws, **svd_kw)
     torch.cuda.synchronize()
     times = []
     with ClockSampler(0, period=0.05) as clk:
         for _ in range(args.build_steps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(st)
-            out = bld.build_head(W, H, r_c, r_r, g, g_B, ws=ws)
+            out = bld.build_head(W, H, r_c, r_r, g, g_B, ws=ws, **svd_kw)
             e1.record(st)
             torch.cuda.synchronize()
             times.append(e0.elapsed_time(e1) / 1e3)
     sec = sum(times) / len(times)
-    flops = build_flops(V, d, r_c, r_r, N)
+    flops = build_flops(V, d, r_c, r_r, N, svd=args.svd, oversample=svd_kw.get("oversample", 0),
+                        power_iters=svd_kw.get("power_iters", 0))
     peak = dgemm_peak_tflops(torch)
     # End to end: pinned host W and H in, every packed component back to pinned host memory.
     Wh, Hh = W.cpu().pin_memory(), H.cpu().pin_memory()
@@ -461,7 +487,7 @@ def run_build(args):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         Wd, Hd = Wh.cuda(non_blocking=True), Hh.cuda(non_blocking=True)
-        comps = bld.build_head(Wd, Hd, r_c, r_r, g, g_B, ws=ws)
+        comps = bld.build_head(Wd, Hd, r_c, r_r, g, g_B, ws=ws, **svd_kw)
         for k, v in comps.items():
             outs_h[k].copy_(v, non_blocking=True)
         torch.cuda.synchronize()
@@ -475,7 +501,8 @@ def run_build(args):
         ms_per_step=sec * 1e3, higher_is_better=False, scaling="weak", vs_baseline=None, dtype="f64",
         data="synthetic (seeded dense head: rank-32 Gaussian part + noise; anisotropic calibration states)",
         config=dict(workload=f"qwen3-8b-head build N{N}", V=V, d=d, r_c=r_c, r_r=r_r, g=g, g_B=g_B, n_calib=N,
-                    p=0.75, lam=1e-2, parallelism="replicas x1", l2="inputs larger than L2 (W 2.5 GB fp32)"),
+                    p=0.75, lam=1e-2, svd=svd_kw, parallelism="replicas x1",
+                    l2="inputs larger than L2 (W 2.5 GB fp32)"),
         roofline=dict(bound="tensor", achieved=flops / sec / 1e12, peak=peak, unit="TFLOP/s",
                       frac=flops / sec / 1e12 / peak, traffic=None, kernel="whole build (cuBLAS fp64 products, "
                       "cuSOLVER eigensolvers, own kernels)", algorithmic_flops_per_launch=flops,
@@ -485,7 +512,8 @@ def run_build(args):
             value=e_sec, unit="s per build", h2d_bytes_per_step=(W.numel() + H.numel()) * 4,
             d2h_bytes_per_step=sum(v.numel() * v.element_size() for v in out.values()),
             call="builder.build_head with pinned host W, H in and components out"),
-        clocks=clk.summary(), gpu_launches=args.build_steps * BUILD_OWN_KERNELS,
+        clocks=clk.summary(),
+        gpu_launches=args.build_steps * (BUILD_OWN_KERNELS + (2 if args.svd == "randomized" else 0)),
         step_seconds=times)
     print(json.dumps(line))
     return 0

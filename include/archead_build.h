@@ -16,10 +16,11 @@
  * Readings of points the paper leaves open (the same ones the CPU oracle takes):
  *   - the rank-r_c core A_c B_c is the exact truncated SVD of W with
  *     A_c = U S and B_c = V^T (Eq. 3 names no metric for it);
- *   - both truncated SVDs are exact (the paper's randomised SVD approximates
- *     this); they are computed as eigendecompositions of the d x d Gram
- *     matrices W^T W and T_p E^T E T_p, whose eigenvectors are the right
- *     singular vectors, with the left factor as W V (resp. E T_p V);
+ *   - both truncated SVDs are exact by default (the paper's randomised SVD
+ *     approximates this; archead_build_head_svd runs the randomised one);
+ *     they are computed from the d x d Gram matrices W^T W and T_p E^T E T_p,
+ *     whose eigenvectors are the right singular vectors, with the left factor
+ *     as W V (resp. E T_p V);
  *   - each singular pair's sign is fixed so that the largest-magnitude entry
  *     of the right singular vector is positive (first index on ties);
  *   - quantisers are symmetric: s = fp16(amax / qmax), codes
@@ -33,8 +34,9 @@
  *   - All matrices are row-major device buffers owned by the caller.  Scratch
  *     comes from the caller's workspace (archead_build_workspace_bytes,
  *     256-byte aligned); the only device memory allocated inside a call is
- *     what the cuBLAS and cuSOLVER handles it creates (and destroys before
- *     returning) reserve for themselves.
+ *     what the cuBLAS and cuSOLVER handles reserve for themselves: the
+ *     library creates one of each on a thread's first call on a device and
+ *     keeps them for the life of the process.
  *   - Arithmetic is IEEE fp64 (cuBLAS DGEMM / DSYRK / DSYMM for the dense
  *     products, cuSOLVER DSYEVD for the symmetric eigenproblems, this
  *     library's kernels for everything else).
@@ -104,6 +106,46 @@ ARCHEAD_API int archead_build_correction(const archead_desc* desc, const double*
 ARCHEAD_API int archead_build_head(const archead_desc* desc, const float* W, const float* H, int32_t n_calib,
                                    double lam, double p, const archead_device_components* out, void* workspace,
                                    size_t ws_bytes, archead_stream_t stream);
+
+/* Method of the two rank-r truncated SVDs (the core of Eq. 3 and E T_p of
+ * Eq. 4).
+ *   ARCHEAD_SVD_EXACT       the full eigendecomposition of the d x d Gram
+ *                           matrix (the readings above; archead_build_head
+ *                           and archead_build_correction use it).
+ *   ARCHEAD_SVD_RANDOMIZED  the randomised truncated SVD that §3.2 Eq. 4
+ *                           prescribes (used for both factorisations): on the
+ *                           Gram matrix G = M^T M, a Gaussian test matrix of
+ *                           k = min(d, r + oversample, rounded up to a
+ *                           multiple of 64 above 64) columns, power_iters
+ *                           steps of subspace iteration (Householder QR, then
+ *                           G Q), a last QR, and the eigenvectors of the k x k
+ *                           projection Q^T G Q mapped back (Rayleigh-Ritz;
+ *                           Halko, Martinsson and Tropp 2011).  The r Ritz
+ *                           vectors of the largest Ritz values, signs as
+ *                           above, replace the exact right singular vectors;
+ *                           the rest of the build is unchanged.  When
+ *                           k (d + k) > d^2 the exact method is used.  The
+ *                           test matrix is a function of seed and the entry
+ *                           index (SplitMix64, Box-Muller), so builds repeat.
+ * oversample >= 0, 0 <= power_iters <= 64; EINVAL otherwise. */
+enum { ARCHEAD_SVD_EXACT = 0, ARCHEAD_SVD_RANDOMIZED = 1 };
+typedef struct archead_svd_opts {
+  int32_t method;        /* ARCHEAD_SVD_EXACT or ARCHEAD_SVD_RANDOMIZED */
+  int32_t oversample;    /* extra sketch columns beyond r */
+  int32_t power_iters;   /* subspace iteration steps */
+  uint64_t seed;         /* of the Gaussian test matrix */
+} archead_svd_opts;
+
+/* archead_build_correction / archead_build_head with the SVD method of svd
+ * (NULL: exact).  Same arguments, workspace and errors otherwise. */
+ARCHEAD_API int archead_build_correction_svd(const archead_desc* desc, const double* E, const double* T_p,
+                                             const double* T_p_inv, const archead_svd_opts* svd, int8_t* A,
+                                             uint16_t* s_A, int8_t* B, uint16_t* s_B, void* workspace,
+                                             size_t ws_bytes, archead_stream_t stream);
+ARCHEAD_API int archead_build_head_svd(const archead_desc* desc, const float* W, const float* H, int32_t n_calib,
+                                       double lam, double p, const archead_svd_opts* svd,
+                                       const archead_device_components* out, void* workspace, size_t ws_bytes,
+                                       archead_stream_t stream);
 
 /* Description of this thread's last failure ("" if none). */
 ARCHEAD_API const char* archead_build_last_error(void);

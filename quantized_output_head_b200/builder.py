@@ -52,8 +52,18 @@ _blib = ctypes.CDLL(BUILD_LIB_PATH)
 
 EXPORTED_BUILD = (
     "archead_build_workspace_bytes", "archead_build_quantize", "archead_build_metric",
-    "archead_build_correction", "archead_build_head", "archead_build_last_error",
+    "archead_build_correction", "archead_build_head", "archead_build_correction_svd", "archead_build_head_svd",
+    "archead_build_last_error",
 )
+ARCHEAD_SVD_EXACT, ARCHEAD_SVD_RANDOMIZED = 0, 1
+# Defaults of the randomised truncated SVD (sketch columns r + oversample,
+# subspace iteration steps); see archead_svd_opts.
+RANDOMIZED_OVERSAMPLE, RANDOMIZED_POWER_ITERS = 32, 2
+
+
+class ArcheadSvdOpts(ctypes.Structure):
+    _fields_ = [("method", ctypes.c_int32), ("oversample", ctypes.c_int32), ("power_iters", ctypes.c_int32),
+                ("seed", ctypes.c_uint64)]
 
 
 class ArcheadDeviceComponents(ctypes.Structure):
@@ -69,6 +79,10 @@ _sig = {
     "archead_build_correction": (ctypes.c_int, [_DESC, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "archead_build_head": (ctypes.c_int, [_DESC, _vp, _vp, _i32, _f64, _f64, ctypes.POINTER(ArcheadDeviceComponents),
                                           _vp, _sz, _vp]),
+    "archead_build_correction_svd": (ctypes.c_int, [_DESC, _vp, _vp, _vp, ctypes.POINTER(ArcheadSvdOpts), _vp, _vp,
+                                                    _vp, _vp, _vp, _sz, _vp]),
+    "archead_build_head_svd": (ctypes.c_int, [_DESC, _vp, _vp, _i32, _f64, _f64, ctypes.POINTER(ArcheadSvdOpts),
+                                              ctypes.POINTER(ArcheadDeviceComponents), _vp, _sz, _vp]),
     "archead_build_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _sig.items():
@@ -135,8 +149,19 @@ def metric(H: torch.Tensor, lam: float, p: float) -> Tuple[torch.Tensor, torch.T
     return T_p, T_inv
 
 
-def correction(E: torch.Tensor, T_p: torch.Tensor, T_inv: torch.Tensor, r_r: int, g_B: int) -> Dict[str, torch.Tensor]:
-    """Eq. 4-5 with INT8 factors: A, s_A, B, s_B from the core's remainder E [V, d]."""
+def svd_opts(svd: str = "exact", oversample: int = RANDOMIZED_OVERSAMPLE, power_iters: int = RANDOMIZED_POWER_ITERS,
+             seed: int = 0) -> ArcheadSvdOpts:
+    """archead_svd_opts for svd = "exact" or "randomized"."""
+    if svd not in ("exact", "randomized"):
+        raise ValueError(f"svd must be 'exact' or 'randomized', not {svd!r}")
+    method = ARCHEAD_SVD_EXACT if svd == "exact" else ARCHEAD_SVD_RANDOMIZED
+    return ArcheadSvdOpts(method, int(oversample), int(power_iters), int(seed) & (2**64 - 1))
+
+
+def correction(E: torch.Tensor, T_p: torch.Tensor, T_inv: torch.Tensor, r_r: int, g_B: int, svd: str = "exact",
+               **svd_kw) -> Dict[str, torch.Tensor]:
+    """Eq. 4-5 with INT8 factors: A, s_A, B, s_B from the core's remainder E [V, d]
+    (svd: "exact" or "randomized", with svd_opts' keywords)."""
     for t, n in ((E, "E"), (T_p, "T_p"), (T_inv, "T_inv")):
         _dev(t, torch.float64, n)
     V, d = E.shape
@@ -146,18 +171,21 @@ def correction(E: torch.Tensor, T_p: torch.Tensor, T_inv: torch.Tensor, r_r: int
                s_A=torch.empty(V, dtype=torch.int16, device=E.device),
                B=torch.empty(r_r, d, dtype=torch.int8, device=E.device),
                s_B=torch.empty(r_r, d // g_B, dtype=torch.int16, device=E.device))
-    _check(_blib.archead_build_correction(ctypes.byref(desc), E.data_ptr(), T_p.data_ptr(), T_inv.data_ptr(),
-                                          out["A"].data_ptr(), out["s_A"].data_ptr(), out["B"].data_ptr(),
-                                          out["s_B"].data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
-           "archead_build_correction")
+    opts = svd_opts(svd, **svd_kw)
+    _check(_blib.archead_build_correction_svd(ctypes.byref(desc), E.data_ptr(), T_p.data_ptr(), T_inv.data_ptr(),
+                                              ctypes.byref(opts), out["A"].data_ptr(), out["s_A"].data_ptr(),
+                                              out["B"].data_ptr(), out["s_B"].data_ptr(), ws.data_ptr(), ws.numel(),
+                                              _stream()),
+           "archead_build_correction_svd")
     return out
 
 
 def build_head(W: torch.Tensor, H: torch.Tensor, r_c: int, r_r: int, g: int, g_B: int, p: float = 0.75,
-               lam: float = 1e-2, ws: torch.Tensor = None) -> Dict[str, torch.Tensor]:
+               lam: float = 1e-2, ws: torch.Tensor = None, svd: str = "exact", **svd_kw) -> Dict[str, torch.Tensor]:
     """Algorithm 1: every packed component (device tensors, canonical names;
     scales as int16 storage of fp16 bits) from the dense head W [V, d] and
-    calibration states H [N, d], both fp32 CUDA tensors."""
+    calibration states H [N, d], both fp32 CUDA tensors.  svd: "exact" or
+    "randomized" (the truncated SVDs; svd_opts' keywords)."""
     _dev(W, torch.float32, "W")
     _dev(H, torch.float32, "H")
     V, d = W.shape
@@ -176,8 +204,10 @@ def build_head(W: torch.Tensor, H: torch.Tensor, r_c: int, r_r: int, g: int, g_B
                B=torch.empty(r_r, d, dtype=torch.int8, device=dev),
                s_B=torch.empty(r_r, d // g_B, dtype=torch.int16, device=dev))
     dc = ArcheadDeviceComponents(**{k: (v.data_ptr() if v.numel() else None) for k, v in out.items()})
-    _check(_blib.archead_build_head(ctypes.byref(desc), W.data_ptr(), H.data_ptr(), N, float(lam), float(p),
-                                    ctypes.byref(dc), ws.data_ptr(), ws.numel(), _stream()), "archead_build_head")
+    opts = svd_opts(svd, **svd_kw)
+    _check(_blib.archead_build_head_svd(ctypes.byref(desc), W.data_ptr(), H.data_ptr(), N, float(lam), float(p),
+                                        ctypes.byref(opts), ctypes.byref(dc), ws.data_ptr(), ws.numel(), _stream()),
+           "archead_build_head_svd")
     return out
 
 

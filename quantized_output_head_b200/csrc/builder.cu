@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 #include <cusolverDn.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdarg>
@@ -129,15 +130,15 @@ __global__ void scale_columns_kernel(const double* __restrict__ Q, const double*
 }
 
 // The r eigenvectors of the largest eigenvalues (DSYEVD orders them
-// ascending: columns d-1, d-2, ...) as columns 0..r-1 of Vr (column-major
-// d x r), in descending order, each negated when its first entry of largest
-// magnitude is negative.  One block per vector.
-__global__ void top_vectors_kernel(const double* __restrict__ Q, int d, int r, double* __restrict__ Vr) {
+// ascending: columns n-1, n-2, ... of the column-major d x n matrix Q) as
+// columns 0..r-1 of Vr (column-major d x r), in descending order, each negated
+// when its first entry of largest magnitude is negative.  One block per vector.
+__global__ void top_vectors_kernel(const double* __restrict__ Q, int d, int n, int r, double* __restrict__ Vr) {
   __shared__ double best_v[kThreads];
   __shared__ int best_i[kThreads];
   const int i = blockIdx.x;
   if (i >= r) return;
-  const double* src = Q + static_cast<size_t>(d - 1 - i) * d;
+  const double* src = Q + static_cast<size_t>(n - 1 - i) * d;
   double bv = -1.0;
   int bi = INT_MAX;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {   // increasing j: '>' keeps the first maximum
@@ -165,6 +166,25 @@ __global__ void top_vectors_kernel(const double* __restrict__ Q, int d, int r, d
   const double sgn = (j0 < d && src[j0] < 0.0) ? -1.0 : 1.0;
   double* dst = Vr + static_cast<size_t>(i) * d;
   for (int j = threadIdx.x; j < d; j += blockDim.x) dst[j] = sgn * src[j];
+}
+
+// Standard normal entries of the randomised SVD's test matrix, a function of
+// the seed and the entry's index only: SplitMix64 (Steele, Lea, Flood 2014)
+// of seed + 2i and seed + 2i + 1 gives two 53-bit uniforms in (0, 1), and the
+// Box-Muller transform the normal deviate.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  x += 0x9E3779B97F4A7C15ull;
+  x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+  x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+  return x ^ (x >> 31);
+}
+__global__ void gaussian_kernel(double* __restrict__ x, size_t n, uint64_t seed) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const double u1 = (static_cast<double>(splitmix64(seed + 2 * i) >> 11) + 0.5) * 0x1.0p-53;
+    const double u2 = (static_cast<double>(splitmix64(seed + 2 * i + 1) >> 11) + 0.5) * 0x1.0p-53;
+    x[i] = sqrt(-2.0 * log(u1)) * cospi(2.0 * u2);
+  }
 }
 
 // Symmetric quantiser, one warp per group of G consecutive elements of a row:
@@ -218,32 +238,43 @@ int launch_quantize(const double* x, int rows, int cols, int bits, int G, int8_t
 }
 
 // ----------------------------------------------------------- library state
+// cuBLAS and cuSOLVER handles, created on a thread's first call on a device
+// and kept for the life of the process (creating and destroying them on every
+// call measured sporadic stalls of 0.3-1.3 s on builds of ~0.4 s); each call
+// binds them to its stream.
 struct Handles {
   cublasHandle_t blas = nullptr;
   cusolverDnHandle_t solver = nullptr;
-  cudaStream_t stream = nullptr;
-  bool bound = false;
-  // Work queued on the stream may still use the handles' scratch when a call
-  // returns early with an error: drain it before the handles go.
-  ~Handles() {
-    if (bound) cudaStreamSynchronize(stream);
-    if (blas) cublasDestroy(blas);
-    if (solver) cusolverDnDestroy(solver);
-  }
-  int init(cudaStream_t st) {
-    stream = st;
-    bound = true;
-    CK_BLAS(cublasCreate(&blas));
-    CK_BLAS(cublasSetStream(blas, st));
-    CK_SOLVER(cusolverDnCreate(&solver));
-    CK_SOLVER(cusolverDnSetStream(solver, st));
-    return ARCHEAD_OK;
-  }
 };
 
+constexpr int kMaxDevices = 64;
+
+int get_handles(cudaStream_t st, const Handles** out) {
+  thread_local Handles cache[kMaxDevices];
+  int dev = 0;
+  CK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) {
+    set_err("device %d out of range", dev);
+    return ARCHEAD_EINVAL;
+  }
+  Handles& h = cache[dev];
+  if (h.blas == nullptr) CK_BLAS(cublasCreate(&h.blas));
+  if (h.solver == nullptr) CK_SOLVER(cusolverDnCreate(&h.solver));
+  CK_BLAS(cublasSetStream(h.blas, st));
+  CK_SOLVER(cusolverDnSetStream(h.solver, st));
+  *out = &h;
+  return ARCHEAD_OK;
+}
+
+// Solver scratch (doubles) for a d x d eigendecomposition, and for the
+// randomised SVD's Householder QR of up to d columns.
 int eig_lwork(cusolverDnHandle_t h, int d, int* lwork) {
+  int le = 0, lq = 0, lo = 0;
   CK_SOLVER(cusolverDnDsyevd_bufferSize(h, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, d, nullptr, d,
-                                        nullptr, lwork));
+                                        nullptr, &le));
+  CK_SOLVER(cusolverDnDgeqrf_bufferSize(h, d, d, nullptr, d, &lq));
+  CK_SOLVER(cusolverDnDorgqr_bufferSize(h, d, d, d, nullptr, d, nullptr, &lo));
+  *lwork = std::max(le, std::max(lq, lo));
   return ARCHEAD_OK;
 }
 
@@ -302,6 +333,87 @@ int eigh(const Handles& h, double* A, int d, double* w, double* work, int lwork,
   return ARCHEAD_OK;
 }
 
+// Method of the two rank-r factorisations (archead_svd_opts).
+struct SvdOpts {
+  int method = ARCHEAD_SVD_EXACT;
+  int oversample = 0, power_iters = 0;
+  uint64_t seed = 0;
+};
+
+// Columns of the randomised method's sketch: k = min(d, r + oversample, above
+// 64 rounded up to a multiple of 64: the solver's blocked QR measured up to 2x
+// slower on other widths); 0 when the sketch would not fit beside its k x k
+// projection in a d x d region (k (d + k) > d^2), where the exact method is
+// used instead.
+int sketch_cols(int d, int r, const SvdOpts& o) {
+  if (o.method != ARCHEAD_SVD_RANDOMIZED) return 0;
+  long long k = static_cast<long long>(r) + o.oversample;
+  if (k > 64) k = (k + 63) / 64 * 64;
+  k = std::min<long long>(d, k);
+  return k * (d + k) <= static_cast<long long>(d) * d ? static_cast<int>(k) : 0;
+}
+
+// Householder QR of the column-major d x k matrix Y, replaced by its Q factor.
+int orthonormalise(const Handles& h, const Plan& pl, int lwork, double* Y, int d, int k) {
+  int lq = 0, lo = 0;
+  CK_SOLVER(cusolverDnDgeqrf_bufferSize(h.solver, d, k, Y, d, &lq));
+  CK_SOLVER(cusolverDnDorgqr_bufferSize(h.solver, d, k, k, Y, d, pl.fp, &lo));
+  if (lq > lwork || lo > lwork) {
+    set_err("orthonormalise: QR scratch %d / %d > %d", lq, lo, lwork);
+    return ARCHEAD_ENOMEM;
+  }
+  CK_SOLVER(cusolverDnDgeqrf(h.solver, d, k, Y, d, pl.fp, pl.eig, lwork, pl.info));
+  CK_SOLVER(cusolverDnDorgqr(h.solver, d, k, k, Y, d, pl.fp, pl.eig, lwork, pl.info));
+  return ARCHEAD_OK;
+}
+
+// The r right singular vectors of M from its d x d Gram matrix G = M^T M
+// (lower triangle, column-major), as columns of Vr (column-major d x r), in
+// descending order of the singular value, signs as top_vectors_kernel fixes
+// them.  s1, s2: d x d scratch regions.  Exact: the eigendecomposition of G
+// (G is overwritten).  Randomised (ARCHead paper §3.2 Eq. 4; Halko, Martinsson
+// and Tropp 2011, subspace iteration and Rayleigh-Ritz on G): Y = G Omega with
+// a Gaussian Omega of k columns; power_iters times Q = qr(Y), Y = G Q; then
+// Q = qr(Y), the k x k projection Q^T G Q, its eigenvectors Phi, and the Ritz
+// vectors Q Phi of the r largest Ritz values.
+int right_vectors(const Handles& h, const Plan& pl, int lwork, double* G, double* s1, double* s2, int d, int r,
+                  const SvdOpts& o, double* Vr, cudaStream_t st) {
+  const int k = sketch_cols(d, r, o);
+  if (k == 0) {
+    CK(eigh(h, G, d, pl.w, pl.eig, lwork, pl.info, st));
+    top_vectors_kernel<<<r, kThreads, 0, st>>>(G, d, d, r, Vr);
+    CK_CUDA(cudaGetLastError());
+    return ARCHEAD_OK;
+  }
+  const double zero = 0.0, one = 1.0;
+  double* Y = s1;                                        // d x k: the sketch, then Q
+  double* P = s1 + static_cast<size_t>(d) * k;           // k x k projection (fits: k (d + k) <= d^2)
+  double* Z = s2;                                        // d x k: G Q, then the Ritz vectors
+  gaussian_kernel<<<grid_for(static_cast<size_t>(d) * k), kThreads, 0, st>>>(Z, static_cast<size_t>(d) * k, o.seed);
+  CK_CUDA(cudaGetLastError());
+  CK_BLAS(cublasDsymm(h.blas, CUBLAS_SIDE_LEFT, CUBLAS_FILL_MODE_LOWER, d, k, &one, G, d, Z, d, &zero, Y, d));
+  for (int it = 0; it < o.power_iters; ++it) {
+    CK(orthonormalise(h, pl, lwork, Y, d, k));
+    CK_BLAS(cublasDsymm(h.blas, CUBLAS_SIDE_LEFT, CUBLAS_FILL_MODE_LOWER, d, k, &one, G, d, Y, d, &zero, Z, d));
+    CK_CUDA(cudaMemcpyAsync(Y, Z, static_cast<size_t>(d) * k * sizeof(double), cudaMemcpyDeviceToDevice, st));
+  }
+  CK(orthonormalise(h, pl, lwork, Y, d, k));
+  CK_BLAS(cublasDsymm(h.blas, CUBLAS_SIDE_LEFT, CUBLAS_FILL_MODE_LOWER, d, k, &one, G, d, Y, d, &zero, Z, d));
+  CK_BLAS(cublasDgemm(h.blas, CUBLAS_OP_T, CUBLAS_OP_N, k, k, d, &one, Y, d, Z, d, &zero, P, k));
+  int lk = 0;
+  CK_SOLVER(cusolverDnDsyevd_bufferSize(h.solver, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, k, P, k, pl.w,
+                                        &lk));
+  if (lk > lwork) {
+    set_err("right_vectors: eigensolver scratch %d > %d", lk, lwork);
+    return ARCHEAD_ENOMEM;
+  }
+  CK(eigh(h, P, k, pl.w, pl.eig, lwork, pl.info, st));
+  CK_BLAS(cublasDgemm(h.blas, CUBLAS_OP_N, CUBLAS_OP_N, d, k, k, &one, Y, d, P, k, &zero, Z, d));
+  top_vectors_kernel<<<r, kThreads, 0, st>>>(Z, d, k, r, Vr);
+  CK_CUDA(cudaGetLastError());
+  return ARCHEAD_OK;
+}
+
 // §3.1 Eq. 1-2 into Tp, Ti (column-major d x d; both symmetric).  Uses
 // big1 (H in fp64), mat[0] (C, then Q), mat[3], mat[4] (Q Lambda^{+-p}).
 int metric_impl(const Handles& h, const Plan& pl, int lwork, int d, int N, const float* H, double lam, double p,
@@ -336,8 +448,8 @@ int metric_impl(const Handles& h, const Plan& pl, int lwork, int d, int N, const
 // d x V matrix E^T).  Uses mat[0] (E^T E), mat[3] (E^T E T_p), mat[4]
 // (T_p E^T E T_p, then its eigenvectors), vec (V_w), vec2, fac.
 int correction_impl(const Handles& h, const Plan& pl, int lwork, int V, int d, int r_r, int g_B, const double* E,
-                    const double* Tp, const double* Ti, int8_t* A, uint16_t* s_A, int8_t* B, uint16_t* s_B,
-                    cudaStream_t st) {
+                    const double* Tp, const double* Ti, const SvdOpts& svd, int8_t* A, uint16_t* s_A, int8_t* B,
+                    uint16_t* s_B, cudaStream_t st) {
   const double zero = 0.0, one = 1.0;
   // The right singular vectors of E T_p are the eigenvectors of its Gram
   // matrix (E T_p)^T (E T_p) = T_p (E^T E) T_p.
@@ -345,9 +457,7 @@ int correction_impl(const Handles& h, const Plan& pl, int lwork, int V, int d, i
   CK_BLAS(cublasDsymm(h.blas, CUBLAS_SIDE_LEFT, CUBLAS_FILL_MODE_LOWER, d, d, &one, pl.mat[0], d, Tp, d, &zero,
                       pl.mat[3], d));
   CK_BLAS(cublasDgemm(h.blas, CUBLAS_OP_N, CUBLAS_OP_N, d, d, d, &one, Tp, d, pl.mat[3], d, &zero, pl.mat[4], d));
-  CK(eigh(h, pl.mat[4], d, pl.w, pl.eig, lwork, pl.info, st));
-  top_vectors_kernel<<<r_r, kThreads, 0, st>>>(pl.mat[4], d, r_r, pl.vec);
-  CK_CUDA(cudaGetLastError());
+  CK(right_vectors(h, pl, lwork, pl.mat[4], pl.mat[0], pl.mat[3], d, r_r, svd, pl.vec, st));
   // Z = T_p V_w (d x r_r); A_w = U S = E T_p V_w = E Z, row-major [V, r_r] =
   // the column-major r_r x V matrix Z^T E^T.
   CK_BLAS(cublasDgemm(h.blas, CUBLAS_OP_N, CUBLAS_OP_N, d, r_r, d, &one, Tp, d, pl.vec, d, &zero, pl.vec2, d));
@@ -368,8 +478,9 @@ bool valid_desc(const archead_desc* x) {
 }
 
 int query_lwork(int d, int* lwork) {
-  Handles h;
-  CK(h.init(nullptr));
+  const Handles* hp = nullptr;
+  CK(get_handles(nullptr, &hp));
+  const Handles& h = *hp;
   return eig_lwork(h.solver, d, lwork);
 }
 
@@ -423,8 +534,9 @@ ARCHEAD_API int archead_build_metric(int32_t d, int32_t n_calib, const float* H,
     return ARCHEAD_EINVAL;
   }
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  Handles h;
-  CK(h.init(st));
+  const Handles* hp = nullptr;
+  CK(get_handles(st, &hp));
+  const Handles& h = *hp;
   int lwork = 0;
   CK(eig_lwork(h.solver, d, &lwork));
   const Plan need = make_plan(nullptr, 1, d, n_calib, 1, lwork);
@@ -435,32 +547,61 @@ ARCHEAD_API int archead_build_metric(int32_t d, int32_t n_calib, const float* H,
   return ARCHEAD_OK;
 }
 
-ARCHEAD_API int archead_build_correction(const archead_desc* desc, const double* E, const double* T_p,
-                                         const double* T_p_inv, int8_t* A, uint16_t* s_A, int8_t* B,
-                                         uint16_t* s_B, void* workspace, size_t ws_bytes,
-                                         archead_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// archead_svd_opts -> SvdOpts (null: exact); false on a bad option.
+bool read_svd(const archead_svd_opts* o, SvdOpts* out) {
+  *out = SvdOpts{};
+  if (o == nullptr) return true;
+  if ((o->method != ARCHEAD_SVD_EXACT && o->method != ARCHEAD_SVD_RANDOMIZED) || o->oversample < 0 ||
+      o->power_iters < 0 || o->power_iters > 64)
+    return false;
+  out->method = o->method;
+  out->oversample = o->oversample;
+  out->power_iters = o->power_iters;
+  out->seed = o->seed;
+  return true;
+}
+
+int build_correction(const archead_desc* desc, const double* E, const double* T_p, const double* T_p_inv,
+                     const archead_svd_opts* svd_opts, int8_t* A, uint16_t* s_A, int8_t* B, uint16_t* s_B,
+                     void* workspace, size_t ws_bytes, archead_stream_t stream) {
   g_err[0] = '\0';
+  SvdOpts svd;
+  if (!read_svd(svd_opts, &svd)) {
+    set_err("correction: bad SVD options");
+    return ARCHEAD_EINVAL;
+  }
   if (!valid_desc(desc) || desc->r_r < 1 || !E || !T_p || !T_p_inv || !A || !s_A || !B || !s_B) {
     set_err("correction: bad argument");
     return ARCHEAD_EINVAL;
   }
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  Handles h;
-  CK(h.init(st));
+  const Handles* hp = nullptr;
+  CK(get_handles(st, &hp));
+  const Handles& h = *hp;
   int lwork = 0;
   CK(eig_lwork(h.solver, desc->d, &lwork));
   const Plan need = make_plan(nullptr, desc->V, desc->d, 1, desc->r_r, lwork);
   CK(check_ws(need, workspace, ws_bytes));
   const Plan pl = make_plan(static_cast<uint8_t*>(workspace), desc->V, desc->d, 1, desc->r_r, lwork);
-  CK(correction_impl(h, pl, lwork, desc->V, desc->d, desc->r_r, desc->g_B, E, T_p, T_p_inv, A, s_A, B, s_B, st));
+  CK(correction_impl(h, pl, lwork, desc->V, desc->d, desc->r_r, desc->g_B, E, T_p, T_p_inv, svd, A, s_A, B, s_B,
+                     st));
   CK_CUDA(cudaStreamSynchronize(st));
   return ARCHEAD_OK;
 }
 
-ARCHEAD_API int archead_build_head(const archead_desc* desc, const float* W, const float* H, int32_t n_calib,
-                                   double lam, double p, const archead_device_components* out, void* workspace,
-                                   size_t ws_bytes, archead_stream_t stream) {
+int build_head(const archead_desc* desc, const float* W, const float* H, int32_t n_calib, double lam, double p,
+               const archead_svd_opts* svd_opts, const archead_device_components* out, void* workspace,
+               size_t ws_bytes, archead_stream_t stream) {
   g_err[0] = '\0';
+  SvdOpts svd;
+  if (!read_svd(svd_opts, &svd)) {
+    set_err("build_head: bad SVD options");
+    return ARCHEAD_EINVAL;
+  }
   if (!valid_desc(desc) || desc->r_c + desc->r_r < 1 || !W || !H || n_calib < 1 || !out || !out->q ||
       !out->s_res || !(lam >= 0.0) || !std::isfinite(p)) {
     set_err("build_head: bad argument");
@@ -473,8 +614,9 @@ ARCHEAD_API int archead_build_head(const archead_desc* desc, const float* W, con
     return ARCHEAD_EINVAL;
   }
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  Handles h;
-  CK(h.init(st));
+  const Handles* hp = nullptr;
+  CK(get_handles(st, &hp));
+  const Handles& h = *hp;
   int lwork = 0;
   CK(eig_lwork(h.solver, d, &lwork));
   const int rmax = r_c > r_r ? r_c : r_r;
@@ -501,10 +643,8 @@ ARCHEAD_API int archead_build_head(const archead_desc* desc, const float* W, con
   CK_CUDA(cudaMemcpyAsync(pl.big1, pl.big0, nw * sizeof(double), cudaMemcpyDeviceToDevice, st));
   if (r_c > 0) {
     CK_BLAS(cublasDsyrk(h.blas, CUBLAS_FILL_MODE_LOWER, CUBLAS_OP_N, d, V, &one, pl.big0, d, &zero, pl.mat[0], d));
-    CK(eigh(h, pl.mat[0], d, pl.w, pl.eig, lwork, pl.info, st));
     // V_c, column-major d x r_c: also B_c = V_c^T as a row-major [r_c, d].
-    top_vectors_kernel<<<r_c, kThreads, 0, st>>>(pl.mat[0], d, r_c, pl.vec);
-    CK_CUDA(cudaGetLastError());
+    CK(right_vectors(h, pl, lwork, pl.mat[0], pl.mat[3], pl.mat[4], d, r_c, svd, pl.vec, st));
     // A_c row-major [V, r_c] = the column-major r_c x V matrix V_c^T W^T.
     CK_BLAS(cublasDgemm(h.blas, CUBLAS_OP_T, CUBLAS_OP_N, r_c, V, d, &one, pl.vec, d, pl.big0, d, &zero, pl.fac,
                         r_c));
@@ -526,10 +666,41 @@ ARCHEAD_API int archead_build_head(const archead_desc* desc, const float* W, con
 
   // Eq. 4-5: the activation-metric correction of E.
   if (r_r > 0)
-    CK(correction_impl(h, pl, lwork, V, d, r_r, desc->g_B, pl.big1, Tp, Ti, out->A, out->s_A, out->B, out->s_B,
-                       st));
+    CK(correction_impl(h, pl, lwork, V, d, r_r, desc->g_B, pl.big1, Tp, Ti, svd, out->A, out->s_A, out->B,
+                       out->s_B, st));
   CK_CUDA(cudaStreamSynchronize(st));
   return ARCHEAD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ARCHEAD_API int archead_build_correction(const archead_desc* desc, const double* E, const double* T_p,
+                                         const double* T_p_inv, int8_t* A, uint16_t* s_A, int8_t* B,
+                                         uint16_t* s_B, void* workspace, size_t ws_bytes,
+                                         archead_stream_t stream) {
+  return build_correction(desc, E, T_p, T_p_inv, nullptr, A, s_A, B, s_B, workspace, ws_bytes, stream);
+}
+
+ARCHEAD_API int archead_build_correction_svd(const archead_desc* desc, const double* E, const double* T_p,
+                                             const double* T_p_inv, const archead_svd_opts* svd, int8_t* A,
+                                             uint16_t* s_A, int8_t* B, uint16_t* s_B, void* workspace,
+                                             size_t ws_bytes, archead_stream_t stream) {
+  return build_correction(desc, E, T_p, T_p_inv, svd, A, s_A, B, s_B, workspace, ws_bytes, stream);
+}
+
+ARCHEAD_API int archead_build_head(const archead_desc* desc, const float* W, const float* H, int32_t n_calib,
+                                   double lam, double p, const archead_device_components* out, void* workspace,
+                                   size_t ws_bytes, archead_stream_t stream) {
+  return build_head(desc, W, H, n_calib, lam, p, nullptr, out, workspace, ws_bytes, stream);
+}
+
+ARCHEAD_API int archead_build_head_svd(const archead_desc* desc, const float* W, const float* H, int32_t n_calib,
+                                       double lam, double p, const archead_svd_opts* svd,
+                                       const archead_device_components* out, void* workspace, size_t ws_bytes,
+                                       archead_stream_t stream) {
+  return build_head(desc, W, H, n_calib, lam, p, svd, out, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"
