@@ -171,19 +171,32 @@ __device__ __forceinline__ void dequant_residual(const uint8_t* slot, float sc, 
   }
 }
 
-// The same from the slot's shared-memory address: codes at slot + code_off
-// (code_off = 16 lane), this lane's scale pair at slot + scale_off
-// (scale_off = kSlotResScales + 4 gr).
+// The same in two parts, so that a stage's shared-memory loads can all be in
+// flight before any unpacking: the codes (16 bytes at slot + code_off,
+// code_off = 16 lane) and this lane's scale pair of each local group (at
+// slot + scale_off, scale_off = kSlotResScales + 4 gr) of one k-step ...
 template <int GM>
-__device__ __forceinline__ void dequant_residual_s(uint32_t slot, uint32_t code_off, uint32_t scale_off, float sc,
-                                                   uint32_t (&r)[16]) {
-  const uint4 c = lds128(slot + code_off);
-  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+struct ResidualRaw {
+  uint4 c;
+  uint32_t s[1 << GM];
+};
+template <int GM>
+__device__ __forceinline__ ResidualRaw<GM> load_residual(uint32_t slot, uint32_t code_off, uint32_t scale_off) {
+  ResidualRaw<GM> x;
+  x.c = lds128(slot + code_off);
+#pragma unroll
+  for (int g = 0; g < (1 << GM); ++g) x.s[g] = lds32(slot + scale_off + g * kSresGroupBytes);
+  return x;
+}
+// ... then the tcgen05.st operands from them.
+template <int GM>
+__device__ __forceinline__ void dequant_residual_raw(const ResidualRaw<GM>& x, float sc, uint32_t (&r)[16]) {
+  const uint32_t w[4] = {x.c.x, x.c.y, x.c.z, x.c.w};
   uint32_t s0 = 0, s1 = 0;
 #pragma unroll
   for (int st = 0; st < 4; ++st) {
     if (st % (4 >> GM) == 0) {
-      const float2 f = half2_bits_to_float2(lds32(slot + scale_off + (st >> (2 - GM)) * kSresGroupBytes));
+      const float2 f = half2_bits_to_float2(x.s[st >> (2 - GM)]);
       s0 = pack_half2(f.x * sc, f.x * sc);
       s1 = pack_half2(f.y * sc, f.y * sc);
     }
@@ -348,12 +361,13 @@ __device__ void dequant_loop(const TcParams& p, const TcSmem& sm, uint32_t tmem_
       // issues), so only one k-step's 16 result registers are live.
       if (blk != nullptr) {
         const uint32_t slot = ring_s + slot_i * kPair;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[16];
-          dequant_residual_s<GM>(slot + h * kTcSlotBytes, code_off, scale_off, p.sc_res, r);
-          tmem_st_16x256b_x4(ta + 32u * h, r);
-        }
+        const ResidualRaw<GM> x0 = load_residual<GM>(slot, code_off, scale_off);
+        const ResidualRaw<GM> x1 = load_residual<GM>(slot + kTcSlotBytes, code_off, scale_off);
+        uint32_t r[16];
+        dequant_residual_raw<GM>(x0, p.sc_res, r);
+        tmem_st_16x256b_x4(ta, r);
+        dequant_residual_raw<GM>(x1, p.sc_res, r);
+        tmem_st_16x256b_x4(ta + 32u, r);
       } else {
         uint32_t r[16];
 #pragma unroll
