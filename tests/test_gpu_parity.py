@@ -491,6 +491,39 @@ def test_argmax_ties_resolve_to_lowest_index(qoh, T, spacing):
     check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, targets)
 
 
+@pytest.mark.parametrize("T,kernel", [(5, "decode"), (24, "tensor_core")])
+def test_activation_splits_with_uneven_columns(qoh, T, kernel):
+    """Column ranges of h under powers of two of their own: on the tensor-core
+    path the activation kernel splits d over 8 blocks of 128 columns at this
+    shape and the last split rescales the others to the token's exponent; on
+    the decode path each residual warp scales its own 256 columns (warps past
+    d have none).  Tokens whose columns are zero outside one split, 2^40
+    larger or 2^-40 smaller in one split, or zero but for one entry, against
+    the oracle."""
+    shape = (3000, 1024, 64, 16, 64, 64)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=616)
+    h_bits, targets = gen.random_hidden(1024, T, seed=617, V=shape[0])
+    h = gen.bf16_bits_to_f32(h_bits).copy()
+    h[0, 128:] = 0.0                                  # only the first split
+    h[1, :896] = 0.0                                  # only the last split
+    h[2, 384:512] *= np.float32(2.0 ** 40)            # one split far above the rest
+    h[3, 640:768] *= np.float32(2.0 ** -40)           # one split far below the rest
+    h[4, :] = 0.0
+    h[4, 700] = np.float32(3.0)                       # one entry in the sixth split
+    h_bits = gen.f32_to_bf16_bits(h)
+    assert np.array_equal(gen.bf16_bits_to_f32(h_bits), h)   # the scaling is exact in bf16
+    head = qoh.PackedHead(*shape, comps)
+    assert head.forward_kernel(T) == kernel
+    y, tol = _oracle(comps, shape, h_bits)
+    lg, am = head.logits(_dev_hidden(h_bits))
+    lse, am2, ce = head.lse_argmax(_dev_hidden(h_bits), torch.from_numpy(targets))
+    check_logits(lg.cpu().numpy(), y, tol)
+    check_argmax(am.cpu().numpy(), y, tol)
+    check_argmax(am2.cpu().numpy(), y, tol)
+    check_lse_ce(lse.cpu().numpy(), ce.cpu().numpy(), y, tol, targets)
+    assert head.status(head.workspace(T)) == 0
+
+
 @pytest.mark.parametrize("T", [5, 24])   # decode kernel, tensor-core kernel
 def test_zero_and_extreme_magnitude_tokens(qoh, T):
     """Token 0 all zero (every logit exactly 0: argmax 0, LSE = log V), token 1
