@@ -262,6 +262,24 @@ ARCHEAD_API int archead_shard_partials(const archead_handle* handle, const uint1
 ARCHEAD_API int archead_merge_shards(const float* partials, int32_t n_shards, int32_t T, float* lse,
                                      int32_t* argmax, float* ce, archead_stream_t stream);
 
+/* Sampling across vocabulary shards (with archead_set_vocab_shard):
+ * archead_sample_partials: per token t, sample_partials[2t .. 2t+1] = (the
+ *   largest y[t,v] / temperature + G[t,v] over this shard's rows, the global
+ *   row of its first occurrence as int32 bits), G drawn for the global row v
+ *   exactly as archead_sample draws it, so a pick does not depend on how the
+ *   vocabulary is split.  sample_partials: device, 8-byte aligned, [T][2]
+ *   floats (also scratch for the call).  Same arguments, workspace and
+ *   stream rules as archead_sample otherwise.
+ * archead_merge_sample_shards: pairs of n_shards shards stacked
+ *   [n_shards][T][2] in increasing row order -> sampled[t], the first maximum
+ *   over all rows: the id archead_sample returns for the unsharded head.
+ *   Device pointers; no workspace. */
+ARCHEAD_API int archead_sample_partials(const archead_handle* handle, const uint16_t* hidden, int32_t T,
+                                        float temperature, uint64_t seed, uint64_t offset, float* sample_partials,
+                                        void* workspace, size_t workspace_bytes, archead_stream_t stream);
+ARCHEAD_API int archead_merge_sample_shards(const float* sample_partials, int32_t n_shards, int32_t T,
+                                            int32_t* sampled, archead_stream_t stream);
+
 /* Read (and with clear != 0, reset) the device status word of a workspace:
  * a bitwise OR of ARCHEAD_STATUS_* since the last clear.  Synchronises the
  * stream.  Returns ARCHEAD_ETIMEOUT if ARCHEAD_STATUS_WAIT_TIMEOUT is set. */

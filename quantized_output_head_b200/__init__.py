@@ -36,7 +36,7 @@ EXPORTED = (
     "archead_static_workspace_status", "archead_test_decode_waits", "archead_host_logits_workspace_bytes",
     "archead_logits_host",
     "archead_forward_kernel", "archead_set_vocab_shard", "archead_shard_partials", "archead_merge_shards",
-    "archead_sample",
+    "archead_sample", "archead_sample_partials", "archead_merge_sample_shards",
 )
 
 
@@ -74,6 +74,9 @@ _sig = {
                                       _vp, _vp, _sz, _vp]),
     "archead_shard_partials": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "archead_merge_shards": (ctypes.c_int, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "archead_sample_partials": (ctypes.c_int, [_vp, _vp, _i32, ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, _vp,
+                                               _vp, _sz, _vp]),
+    "archead_merge_sample_shards": (ctypes.c_int, [_vp, _i32, _i32, _vp, _vp]),
     "archead_test_decode_waits": (ctypes.c_int, [_vp, ctypes.c_uint64, ctypes.c_int]),
     "archead_free": (None, [_vp]),
     "archead_last_cuda_error": (ctypes.c_int, []),
@@ -329,6 +332,19 @@ class PackedHead:
                                            ws.data_ptr(), ws.numel(), _stream_ptr(None)), "archead_shard_partials")
         return out
 
+    def sample_partials(self, hidden: torch.Tensor, temperature: float, seed: int, offset: int = 0) -> torch.Tensor:
+        """This shard's share of a sampled draw: [T, 2] fp32 rows (the largest
+        y / temperature + G over its rows, the global row as int32 bits), the
+        noise of each global row as sample() draws it."""
+        _check_hidden(hidden, self.d)
+        T = int(hidden.shape[0])
+        out = torch.empty((T, 2), dtype=torch.float32, device=self.device)
+        ws = self.workspace(T)
+        _check(_lib.archead_sample_partials(self.handle, hidden.data_ptr(), T, float(temperature), int(seed),
+                                            int(offset), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(None)),
+               "archead_sample_partials")
+        return out
+
     def forward_kernel(self, T: int) -> str:
         """'decode' or 'tensor_core': the kernel a call with T tokens runs on."""
         k = _lib.archead_forward_kernel(self.handle, int(T))
@@ -388,8 +404,9 @@ def shard_components(comps: Dict[str, np.ndarray], v0: int, v1: int) -> Dict[str
 
 
 def gather_partials(parts: torch.Tensor, group=None) -> torch.Tensor:
-    """All-gather every rank's [T, 4] shard partials into [world, T, 4], in rank
-    order (the one cross-GPU exchange of a vocabulary-sharded head)."""
+    """All-gather every rank's shard partials ([T, 4] statistics or [T, 2]
+    sampling pairs) into [world, T, ...], in rank order (the one cross-GPU
+    exchange of a vocabulary-sharded head)."""
     import torch.distributed as dist
     world = dist.get_world_size(group)
     bufs = [torch.empty_like(parts) for _ in range(world)]
@@ -411,6 +428,20 @@ def merge_shards(parts: torch.Tensor):
         _check(_lib.archead_merge_shards(parts.data_ptr(), n, T, lse.data_ptr(), am.data_ptr(), ce.data_ptr(),
                                          _stream_ptr(None)), "archead_merge_shards")
     return lse, am, ce
+
+
+def merge_sample_shards(parts: torch.Tensor) -> torch.Tensor:
+    """Fold [n_shards, T, 2] sampling pairs (increasing row order) into the
+    sampled ids [T] int32: the draw of the unsharded head."""
+    if parts.dim() != 3 or parts.shape[2] != 2 or parts.dtype != torch.float32 or not parts.is_cuda:
+        raise ValueError("parts must be a [n_shards, T, 2] float32 CUDA tensor")
+    parts = parts.contiguous()
+    n, T = int(parts.shape[0]), int(parts.shape[1])
+    out = torch.empty(T, dtype=torch.int32, device=parts.device)
+    with torch.cuda.device(parts.device):
+        _check(_lib.archead_merge_sample_shards(parts.data_ptr(), n, T, out.data_ptr(), _stream_ptr(None)),
+               "archead_merge_sample_shards")
+    return out
 
 
 def _check_hidden(hidden: torch.Tensor, d: int) -> None:

@@ -15,6 +15,7 @@
 #include <mutex>
 #include <new>
 
+#include "device.cuh"
 #include "handle.h"
 
 namespace archead {
@@ -509,6 +510,74 @@ extern "C" ARCHEAD_API int archead_sample(const archead_handle* handle, const ui
   const SampleArgs sa{sampled, 1.f / temperature, seed, offset};
   return forward(handle, hidden, T, nullptr, nullptr, argmax, lse, nullptr, workspace, workspace_bytes,
                  reinterpret_cast<cudaStream_t>(stream), nullptr, &sa);
+}
+
+namespace archead {
+
+// Sampling across vocabulary shards.  The decode kernel leaves each block's
+// pick in the workspace (spart [T][grid]: the largest y / tau + G of the
+// block's rows, its global row); one warp per token folds them into this
+// shard's pair.  First maximum: pick_merge keeps the lower row on ties.
+__global__ void sample_partials_kernel(const float2* __restrict__ spart, int grid, int T, float2* __restrict__ out) {
+  const int t = static_cast<int>(blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32), lane = threadIdx.x & 31;
+  if (t >= T) return;
+  PickState b = pick_init();
+  for (int k = lane; k < grid; k += 32) {
+    const float2 q = spart[static_cast<size_t>(t) * grid + k];
+    b = pick_merge(b, PickState{q.x, __float_as_int(q.y)});
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) b = pick_merge(b, pick_shfl_xor(b, o));
+  if (lane == 0) out[t] = make_float2(b.z, __int_as_float(b.idx));
+}
+
+// Per token, the first maximum over n shards' pairs stacked in increasing row
+// order: the pick over all rows.
+__global__ void merge_sample_shards_kernel(const float2* __restrict__ parts, int n, int T,
+                                           int32_t* __restrict__ sampled) {
+  const int t = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+  if (t >= T) return;
+  PickState b = pick_init();
+  for (int r = 0; r < n; ++r) {
+    const float2 q = parts[static_cast<size_t>(r) * T + t];
+    b = pick_merge(b, PickState{q.x, __float_as_int(q.y)});
+  }
+  sampled[t] = b.idx;
+}
+
+}  // namespace archead
+
+extern "C" ARCHEAD_API int archead_sample_partials(const archead_handle* handle, const uint16_t* hidden,
+                                                   int32_t T, float temperature, uint64_t seed, uint64_t offset,
+                                                   float* sample_partials, void* workspace, size_t workspace_bytes,
+                                                   archead_stream_t stream) {
+  if (handle == nullptr || sample_partials == nullptr || !(temperature > 0.f) || !(temperature < INFINITY))
+    return ARCHEAD_EINVAL;
+  if (!aligned(sample_partials, 8)) return ARCHEAD_EALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // The kernel's own picks land in the first half of the output buffer, which
+  // the fold below then overwrites with the (value, row) pairs.
+  const SampleArgs sa{reinterpret_cast<int32_t*>(sample_partials), 1.f / temperature, seed, offset};
+  const int rc = forward(handle, hidden, T, nullptr, nullptr, nullptr, nullptr, nullptr, workspace, workspace_bytes,
+                         s, nullptr, &sa);
+  if (rc != ARCHEAD_OK) return rc;
+  const WsLayout w = ws_layout(*handle, T);
+  archead::sample_partials_kernel<<<(T + 7) / 8, 256, 0, s>>>(
+      reinterpret_cast<const float2*>(static_cast<const uint8_t*>(workspace) + w.spart), handle->grid, T,
+      reinterpret_cast<float2*>(sample_partials));
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
+}
+
+extern "C" ARCHEAD_API int archead_merge_sample_shards(const float* sample_partials, int32_t n_shards, int32_t T,
+                                                       int32_t* sampled, archead_stream_t stream) {
+  if (sample_partials == nullptr || sampled == nullptr || n_shards <= 0 || T <= 0 || T > kMaxTokens)
+    return ARCHEAD_EINVAL;
+  if (!aligned(sample_partials, 8) || !aligned(sampled, 4)) return ARCHEAD_EALIGN;
+  archead::merge_sample_shards_kernel<<<(T + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const float2*>(sample_partials), n_shards, T, sampled);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ARCHEAD_OK : set_cuda_error(e);
 }
 
 extern "C" ARCHEAD_API int archead_set_vocab_shard(archead_handle* handle, int32_t row_offset, int32_t vocab_total) {

@@ -196,6 +196,14 @@ def test_sampling_and_shard_calls_refuse_bad_arguments_on_the_host(qoh):
     assert L.archead_merge_shards(fake, 2, 0, fake, fake, fake, None) == qoh.ARCHEAD_EINVAL
     assert L.archead_merge_shards(fake, 2, 1, None, None, None, None) == qoh.ARCHEAD_EINVAL
     assert L.archead_merge_shards(fake + 4, 2, 1, fake, fake, fake, None) == qoh.ARCHEAD_EALIGN
+    for temp in (0.0, float("inf")):
+        assert L.archead_sample_partials(fake, fake, 1, temp, 1, 0, fake, fake, 1 << 20, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_sample_partials(fake, fake, 1, 1.0, 1, 0, None, fake, 1 << 20, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_sample_partials(fake, fake, 1, 1.0, 1, 0, fake + 4, fake, 1 << 20, None) == qoh.ARCHEAD_EALIGN
+    assert L.archead_merge_sample_shards(None, 2, 1, fake, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_merge_sample_shards(fake, 0, 1, fake, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_merge_sample_shards(fake, 2, 1, None, None) == qoh.ARCHEAD_EINVAL
+    assert L.archead_merge_sample_shards(fake + 4, 2, 1, fake, None) == qoh.ARCHEAD_EALIGN
     status = ct.c_uint32(0)
     assert L.archead_workspace_status(None, 0, None, ct.byref(status)) == qoh.ARCHEAD_EINVAL
     assert L.archead_workspace_status(fake + 16, 0, None, ct.byref(status)) == qoh.ARCHEAD_EALIGN

@@ -357,6 +357,33 @@ def test_sampling_matches_oracle(qoh, T):
     assert not torch.equal(a, b)                        # another counter range draws other noise
 
 
+@pytest.mark.parametrize("T", [5, 20])   # one and three decode launches
+def test_sampling_across_vocabulary_shards(qoh, T):
+    """Three vocabulary shards' sampling pairs, merged, draw exactly what the
+    unsharded head draws (the noise follows the global row); each shard's
+    pair is the best perturbed logit of its own rows."""
+    shape = (1000, 256, 32, 8, 64, 64)
+    comps = gen.random_components(gen.HeadShape(*shape), seed=88)
+    h_bits, _ = gen.random_hidden(256, T, seed=89, V=shape[0])
+    hd = _dev_hidden(h_bits)
+    whole = qoh.PackedHead(*shape, comps)
+    for temperature, seed, offset in ((0.7, 4242, 0), (1.3, 2**41 + 5, 2**35 + 1)):
+        want, _, _ = whole.sample(hd, temperature, seed, offset)
+        parts = []
+        for r in range(3):
+            v0, v1 = qoh.shard_rows(shape[0], 3, r)
+            head = qoh.PackedHead(v1 - v0, *shape[1:], qoh.shard_components(comps, v0, v1))
+            head.set_vocab_shard(v0, shape[0])
+            p = head.sample_partials(hd, temperature, seed, offset)
+            rows = p[:, 1].contiguous().view(torch.int32).cpu().numpy()
+            assert np.all((rows >= v0) & (rows < v1))
+            own, _, _ = head.sample(hd, temperature, seed, offset)
+            np.testing.assert_array_equal(rows, own.cpu().numpy())   # the shard's own draw over its rows
+            parts.append(p)
+        got = qoh.merge_sample_shards(torch.stack(parts))
+        assert torch.equal(got, want)
+
+
 def test_sampling_frequencies_follow_softmax(qoh):
     """One token repeated 16384 times over a 64-row head: chi-square of the GPU's
     draws against softmax(y / tau) of the oracle's logits."""

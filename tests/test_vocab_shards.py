@@ -68,19 +68,26 @@ def _rank_main(rank, world, port, out):
         import quantized_output_head_b200 as qoh
         T = 5
         mine = torch.full((T, 4), float(rank)) + torch.arange(T, dtype=torch.float32)[:, None]
-        out[rank] = qoh.gather_partials(mine).numpy()
+        # sampling pairs: (perturbed value, global row as int32 bits)
+        pairs = torch.stack([torch.full((T,), 10.0 * rank),
+                             torch.arange(T, dtype=torch.int32).add(100 * rank).view(torch.float32)], dim=1)
+        out[rank] = (qoh.gather_partials(mine).numpy(), qoh.gather_partials(pairs).numpy())
     finally:
         dist.destroy_process_group()
 
 
 def test_two_gloo_ranks_gather_partials_in_rank_order():
+    """Both kinds of shard partials (softmax statistics, sampling pairs) cross
+    the ranks bit for bit and in rank order."""
     world = 2
     with mp.Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
         res = dict(out)
     for rank in range(world):
-        g = res[rank]
-        assert g.shape == (world, 5, 4)
+        g, pr = res[rank]
+        assert g.shape == (world, 5, 4) and pr.shape == (world, 5, 2)
         for r in range(world):
             assert np.array_equal(g[r], np.full((5, 4), float(r)) + np.arange(5)[:, None])
+            assert np.array_equal(pr[r, :, 0], np.full(5, 10.0 * r))
+            assert np.array_equal(pr[r, :, 1].view(np.int32), np.arange(5) + 100 * r)
