@@ -51,6 +51,7 @@ FALLBACK_HBM_GBS = 6650.0
 CPU_SAMPLE_SECONDS = 12.0   # target length of the CPU-oracle sample behind cpu_baseline
 REFERENCE_SECONDS = 120.0   # target length of a whole --impl reference run
 FALLBACK_BF16_TFLOPS = 1590.0
+DATASHEET_BF16_TFLOPS = 2250.0   # B200 dense bf16, nominal (NVIDIA's figure halved: theirs assumes 2:4 sparsity)
 
 OPS = {  # config -> what one call produces
     2: dict(logits=True, argmax=True, lse=False, ce=False),
@@ -717,7 +718,10 @@ def main():
             roofline=dict(bound=bound, achieved=achieved, peak=peak, unit=unit, frac=achieved / peak,
                           traffic=traffic, kernel=f"archead::{PROFILE_STEM[kind]}", kernel_us=kernel_ms * 1e3,
                           algorithmic_bytes_per_launch=kbytes, algorithmic_flops_per_launch=kflops,
-                          peak_source=peak_src + (" (sustained bf16)" if bound == "tensor" else "")),
+                          peak_source=peak_src + ((" (sustained bf16)" if peak_src == "measured" else
+                                                   " (the pool's burst bf16 figure)") if bound == "tensor" else ""),
+                          **(dict(datasheet_peak=DATASHEET_BF16_TFLOPS, datasheet_frac=achieved / DATASHEET_BF16_TFLOPS)
+                             if bound == "tensor" else {})),
             call=dict(algorithmic_bytes=ab, algorithmic_flops=af, gbs=ab / (ms_per_step / 1e3) / 1e9,
                       hbm_frac=ab / (ms_per_step / 1e3) / 1e9 / hbm),
             cpu_baseline=cpu, parity=parity, e2e=e2e, clocks=clk.summary(),
