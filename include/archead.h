@@ -133,9 +133,10 @@ ARCHEAD_API int archead_forward_kernel(const archead_handle* handle, int32_t T);
 /* Workspace bytes one forward call with T tokens needs (256-byte aligned
  * scratch, caller-owned; reused across calls on one stream).  Holds the
  * low-rank prologue output z (decode kernel) or the fp16 activation operand
- * [h | z] (tensor-core kernel), per-block log-sum-exp partials, a completion
- * counter and the status word.  Zero-fill a workspace once before its first
- * use (the status word is sticky); afterwards the calls keep it consistent.
+ * [h | z] (tensor-core kernel), per-block log-sum-exp partials, completion
+ * tickets and the status word.  Zero-fill a workspace once before its first
+ * use (the status word is sticky; every ticket is back at zero when a call
+ * ends); afterwards the calls keep it consistent.
  * Calls that share a workspace must be ordered (same stream).  0 if handle is
  * null or T <= 0. */
 ARCHEAD_API size_t archead_workspace_bytes(const archead_handle* handle, int32_t T);
