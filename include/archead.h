@@ -167,10 +167,13 @@ ARCHEAD_API int archead_logits_lse_argmax(const archead_handle* handle, const ui
  * are HOST pointers (pinned memory recommended), copied to the device inside
  * the workspace; lse / argmax / ce are HOST pointers filled before return.
  * workspace must be >= archead_host_workspace_bytes(handle, T).  Synchronises
- * the stream.  When every host buffer is pinned, the call's fixed sequence
- * (copies in, the forward launches, copies out) is captured once per distinct
- * set of arguments (the last four are kept per handle) and replayed with one
- * graph launch; otherwise, or if the capture fails, it runs directly. */
+ * the stream.  An output in pinned (page-locked, device-mapped) host memory is
+ * written there by the kernels, with no copy after them; outputs in pageable
+ * memory go through the workspace and a device-to-host copy.  When every host buffer is
+ * pinned, the call's fixed sequence (copies in, the forward launches, any
+ * copies out) is captured once per distinct set of arguments (the last four
+ * are kept per handle) and replayed with one graph launch; otherwise, or if
+ * the capture fails, it runs directly. */
 ARCHEAD_API size_t archead_host_workspace_bytes(const archead_handle* handle, int32_t T);
 ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint16_t* hidden_host,
                                         int32_t T, const int32_t* targets_host, float* lse_host,
@@ -182,9 +185,11 @@ ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint
  * logits [T, V] fp32 and argmax [T] int32 are HOST pointers filled before
  * return (either may be NULL, not both).  workspace (device, 256-byte
  * aligned) must be >= archead_host_logits_workspace_bytes(handle, T): it
- * stages the hidden states and the logits on the device.  Synchronises the
- * stream.  Pinned host buffers take the captured sequence as
- * archead_lse_argmax_host does. */
+ * stages the hidden states and the logits on the device (the logits always
+ * reach the host by one copy: the kernels' scattered stores into host memory
+ * measured twice as slow).  Synchronises the stream.  A pinned argmax is
+ * written by the kernels and pinned buffers take the captured sequence, as in
+ * archead_lse_argmax_host. */
 ARCHEAD_API size_t archead_host_logits_workspace_bytes(const archead_handle* handle, int32_t T);
 ARCHEAD_API int archead_logits_host(const archead_handle* handle, const uint16_t* hidden_host, int32_t T,
                                     float* logits_host, int32_t* argmax_host, void* workspace,
