@@ -185,9 +185,8 @@ ARCHEAD_API int archead_lse_argmax_host(const archead_handle* handle, const uint
  * logits [T, V] fp32 and argmax [T] int32 are HOST pointers filled before
  * return (either may be NULL, not both).  workspace (device, 256-byte
  * aligned) must be >= archead_host_logits_workspace_bytes(handle, T): it
- * stages the hidden states and the logits on the device (the logits always
- * reach the host by one copy: the kernels' scattered stores into host memory
- * measured twice as slow).  Synchronises the stream.  A pinned argmax is
+ * stages the hidden states (and logits bound for pageable memory) on the
+ * device.  Synchronises the stream.  Pinned outputs, the logits included, are
  * written by the kernels and pinned buffers take the captured sequence, as in
  * archead_lse_argmax_host. */
 ARCHEAD_API size_t archead_host_logits_workspace_bytes(const archead_handle* handle, int32_t T);

@@ -767,13 +767,22 @@ __device__ void epilogue_warp(const DecodeParams& p, const SmemView& sv, int n_m
       }
       if (v < p.V) {
         lse_push(st, y0, v);
-        if (p.logits != nullptr) p.logits[static_cast<size_t>(p.t0 + t) * p.V + v] = y0;
         if (v == target) p.tgt[p.t0 + t] = y0;
       }
       if (v + 1 < p.V) {
         lse_push(st, y1, v + 1);
-        if (p.logits != nullptr) p.logits[static_cast<size_t>(p.t0 + t) * p.V + v + 1] = y1;
         if (v + 1 == target) p.tgt[p.t0 + t] = y1;
+      }
+      if (p.logits != nullptr && v < p.V) {
+        // The row pair in one 8-byte store where it is aligned (a warp then
+        // writes 256 contiguous bytes, also when the logits live in host memory).
+        float* dst = p.logits + static_cast<size_t>(p.t0 + t) * p.V + v;
+        if (v + 1 < p.V && (reinterpret_cast<uintptr_t>(dst) & 7u) == 0) {
+          *reinterpret_cast<float2*>(dst) = make_float2(y0, y1);
+        } else {
+          dst[0] = y0;
+          if (v + 1 < p.V) dst[1] = y1;
+        }
       }
     }
     __syncwarp();
