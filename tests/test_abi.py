@@ -209,6 +209,25 @@ def test_sampling_and_shard_calls_refuse_bad_arguments_on_the_host(qoh):
     assert L.archead_workspace_status(fake + 16, 0, None, ct.byref(status)) == qoh.ARCHEAD_EALIGN
 
 
+def test_builder_svd_options_are_checked_first(qoh):
+    """Bad randomised-SVD options: the binding refuses an unknown method, and
+    the library returns EINVAL before it touches a pointer or the GPU."""
+    import ctypes as ct
+    import quantized_output_head_b200.builder as bld
+    with pytest.raises(ValueError):
+        bld.svd_opts("approximate")
+    fake = 4096                                   # never dereferenced: the option check fails first
+    desc = bld._desc(1024, 256, 32, 8, 64, 64)
+    comps = bld.ArcheadDeviceComponents(*([fake] * 10))
+    for method, oversample, iters in ((7, 8, 2), (bld.ARCHEAD_SVD_RANDOMIZED, -1, 2),
+                                      (bld.ARCHEAD_SVD_RANDOMIZED, 8, 65)):
+        opts = bld.ArcheadSvdOpts(method, oversample, iters, 1)
+        assert bld._blib.archead_build_head_svd(ct.byref(desc), fake, fake, 16, 0.01, 0.75, ct.byref(opts),
+                                                ct.byref(comps), fake, 1 << 20, None) == qoh.ARCHEAD_EINVAL
+        assert bld._blib.archead_build_correction_svd(ct.byref(desc), fake, fake, fake, ct.byref(opts), fake, fake,
+                                                      fake, fake, fake, 1 << 20, None) == qoh.ARCHEAD_EINVAL
+
+
 def test_builder_binding_refuses_host_or_wrongly_typed_tensors(qoh):
     """The construction binding checks its tensors before it calls the library."""
     import torch

@@ -59,3 +59,20 @@ def test_oracle_call_model_splits_fixed_and_per_row_time():
     comps, h_bits, _, _ = _case(T=1)
     t_fixed, t_row = bench.oracle_call_model(oracle, comps, SHAPE, h_bits, small=256, large=2048)
     assert t_fixed >= 0.0 and t_row > 0.0
+
+
+def test_randomized_build_flops_add_the_sketch_products():
+    """The randomised SVD's sketch is r + oversample columns, rounded up to a
+    multiple of 64 above 64 and capped at d; each factorisation adds
+    power_iters + 2 products G Q (2 d^2 k flops each) and two d x k x k ones."""
+    assert bench.sketch_cols(4096, 512, 32) == 576
+    assert bench.sketch_cols(4096, 64, 32) == 128
+    assert bench.sketch_cols(256, 8, 0) == 8
+    assert bench.sketch_cols(256, 240, 64) == 256
+    V, d, r_c, r_r, N = 151936, 4096, 512, 64, 16384
+    exact = bench.build_flops(V, d, r_c, r_r, N)
+    rand = bench.build_flops(V, d, r_c, r_r, N, svd="randomized", oversample=32, power_iters=2)
+    extra = sum(2 * d * d * k * 4 + 4 * d * k * k for k in (576, 128))
+    assert rand - exact == extra
+    # the default bench line: ~8.02 TFLOP of dense products
+    assert abs(rand / 1e12 - 8.02) < 0.01
